@@ -1,0 +1,298 @@
+/*
+ * bitlinear_oracle.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, CPU statement of the BitNet b1.58 BitLinear product, used to
+ * check the CUDA library.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load it; the product path never does.  It
+ * shares no code, header, table or constant generator with the CUDA sources.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [GUIDE]  "How to Run BitNet Inference on GPU Using CUDA Kernels: A Complete
+ *            Guide", section "Understanding the Two-Phase Architecture"
+ *            (BitLinearKernel quantises inputs to INT8 with scaling factors and
+ *            calls an INT8 x INT2 linear) and FAQ "Can I use the CUDA kernel for
+ *            models other than the default BitNet architecture?" (generic
+ *            INT8xINT2 GEMM).
+ *   [FLOOR]  "bit-floor" README, section "The core math" (binary GEMV as
+ *            XNOR/popcount, "no floating point until the final scale multiply")
+ *            and section "What's inside" (absmax scale for binary weights,
+ *            mean-abs scale for ternary weights).
+ *   [BITC]   "BitCompute: 1.58-bit LLM Execution Engine", sections "Features"
+ *            (multiplying by -1, 0, +1 is add / subtract / skip) and "Future
+ *            Roadmap" (four 1.58-bit weights packed into one byte).
+ *   [BLOG]   "Run 100B Models on Your Laptop CPU: Microsoft BitNet Exposed",
+ *            section "What is Microsoft BitNet?" (ternary {-1, 0, +1} weights).
+ *
+ * The pages give no formula for the scales; the readings used here are:
+ *   weight scale    gamma = mean |W| over the whole tensor, summed in fp64 in a
+ *                   fixed order (row by row, k ascending inside a row, rows in
+ *                   ascending order), rounded once to fp32, then
+ *                   gamma_eff = max(gamma, 1e-5).
+ *   ternary code    code = clamp(rint(w / gamma_eff), -1, 1), fp32 division,
+ *                   round half to even.
+ *   activation      per token: a = max(max_k |x|, 1e-5); s = 127 / a (fp32);
+ *                   q = clamp(rint(x * s), -128, 127) (fp32 product, round half
+ *                   to even); d = a / 127 (fp32); r = sum_k q.
+ *   product         acc[m][n] = sum_k code[n][k] * q[m][k], exact integer.
+ *   rescale         y = ((float)acc * d[m]) * gamma_eff: two fp32 products in
+ *                   that order, no fused multiply-add; bf16 output rounds y to
+ *                   nearest even.
+ *   binary          bit = (v < 0); acc = 2 * popcount(XNOR(Wb, xb)) - K;
+ *                   y = (float)acc * (s_w * s_x) with s_w = max |W| over the
+ *                   tensor and s_x = max |x| over the token.
+ * Floating-point decisions that produce integers (codes, q) are taken in fp32,
+ * the precision the kernels use, so that both sides decide identically.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC.
+ * Parity of the fp64 weight-scale sum is exact by construction because the
+ * order of additions is part of the definition above.
+ */
+#include <stdint.h>
+#include <string.h>
+#include <math.h>
+
+#define ORACLE_EPS 1e-5f
+#define ORACLE_QB 127.0f
+
+/* ---------------------------------------------------------------------------
+ * Weight scale (absmean).  [FLOOR] "What's inside": mean-abs scale for ternary
+ * weights; [BLOG] "What is Microsoft BitNet?": ternary weights.
+ * ------------------------------------------------------------------------- */
+float oracle_weight_scale(const float *W, int64_t N, int64_t K)
+{
+    double S = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+        double row = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+            row += fabs((double)W[n * K + k]);
+        S += row;
+    }
+    float gamma = (float)(S / (double)(N * K));
+    return gamma > ORACLE_EPS ? gamma : ORACLE_EPS;
+}
+
+/* Ternary round-clip: code = clamp(rint(w / gamma_eff), -1, 1). */
+void oracle_ternary_codes(const float *W, int64_t N, int64_t K, float gamma_eff,
+                          int8_t *codes)
+{
+    for (int64_t i = 0; i < N * K; ++i) {
+        float r = W[i] / gamma_eff;
+        float t = rintf(r);
+        int8_t c = 0;
+        if (t >= 1.0f)
+            c = 1;
+        else if (t <= -1.0f)
+            c = -1;
+        codes[i] = c;
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Packed layout "TL" (the pages fix none: [BITC] "Future Roadmap" packs four
+ * weights per byte; [GUIDE] names an INT2 layout without describing it).
+ *
+ *   stored value  s = code + 1 in {0, 1, 2}; 3 is never written
+ *   rows          padded up to a multiple of 8 with code 0 (s = 1)
+ *   K             a multiple of 64
+ *   byte offset   of (n, k):  ((g * (K/64) + c) * 8 + r) * 16 + w * 4 + j
+ *                 with g = n/8, r = n%8, c = k/64, w = (k%64)/16, j = k%4
+ *   bit offset    2 * i with i = (k%16)/4
+ * So a 16-byte chunk holds 64 consecutive k of one row, and the eight rows of
+ * a row group are adjacent for each chunk.
+ * ------------------------------------------------------------------------- */
+int64_t oracle_packed_bytes(int64_t N, int64_t K)
+{
+    int64_t Np = (N + 7) / 8 * 8;
+    return Np * (K / 4);
+}
+
+static int64_t tl_byte(int64_t n, int64_t k, int64_t K)
+{
+    int64_t g = n / 8, r = n % 8, c = k / 64;
+    int64_t w = (k % 64) / 16, j = k % 4;
+    return ((g * (K / 64) + c) * 8 + r) * 16 + w * 4 + j;
+}
+
+static int tl_shift(int64_t k)
+{
+    return (int)(2 * ((k % 16) / 4));
+}
+
+void oracle_pack(const int8_t *codes, int64_t N, int64_t K, uint8_t *packed)
+{
+    int64_t Np = (N + 7) / 8 * 8;
+    memset(packed, 0, (size_t)oracle_packed_bytes(N, K));
+    for (int64_t n = 0; n < Np; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            int code = n < N ? codes[n * K + k] : 0;
+            unsigned s = (unsigned)(code + 1);
+            packed[tl_byte(n, k, K)] |= (uint8_t)(s << tl_shift(k));
+        }
+}
+
+void oracle_unpack(const uint8_t *packed, int64_t N, int64_t K, int8_t *codes)
+{
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            unsigned s = (packed[tl_byte(n, k, K)] >> tl_shift(k)) & 3u;
+            codes[n * K + k] = (int8_t)((int)s - 1);
+        }
+}
+
+/* ---------------------------------------------------------------------------
+ * Per-token absmax int8 activation quantisation.  [GUIDE] "Understanding the
+ * Two-Phase Architecture": inputs quantised to INT8 with scaling factors.  The
+ * page says "per-batch"; the reading here is per token (identical at M = 1).
+ * ------------------------------------------------------------------------- */
+void oracle_quantize_act(const float *x, int64_t M, int64_t K, int8_t *q,
+                         float *d, int32_t *rowsum)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        const float *xm = x + m * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(xm[k]);
+            if (a > amax)
+                amax = a;
+        }
+        float a_eff = amax > ORACLE_EPS ? amax : ORACLE_EPS;
+        float s = ORACLE_QB / a_eff;
+        int32_t r = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = xm[k] * s;
+            float t = rintf(v);
+            if (t > 127.0f)
+                t = 127.0f;
+            if (t < -128.0f)
+                t = -128.0f;
+            int8_t qi = (int8_t)t;
+            q[m * K + k] = qi;
+            r += qi;
+        }
+        d[m] = a_eff / ORACLE_QB;
+        rowsum[m] = r;
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Ternary product with exact integer accumulation.  [BITC] "Features": a
+ * product with -1 / 0 / +1 is subtract / skip / add.  [GUIDE] FAQ: an
+ * INT8 x INT2 GEMM.  Accumulated in int64 and narrowed (|acc| <= 128 * K).
+ * ------------------------------------------------------------------------- */
+void oracle_ternary_acc(const int8_t *codes, const int8_t *q, int64_t M,
+                        int64_t N, int64_t K, int32_t *acc)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        const int8_t *wn = codes + n * K;
+        for (int64_t m = 0; m < M; ++m) {
+            const int8_t *qm = q + m * K;
+            int64_t s = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                if (wn[k] == 1)
+                    s += qm[k];
+                else if (wn[k] == -1)
+                    s -= qm[k];
+            }
+            acc[m * N + n] = (int32_t)s;
+        }
+    }
+}
+
+/* Rescale: y = ((float)acc * d[m]) * gamma_eff.  [FLOOR] "The core math": no
+ * floating point until the final scale multiply. */
+void oracle_rescale(const int32_t *acc, const float *d, float gamma_eff,
+                    int64_t M, int64_t N, float *y)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float a = (float)acc[m * N + n];
+            float t = a * d[m];
+            y[m * N + n] = t * gamma_eff;
+        }
+}
+
+/* fp32 -> bf16, round to nearest even; NaN stays NaN. */
+void oracle_to_bf16(const float *y, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        uint32_t u;
+        memcpy(&u, &y[i], 4);
+        if ((u & 0x7fffffffu) > 0x7f800000u) {
+            out[i] = (uint16_t)((u >> 16) | 0x40u);
+        } else {
+            uint32_t lsb = (u >> 16) & 1u;
+            u += 0x7fffu + lsb;
+            out[i] = (uint16_t)(u >> 16);
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Binary 1-bit variant.  [FLOOR] "The core math": rows packed into ceil(K/64)
+ * 64-bit words, y = scale_w * scale_x * (2 * POPCNT(XNOR(W, x)) - K);
+ * [FLOOR] "What's inside": absmax scale for binary weights.
+ * Bit j of word w holds k = 64 w + j; the bit is 1 when the value is negative.
+ * Pad bits (K not a multiple of 64) are 0 in W and 1 in x, so XNOR is 0 there.
+ * ------------------------------------------------------------------------- */
+float oracle_absmax(const float *v, int64_t n)
+{
+    float a = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float t = fabsf(v[i]);
+        if (t > a)
+            a = t;
+    }
+    return a;
+}
+
+void oracle_binary_signs(const float *v, int64_t R, int64_t K, int pad_bit,
+                         uint64_t *out)
+{
+    int64_t words = (K + 63) / 64;
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t w = 0; w < words; ++w) {
+            uint64_t word = 0;
+            for (int64_t j = 0; j < 64; ++j) {
+                int64_t k = 64 * w + j;
+                uint64_t bit;
+                if (k < K)
+                    bit = v[r * K + k] < 0.0f ? 1u : 0u;
+                else
+                    bit = (uint64_t)pad_bit;
+                word |= bit << j;
+            }
+            out[r * words + w] = word;
+        }
+}
+
+static int64_t popcount64_plain(uint64_t v)
+{
+    int64_t c = 0;
+    while (v) {
+        c += (int64_t)(v & 1u);
+        v >>= 1;
+    }
+    return c;
+}
+
+void oracle_binary_acc(const uint64_t *Wb, const uint64_t *xb, int64_t N,
+                       int64_t K, int32_t *acc)
+{
+    int64_t words = (K + 63) / 64;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        int64_t pc = 0;
+        for (int64_t w = 0; w < words; ++w)
+            pc += popcount64_plain(~(Wb[n * words + w] ^ xb[w]));
+        acc[n] = (int32_t)(2 * pc - K);
+    }
+}
+
+void oracle_binary_rescale(const int32_t *acc, float s_w, float s_x, int64_t N,
+                           float *y)
+{
+    float s = s_w * s_x;
+    for (int64_t n = 0; n < N; ++n)
+        y[n] = (float)acc[n] * s;
+}

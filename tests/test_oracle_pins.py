@@ -1,0 +1,290 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each test ties one oracle function to a hand-worked example, a closed form, a
+library routine on a special case, a brute-force computation or an invariant,
+chosen so that a plausible slip (a dropped term, a wrong sign, a transposed
+operand, round-half-away instead of half-even, 128 instead of 127, a per-batch
+instead of a per-token scale, a shuffled bit layout) fails at least one test.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs as si
+
+
+def _f32(a):
+    return np.asarray(a, dtype=np.float32)
+
+
+# ---------------------------------------------------------------- hand-worked
+
+def test_hand_worked_4x4(golden):
+    g = golden("hand_4x4.json")
+    W = _f32(g["W"])
+    x = _f32(g["x"])
+    out = oracle.bitlinear(x, W)
+    assert out["gamma"] == pytest.approx(g["gamma"], rel=1e-6)
+    np.testing.assert_array_equal(out["codes"], np.array(g["codes"], np.int8))
+    np.testing.assert_array_equal(out["q"], np.array(g["q"], np.int8))
+    np.testing.assert_array_equal(out["rowsum"], np.array(g["rowsum"], np.int32))
+    np.testing.assert_array_equal(out["acc"], np.array(g["acc"], np.int32))
+    np.testing.assert_allclose(out["d"], np.array(g["d"]), rtol=1e-6)
+    np.testing.assert_allclose(out["y"], np.array(g["y"]), rtol=1e-5, atol=1e-9)
+
+
+# ---------------------------------------------------------------- rounding ties
+
+def test_code_ties_round_half_even():
+    # sum|W| = 4, N*K = 4 -> gamma = 1 exactly; W/gamma = [0.5, -0.5, 1, 2].
+    W = _f32([[0.5, -0.5, 1.0, 2.0]])
+    g = oracle.weight_scale(W)
+    assert g == np.float32(1.0)
+    # half-even: 0.5 -> 0, -0.5 -> 0; 2 clips to 1.  Half-away would give +-1.
+    np.testing.assert_array_equal(oracle.ternary_codes(W, g), [[0, 0, 1, 1]])
+
+
+def test_activation_ties_round_half_even():
+    # amax = 127 -> s = 1 exactly, so x*s = x.
+    x = _f32([[1.5, -1.5, 2.5, -2.5, 0.5, -0.5, 127.0, 0.0]])
+    q, d, r = oracle.quantize_act(x)
+    np.testing.assert_array_equal(q, [[2, -2, 2, -2, 0, 0, 127, 0]])
+    assert d[0] == np.float32(1.0)
+    assert r[0] == 127
+
+
+# ---------------------------------------------------------------- closed forms
+
+def test_weight_scale_closed_forms():
+    rng = np.random.default_rng(1)
+    # every |w| = 0.25 -> mean |W| = 0.25 exactly whatever the signs
+    W = _f32(np.where(rng.random((37, 128)) < 0.5, -0.25, 0.25))
+    assert oracle.weight_scale(W) == np.float32(0.25)
+    # scaling by a power of two scales gamma exactly and keeps the codes
+    W = _f32(rng.standard_normal((64, 192)) * 0.02)
+    g = oracle.weight_scale(W)
+    assert oracle.weight_scale(W * 4) == g * 4
+    np.testing.assert_array_equal(oracle.ternary_codes(W, g),
+                                  oracle.ternary_codes(W * 4, g * 4))
+    # all-zero weights: gamma clamps to 1e-5 and every code is 0
+    Z = np.zeros((8, 64), np.float32)
+    assert oracle.weight_scale(Z) == np.float32(1e-5)
+    assert not oracle.ternary_codes(Z, oracle.weight_scale(Z)).any()
+    # mean|W| of a large Gaussian sample is sigma * sqrt(2/pi)
+    W = si.weight(1024, 1024, seed=3).numpy()
+    sigma = 0.02
+    expect = sigma * math.sqrt(2 / math.pi)
+    # std of the mean of |z| over n draws: sigma*sqrt(1-2/pi)/sqrt(n)
+    tol = 6 * sigma * math.sqrt(1 - 2 / math.pi) / 1024
+    assert abs(float(oracle.weight_scale(W)) - expect) < tol
+    # fp64 sum: mean of values that fp32 cannot accumulate exactly
+    W = np.full((4096, 4096), np.float32(0.1), np.float32)
+    W[0, 0] = np.float32(1e4)
+    S = 4096 * 4096 * 0.1 + 1e4 - 0.1
+    expect = np.float32(S / (4096 * 4096))
+    assert abs(float(oracle.weight_scale(W)) - float(expect)) <= float(np.spacing(expect))
+
+
+def test_gaussian_zero_fraction():
+    # code 0 iff |w| < gamma/2 = sigma*sqrt(2/pi)/2 -> P = erf(sqrt(2/pi)/(2*sqrt(2)))
+    W = si.weight(1024, 1024, seed=5).numpy()
+    codes = oracle.ternary_codes(W, oracle.weight_scale(W))
+    p = math.erf(math.sqrt(2 / math.pi) / (2 * math.sqrt(2)))
+    assert abs(p - 0.3101) < 1e-4
+    frac = float((codes == 0).mean())
+    sd = math.sqrt(p * (1 - p) / codes.size)
+    assert abs(frac - p) < 5 * sd
+    # the +1 and -1 codes are equally likely by symmetry
+    pos, neg = (codes == 1).mean(), (codes == -1).mean()
+    assert abs(pos - neg) < 5 * math.sqrt(0.35 * 0.65 / codes.size) * 2
+
+
+# ---------------------------------------------------------------- quantiser bounds
+
+@pytest.mark.parametrize("M,K", [(1, 64), (3, 256), (16, 2560)])
+def test_activation_quant_properties(M, K):
+    x = si.activations(M, K, seed=7, dtype=torch.float32).numpy()
+    q, d, r = oracle.quantize_act(x)
+    amax = np.abs(x).max(axis=1)
+    # scale: d = amax / 127 per token (not per batch, not /128)
+    np.testing.assert_allclose(d, amax / 127.0, rtol=2e-7)
+    # the largest |x| of each token lands on +-127; all |q| <= 127
+    assert np.abs(q).max() <= 127
+    for m in range(M):
+        i = np.argmax(np.abs(x[m]))
+        assert abs(int(q[m, i])) == 127
+    # round-to-nearest error bound: |x - q*d| <= d/2 (plus fp32 slack)
+    err = np.abs(x - q.astype(np.float64) * d[:, None].astype(np.float64))
+    assert (err <= d[:, None] * (0.5 + 1e-5)).all()
+    # monotone in x within a token
+    for m in range(M):
+        o = np.argsort(x[m], kind="stable")
+        assert (np.diff(q[m, o].astype(np.int32)) >= 0).all()
+    # row sums
+    np.testing.assert_array_equal(r, q.astype(np.int64).sum(axis=1))
+    # scaling a token by a power of two keeps q and scales d exactly
+    q2, d2, r2 = oracle.quantize_act(x * 2)
+    np.testing.assert_array_equal(q2, q)
+    np.testing.assert_array_equal(d2, d * 2)
+
+
+def test_zero_token():
+    x = np.zeros((2, 128), np.float32)
+    x[1, 5] = -3.0
+    q, d, r = oracle.quantize_act(x)
+    assert not q[0].any() and r[0] == 0
+    assert d[0] == np.float32(np.float32(1e-5) / np.float32(127.0))
+    assert q[1, 5] == -127 and r[1] == -127
+
+
+def test_codes_round_clip_bound():
+    W = si.weight(64, 256, seed=11).numpy()
+    g = oracle.weight_scale(W)
+    c = oracle.ternary_codes(W, g)
+    assert set(np.unique(c)).issubset({-1, 0, 1})
+    r = W.astype(np.float64) / float(g)
+    inner = np.abs(r) < 1.4999
+    # inside the clip range the code is the nearest integer
+    assert (np.abs(r[inner] - c[inner]) <= 0.5 + 1e-6).all()
+    # outside it the code carries the sign
+    outer = np.abs(r) > 1.5001
+    assert (c[outer] == np.sign(r[outer])).all()
+
+
+# ---------------------------------------------------------------- product + rescale
+
+@pytest.mark.parametrize("seed", range(6))
+def test_bruteforce_fp64_matmul(seed):
+    rng = np.random.default_rng(100 + seed)
+    M = int(rng.integers(1, 17))
+    N = int(rng.integers(1, 33))
+    K = 64 * int(rng.integers(1, 4))
+    W = si.weight(N, K, seed=seed).numpy()
+    x = si.activations(M, K, seed=seed, dtype=torch.float32).numpy()
+    out = oracle.bitlinear(x, W)
+    # dequantised operands multiplied in fp64 by numpy (the closed form
+    # y = (q d) (codes gamma)^T), against the oracle's integer-then-scale path
+    Xd = out["q"].astype(np.float64) * out["d"].astype(np.float64)[:, None]
+    Wd = out["codes"].astype(np.float64) * float(out["gamma"])
+    ref = Xd @ Wd.T
+    np.testing.assert_array_equal(
+        out["acc"], (out["q"].astype(np.int64) @ out["codes"].astype(np.int64).T))
+    y = out["y"].astype(np.float64)
+    tol = 2.5e-7 * np.abs(ref) + 1e-30
+    assert (np.abs(y - ref) <= tol).all()
+
+
+def test_rowsum_identity_and_bounds():
+    W = si.weight(40, 512, seed=2).numpy()
+    x = si.activations(5, 512, seed=2, dtype=torch.float32).numpy()
+    out = oracle.bitlinear(x, W)
+    stored = out["codes"].astype(np.int64) + 1
+    lhs = out["q"].astype(np.int64) @ stored.T - out["rowsum"][:, None]
+    np.testing.assert_array_equal(lhs, out["acc"])
+    assert np.abs(out["acc"]).max() <= 127 * 512
+
+
+def test_permutation_invariance():
+    rng = np.random.default_rng(9)
+    W = si.weight(16, 320, seed=4).numpy()
+    x = si.activations(3, 320, seed=4, dtype=torch.float32).numpy()
+    p = rng.permutation(320)
+    a = oracle.bitlinear(x, W)
+    b = oracle.bitlinear(x[:, p], W[:, p])
+    np.testing.assert_array_equal(a["acc"], b["acc"])
+    np.testing.assert_array_equal(a["y"], b["y"])
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal(4096).astype(np.float32) * 10
+    # exact ties between two bf16 values, both parities of the kept bit
+    ties = np.array([0x3F808000, 0x3F818000, 0xBF808000, 0x40498000],
+                    np.uint32).view(np.float32)
+    v = np.concatenate([v, ties, np.float32([0.0, -0.0, 1e-40, 3.4e38])])
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle.to_bf16_bits(v), ref)
+
+
+# ---------------------------------------------------------------- packed layout
+
+def _codes_from_rule(case):
+    N, K = case["N"], case["K"]
+    c = np.zeros((N, K), np.int8)
+    for row, ks, val in case["set"]:
+        if ks == "all":
+            c[row, :] = val
+        else:
+            c[row, ks] = val
+    return c
+
+
+def test_layout_hand_fixtures(golden):
+    g = golden("tl_layout.json")
+    for case in g["cases"]:
+        codes = _codes_from_rule(case)
+        packed = oracle.pack(codes)
+        assert packed.size == case["total_bytes"]
+        expect = np.full(case["total_bytes"], case["fill"], np.uint8)
+        for off, val in case["bytes"].items():
+            expect[int(off)] = val
+        np.testing.assert_array_equal(packed, expect)
+        np.testing.assert_array_equal(oracle.unpack(packed, case["N"], case["K"]), codes)
+
+
+@pytest.mark.parametrize("N,K", [(1, 64), (8, 128), (13, 256), (40, 2560)])
+def test_pack_roundtrip_and_padding(N, K):
+    rng = np.random.default_rng(N * 1000 + K)
+    codes = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    packed = oracle.pack(codes)
+    assert packed.size == ((N + 7) // 8) * 8 * K // 4
+    np.testing.assert_array_equal(oracle.unpack(packed, N, K), codes)
+    # no byte holds the unused value 3 in any 2-bit field
+    fields = np.stack([(packed >> s) & 3 for s in (0, 2, 4, 6)])
+    assert (fields != 3).all()
+
+
+def test_packed_words_are_dp4a_ready():
+    # (word >> 2i) & 0x03030303 yields the stored codes of four consecutive k
+    rng = np.random.default_rng(21)
+    N, K = 16, 256
+    codes = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    words = oracle.pack(codes).view("<u4")
+    for n in (0, 5, 8, 15):
+        for k0 in range(0, K, 16):
+            g, r, c, w = n // 8, n % 8, k0 // 64, (k0 % 64) // 16
+            word = int(words[((g * (K // 64) + c) * 8 + r) * 4 + w])
+            for i in range(4):
+                v = (word >> (2 * i)) & 0x03030303
+                got = [(v >> (8 * j)) & 0xFF for j in range(4)]
+                want = [int(codes[n, k0 + 4 * i + j]) + 1 for j in range(4)]
+                assert got == want
+
+
+# ---------------------------------------------------------------- binary variant
+
+@pytest.mark.parametrize("N,K", [(1, 64), (7, 100), (33, 512), (64, 8192)])
+def test_xnor_popcount_identity(N, K):
+    W = si.weight(N, K, seed=N + K).numpy()
+    x = si.activations(1, K, seed=N + K, dtype=torch.float32).numpy()
+    W[0, 0] = -0.0  # sign bit set, but not < 0: counts as +1
+    out = oracle.binary_gemv(W, x)
+    sw = np.where(W < 0, -1, 1).astype(np.int64)
+    sx = np.where(x[0] < 0, -1, 1).astype(np.int64)
+    np.testing.assert_array_equal(out["acc"], sw @ sx)
+    assert out["s_w"] == np.abs(W).max() and out["s_x"] == np.abs(x).max()
+    ref = (sw @ sx).astype(np.float64) * float(out["s_w"]) * float(out["s_x"])
+    assert (np.abs(out["y"] - ref) <= 2.5e-7 * np.abs(ref) + 1e-30).all()
+
+
+def test_binary_bit_order():
+    # bit j of word w <-> k = 64 w + j, bit set for negative values
+    v = np.ones((1, 128), np.float32)
+    v[0, 3] = -1
+    v[0, 64 + 60] = -2
+    b = oracle.binary_signs(v)
+    assert b.shape == (1, 2)
+    assert int(b[0, 0]) == 1 << 3 and int(b[0, 1]) == 1 << 60
