@@ -1,0 +1,258 @@
+"""BitNet b1.58 BitLinear product on B200 (sm_100a): thin ctypes binding.
+
+Every function here only checks and marshals torch tensors (device pointers,
+sizes, dtypes and the current CUDA stream) into the C ABI of
+``libbitlinear.so`` declared in ``include/bitlinear.h``; all arithmetic runs in
+the library's CUDA kernels.  There is no CPU fallback: importing this package
+fails if the library has not been built (``python -m
+bit_ternary_weight_b200.build``), and every call raises ``BitLinearError`` on a
+non-zero status.
+
+Pages the operations follow (title, section):
+  * "How to Run BitNet Inference on GPU Using CUDA Kernels: A Complete
+    Guide", "Understanding the Two-Phase Architecture" -- INT8 activation
+    quantisation in front of an INT8 x INT2 linear, called from Python through
+    ctypes (section "Compiling the INT2 CUDA Kernel").
+  * "bit-floor" README, "The core math" and "What's inside" -- integer inner
+    product, final scale multiply, mean-abs (ternary) and absmax (binary)
+    weight scales, XNOR / popcount binary GEMV.
+  * "BitCompute: 1.58-bit LLM Execution Engine", "Usage" and "Future
+    Roadmap" -- ``ternary_matmul(inputs, weights) -> [M, N]``; four weights
+    per byte.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
+
+BL_OK = 0
+BL_ERR_NULL = 1
+BL_ERR_DTYPE = 2
+BL_ERR_SHAPE = 3
+BL_ERR_ALIGN = 4
+BL_ERR_NOT_DEVICE_PTR = 5
+BL_ERR_WORKSPACE = 6
+BL_ERR_CUDA = 7
+BL_ERR_TIMEOUT = 8
+BL_ERR_UNSUPPORTED = 9
+
+BL_F32 = 0
+BL_BF16 = 1
+
+GEMV_MAX_M = 16
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.bitlinear_status_string(status).decode()
+        if status == BL_ERR_CUDA:
+            msg += " (" + _lib.bitlinear_last_cuda_error().decode() + ")"
+        super().__init__(f"{where}: {msg}")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m bit_ternary_weight_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i64, _int, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+_SIGNATURES = {
+    "bitlinear_status_string": (ctypes.c_char_p, [_int]),
+    "bitlinear_last_cuda_error": (ctypes.c_char_p, []),
+    "bitlinear_packed_bytes": (_sz, [_i64, _i64]),
+    "bitlinear_pack_workspace_bytes": (_sz, [_i64, _i64]),
+    "bitlinear_pack": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
+    "bitlinear_quantize_act": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "bitlinear_gemv": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int, _i64,
+                              _vp, _vp]),
+    "bitlinear_gemv_fused": (_int, [_vp, _vp, _i64, _i64, _vp, _int, _i64, _i64, _vp, _int,
+                                    _i64, _vp, _vp]),
+    "bitlinear_gemm_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "bitlinear_gemm": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int, _i64,
+                              _vp, _vp, _sz, _vp]),
+    "bitlinear_binary_packed_bytes": (_sz, [_i64, _i64]),
+    "bitlinear_binary_pack": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _vp]),
+    "bitlinear_binary_gemv": (_int, [_vp, _vp, _i64, _i64, _vp, _int, _vp, _int, _vp, _vp]),
+    "bitlinear_last_device_status": (_int, [_vp]),
+    "bitlinear_device_sm_count": (_int, []),
+}
+for _name, (_res, _args) in _SIGNATURES.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+lib = _lib  # the raw C ABI, for callers that marshal pointers themselves
+
+
+def _check(status: int, where: str) -> None:
+    if status != BL_OK:
+        raise BitLinearError(status, where)
+
+
+def _dt(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return BL_F32
+    if t == torch.bfloat16:
+        return BL_BF16
+    return -1
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+@dataclass
+class TernaryWeight:
+    """A packed ternary weight: TL bytes, the fp32 gamma_eff and the shape."""
+    packed: torch.Tensor   # uint8 [bitlinear_packed_bytes(N, K)]
+    w_scale: torch.Tensor  # float32 [1]
+    N: int
+    K: int
+
+
+@dataclass
+class BinaryWeight:
+    bits: torch.Tensor     # int64 [N, K/64] (uint64 words)
+    s_w: torch.Tensor      # float32 [1]
+    N: int
+    K: int
+
+
+def packed_bytes(N: int, K: int) -> int:
+    return int(_lib.bitlinear_packed_bytes(N, K))
+
+
+def pack(W: torch.Tensor) -> TernaryWeight:
+    """Absmean-quantise and 2-bit pack a weight [N, K] (fp32 or bf16, CUDA)."""
+    W = W.contiguous()
+    N, K = W.shape
+    nbytes = packed_bytes(N, K)
+    if nbytes == 0:
+        raise BitLinearError(BL_ERR_SHAPE, "pack")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    w_scale = torch.empty(1, dtype=torch.float32, device=W.device)
+    ws_bytes = int(_lib.bitlinear_pack_workspace_bytes(N, K))
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=W.device)
+    _check(_lib.bitlinear_pack(_ptr(W), _dt(W.dtype), N, K, _ptr(packed), _ptr(w_scale),
+                               _ptr(ws), ws.numel(), _stream(W.device)), "bitlinear_pack")
+    return TernaryWeight(packed, w_scale, N, K)
+
+
+def quantize_act(x: torch.Tensor):
+    """Per-token absmax int8: returns (q int8 [M,K], d fp32 [M], rowsum int32 [M])."""
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    M, K = x.shape
+    q = torch.empty(M, K, dtype=torch.int8, device=x.device)
+    d = torch.empty(M, dtype=torch.float32, device=x.device)
+    r = torch.empty(M, dtype=torch.int32, device=x.device)
+    _check(_lib.bitlinear_quantize_act(_ptr(x), _dt(x.dtype), M, K, x.stride(0), _ptr(q),
+                                       _ptr(d), _ptr(r), _stream(x.device)),
+           "bitlinear_quantize_act")
+    return q, d, r
+
+
+def _out(M, N, out_dtype, device, out):
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=device)
+    return out
+
+
+def gemv(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc_dbg=None):
+    """Decode GEMV (1 <= M <= 16) on pre-quantised activations."""
+    M = q.shape[0]
+    out = _out(M, w.N, out_dtype, q.device, out)
+    _check(_lib.bitlinear_gemv(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q), _ptr(d),
+                               _ptr(rowsum), M, _ptr(out), _dt(out.dtype), out.stride(0),
+                               _ptr(acc_dbg), _stream(q.device)), "bitlinear_gemv")
+    return out
+
+
+def gemv_fused(w: TernaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16, out=None,
+               acc_dbg=None):
+    """Decode BitLinear in one launch: quantise x, ternary GEMV, rescale (M <= 16)."""
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    M = x.shape[0]
+    out = _out(M, w.N, out_dtype, x.device, out)
+    _check(_lib.bitlinear_gemv_fused(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(x),
+                                     _dt(x.dtype), x.stride(0), M, _ptr(out), _dt(out.dtype),
+                                     out.stride(0), _ptr(acc_dbg), _stream(x.device)),
+           "bitlinear_gemv_fused")
+    return out
+
+
+def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.bitlinear_gemm_workspace_bytes(M, N, K))
+
+
+def gemm(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc_dbg=None,
+         workspace=None):
+    """Prefill GEMM (any M) on the tcgen05 int8 tensor cores."""
+    M = q.shape[0]
+    out = _out(M, w.N, out_dtype, q.device, out)
+    need = gemm_workspace_bytes(M, w.N, w.K)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.bitlinear_gemm(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q), _ptr(d),
+                               _ptr(rowsum), M, _ptr(out), _dt(out.dtype), out.stride(0),
+                               _ptr(acc_dbg), _ptr(workspace), ws_bytes, _stream(q.device)),
+           "bitlinear_gemm")
+    return out
+
+
+def linear(w: TernaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16):
+    """y = BitLinear(x): the fused GEMV for M <= 16 tokens, else quantise + GEMM."""
+    x2 = x.reshape(-1, x.shape[-1])
+    if x2.shape[0] <= GEMV_MAX_M and x2.shape[0] * w.K <= 196608:
+        y = gemv_fused(w, x2, out_dtype)
+    else:
+        q, d, r = quantize_act(x2)
+        y = gemm(w, q, d, r, out_dtype)
+    return y.reshape(*x.shape[:-1], w.N)
+
+
+def binary_pack(W: torch.Tensor) -> BinaryWeight:
+    W = W.contiguous()
+    N, K = W.shape
+    nbytes = int(_lib.bitlinear_binary_packed_bytes(N, K))
+    if nbytes == 0:
+        raise BitLinearError(BL_ERR_SHAPE, "binary_pack")
+    bits = torch.empty(N, K // 64, dtype=torch.int64, device=W.device)
+    s_w = torch.empty(1, dtype=torch.float32, device=W.device)
+    _check(_lib.bitlinear_binary_pack(_ptr(W), _dt(W.dtype), N, K, _ptr(bits), _ptr(s_w),
+                                      _stream(W.device)), "bitlinear_binary_pack")
+    return BinaryWeight(bits, s_w, N, K)
+
+
+def binary_gemv(w: BinaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16, out=None,
+                acc_dbg=None):
+    x = x.reshape(-1)
+    if out is None:
+        out = torch.empty(w.N, dtype=out_dtype, device=x.device)
+    _check(_lib.bitlinear_binary_gemv(_ptr(w.bits), _ptr(w.s_w), w.N, w.K, _ptr(x),
+                                      _dt(x.dtype), _ptr(out), _dt(out.dtype), _ptr(acc_dbg),
+                                      _stream(x.device)), "bitlinear_binary_gemv")
+    return out
+
+
+def last_device_status(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(_lib.bitlinear_last_device_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def sm_count() -> int:
+    return int(_lib.bitlinear_device_sm_count())

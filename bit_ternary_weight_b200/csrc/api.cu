@@ -1,0 +1,414 @@
+// api.cu -- the extern "C" entry points of libbitlinear.so: argument checks in
+// a fixed order (null -> dtype -> shape -> alignment -> device -> device
+// pointers -> workspace), then the launchers of the other translation units.
+// Every check that can fail runs before any launch, so a rejected call writes
+// nothing.
+#include <cuda_runtime.h>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <stdio.h>
+#include <string.h>
+
+#include "bl_internal.h"
+
+namespace bl {
+
+// Device status word: kernels whose bounded waits run out write an error code
+// here; bitlinear_last_device_status() reads and clears it.
+__device__ int g_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_info_mutex;
+DeviceInfo g_info[kMaxDevices];
+thread_local char g_cuda_err[256] = "";
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_device_ptr(const void *p)
+{
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+bool valid_dtype(int t) { return t == BL_F32 || t == BL_BF16; }
+int elem_bytes(int t) { return t == BL_BF16 ? 2 : 4; }
+
+// Common shape rule: N >= 1, K >= 64, K % 64 == 0, and sizes that keep every
+// index inside int32 tiles and int64 byte offsets comfortably.
+bool valid_nk(int64_t N, int64_t K)
+{
+    return N >= 1 && K >= 64 && K % 64 == 0 && N <= (int64_t(1) << 31) &&
+           K <= (int64_t(1) << 22);
+}
+
+// Device presence and architecture; returns BL_OK and the info, or an error.
+int need_device(const DeviceInfo **out)
+{
+    const DeviceInfo *di = device_info();
+    if (!di)
+        return BL_ERR_CUDA;
+    if (di->cc_major != 10)
+        return BL_ERR_UNSUPPORTED;
+    *out = di;
+    return BL_OK;
+}
+
+int check_dev_ptrs(std::initializer_list<const void *> ptrs)
+{
+    for (const void *p : ptrs)
+        if (p && !is_device_ptr(p))
+            return BL_ERR_NOT_DEVICE_PTR;
+    return BL_OK;
+}
+
+}  // namespace
+
+const DeviceInfo *device_info()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_info_mutex);
+    DeviceInfo &di = g_info[dev];
+    if (di.device == dev)
+        return &di;
+    DeviceInfo t;
+    t.device = dev;
+    if (cudaDeviceGetAttribute(&t.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&t.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&t.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&t.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cuda_status(cudaGetLastError());
+        return nullptr;
+    }
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
+        cuda_status(cudaGetLastError());
+        return nullptr;
+    }
+    t.status = static_cast<int *>(p);
+    di = t;
+    return &di;
+}
+
+int cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess)
+        return BL_OK;
+    snprintf(g_cuda_err, sizeof g_cuda_err, "%s: %s", cudaGetErrorName(e),
+             cudaGetErrorString(e));
+    return BL_ERR_CUDA;
+}
+
+int launch_status() { return cuda_status(cudaGetLastError()); }
+
+int occupancy(const void *func, int threads, size_t smem, int *per_sm)
+{
+    static std::mutex mu;
+    static std::map<std::tuple<int, const void *, int, size_t>, int> cache;
+    static std::map<std::pair<int, const void *>, bool> raised;
+    const DeviceInfo *di = device_info();
+    if (!di)
+        return BL_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_tuple(di->device, func, threads, smem);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+        *per_sm = it->second;
+        return BL_OK;
+    }
+    auto rk = std::make_pair(di->device, func);
+    if (!raised.count(rk)) {
+        int st = cuda_status(cudaFuncSetAttribute(
+            func, cudaFuncAttributeMaxDynamicSharedMemorySize, di->max_smem_optin));
+        if (st)
+            return st;
+        raised[rk] = true;
+    }
+    int n = 0;
+    int st = cuda_status(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem));
+    if (st)
+        return st;
+    cache[key] = n;
+    *per_sm = n;
+    return BL_OK;
+}
+
+}  // namespace bl
+
+using namespace bl;
+
+extern "C" {
+
+const char *bitlinear_status_string(int status)
+{
+    switch (status) {
+    case BL_OK: return "BL_OK";
+    case BL_ERR_NULL: return "BL_ERR_NULL: a required pointer is NULL";
+    case BL_ERR_DTYPE: return "BL_ERR_DTYPE: unsupported element type";
+    case BL_ERR_SHAPE: return "BL_ERR_SHAPE: shape or stride out of range";
+    case BL_ERR_ALIGN: return "BL_ERR_ALIGN: pointer or stride not 16-byte aligned";
+    case BL_ERR_NOT_DEVICE_PTR: return "BL_ERR_NOT_DEVICE_PTR: host pointer where device memory is required";
+    case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE: workspace missing or too small";
+    case BL_ERR_CUDA: return "BL_ERR_CUDA: CUDA runtime error";
+    case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT: a device-side bounded wait ran out";
+    case BL_ERR_UNSUPPORTED: return "BL_ERR_UNSUPPORTED: needs an sm_100 (B200) device";
+    default: return "unknown status";
+    }
+}
+
+const char *bitlinear_last_cuda_error(void) { return g_cuda_err; }
+
+size_t bitlinear_packed_bytes(int64_t N, int64_t K)
+{
+    if (!valid_nk(N, K))
+        return 0;
+    return static_cast<size_t>((N + 7) / 8 * 8) * static_cast<size_t>(K / 4);
+}
+
+size_t bitlinear_pack_workspace_bytes(int64_t N, int64_t K)
+{
+    if (!valid_nk(N, K))
+        return 0;
+    return static_cast<size_t>(N) * sizeof(double);
+}
+
+int bitlinear_pack(const void *W, int wt, int64_t N, int64_t K, uint8_t *packed,
+                   float *w_scale, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!W || !packed || !w_scale)
+        return BL_ERR_NULL;
+    if (!valid_dtype(wt))
+        return BL_ERR_DTYPE;
+    if (!valid_nk(N, K))
+        return BL_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(packed) || !aligned16(ws) || (reinterpret_cast<uintptr_t>(w_scale) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({W, packed, w_scale, ws})))
+        return st;
+    if (!ws || ws_bytes < bitlinear_pack_workspace_bytes(N, K))
+        return BL_ERR_WORKSPACE;
+    return launch_pack(W, wt, N, K, packed, w_scale, static_cast<double *>(ws),
+                       static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_quantize_act(const void *x, int xt, int64_t M, int64_t K, int64_t ldx,
+                           int8_t *q, float *d, int32_t *rowsum, void *stream)
+{
+    if (!x || !q || !d || !rowsum)
+        return BL_ERR_NULL;
+    if (!valid_dtype(xt))
+        return BL_ERR_DTYPE;
+    if (!valid_nk(1, K) || M < 1 || M > (int64_t(1) << 31) || ldx < K)
+        return BL_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(q) || (ldx * elem_bytes(xt)) % 16 ||
+        (reinterpret_cast<uintptr_t>(d) & 3u) || (reinterpret_cast<uintptr_t>(rowsum) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({x, q, d, rowsum})))
+        return st;
+    return launch_quantize_act(x, xt, M, K, ldx, q, d, rowsum,
+                               static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+int check_gemv_common(const uint8_t *packed, const float *w_scale, int64_t N,
+                      int64_t K, int64_t M, void *y, int yt, int64_t ldy,
+                      int64_t max_m)
+{
+    if (!packed || !w_scale || !y)
+        return BL_ERR_NULL;
+    if (!valid_dtype(yt))
+        return BL_ERR_DTYPE;
+    if (!valid_nk(N, K) || M < 1 || M > max_m || ldy < N)
+        return BL_ERR_SHAPE;
+    if (!aligned16(packed) || (reinterpret_cast<uintptr_t>(w_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(y) & (yt == BL_BF16 ? 1u : 3u)))
+        return BL_ERR_ALIGN;
+    return BL_OK;
+}
+
+constexpr int64_t kGemvMaxM = 16;
+constexpr int64_t kGemvMaxMK = 196608;
+
+}  // namespace
+
+int bitlinear_gemv(const uint8_t *packed, const float *w_scale, int64_t N, int64_t K,
+                   const int8_t *q, const float *d, const int32_t *rowsum, int64_t M,
+                   void *y, int yt, int64_t ldy, int32_t *acc_dbg, void *stream)
+{
+    if (!q || !d || !rowsum)
+        return BL_ERR_NULL;
+    int st = check_gemv_common(packed, w_scale, N, K, M, y, yt, ldy, kGemvMaxM);
+    if (st)
+        return st;
+    if (M * K > kGemvMaxMK)
+        return BL_ERR_SHAPE;
+    if (!aligned16(q) || (reinterpret_cast<uintptr_t>(d) & 3u) ||
+        (reinterpret_cast<uintptr_t>(rowsum) & 3u) || (reinterpret_cast<uintptr_t>(acc_dbg) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    if ((st = need_device(&di)))
+        return st;
+    if ((st = check_dev_ptrs({packed, w_scale, q, d, rowsum, y, acc_dbg})))
+        return st;
+    GemvArgs a{packed, w_scale, N, K, M, q, d, rowsum, nullptr, BL_F32, 0, y, yt, ldy, acc_dbg};
+    return launch_gemv(a, false, static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_gemv_fused(const uint8_t *packed, const float *w_scale, int64_t N,
+                         int64_t K, const void *x, int xt, int64_t ldx, int64_t M,
+                         void *y, int yt, int64_t ldy, int32_t *acc_dbg, void *stream)
+{
+    if (!x)
+        return BL_ERR_NULL;
+    int st = check_gemv_common(packed, w_scale, N, K, M, y, yt, ldy, kGemvMaxM);
+    if (st)
+        return st;
+    if (!valid_dtype(xt))
+        return BL_ERR_DTYPE;
+    if (M * K > kGemvMaxMK || ldx < K)
+        return BL_ERR_SHAPE;
+    if (!aligned16(x) || (ldx * elem_bytes(xt)) % 16 ||
+        (reinterpret_cast<uintptr_t>(acc_dbg) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    if ((st = need_device(&di)))
+        return st;
+    if ((st = check_dev_ptrs({packed, w_scale, x, y, acc_dbg})))
+        return st;
+    GemvArgs a{packed, w_scale, N, K, M, nullptr, nullptr, nullptr, x, xt, ldx, y, yt, ldy, acc_dbg};
+    return launch_gemv(a, true, static_cast<cudaStream_t>(stream));
+}
+
+size_t bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    if (!valid_nk(N, K) || M < 1)
+        return 0;
+    return gemm_workspace_bytes(M, N, K);
+}
+
+int bitlinear_gemm(const uint8_t *packed, const float *w_scale, int64_t N, int64_t K,
+                   const int8_t *q, const float *d, const int32_t *rowsum, int64_t M,
+                   void *y, int yt, int64_t ldy, int32_t *acc_dbg, void *ws,
+                   size_t ws_bytes, void *stream)
+{
+    if (!q || !d || !rowsum)
+        return BL_ERR_NULL;
+    int st = check_gemv_common(packed, w_scale, N, K, M, y, yt, ldy, int64_t(1) << 31);
+    if (st)
+        return st;
+    if (!aligned16(q) || (reinterpret_cast<uintptr_t>(d) & 3u) ||
+        (reinterpret_cast<uintptr_t>(rowsum) & 3u) || (reinterpret_cast<uintptr_t>(acc_dbg) & 3u) ||
+        !aligned16(ws))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    if ((st = need_device(&di)))
+        return st;
+    if ((st = check_dev_ptrs({packed, w_scale, q, d, rowsum, y, acc_dbg, ws})))
+        return st;
+    size_t need = gemm_workspace_bytes(M, N, K);
+    if (need && (!ws || ws_bytes < need))
+        return BL_ERR_WORKSPACE;
+    GemvArgs a{packed, w_scale, N, K, M, q, d, rowsum, nullptr, BL_F32, 0, y, yt, ldy, acc_dbg};
+    return launch_gemm(a, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t bitlinear_binary_packed_bytes(int64_t N, int64_t K)
+{
+    if (!valid_nk(N, K))
+        return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>(K / 64) * 8;
+}
+
+int bitlinear_binary_pack(const void *W, int wt, int64_t N, int64_t K, uint64_t *Wb,
+                          float *s_w, void *stream)
+{
+    if (!W || !Wb || !s_w)
+        return BL_ERR_NULL;
+    if (!valid_dtype(wt))
+        return BL_ERR_DTYPE;
+    if (!valid_nk(N, K))
+        return BL_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(Wb) || (reinterpret_cast<uintptr_t>(s_w) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({W, Wb, s_w})))
+        return st;
+    return launch_binary_pack(W, wt, N, K, Wb, s_w, static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_binary_gemv(const uint64_t *Wb, const float *s_w, int64_t N, int64_t K,
+                          const void *x, int xt, void *y, int yt, int32_t *acc_dbg,
+                          void *stream)
+{
+    if (!Wb || !s_w || !x || !y)
+        return BL_ERR_NULL;
+    if (!valid_dtype(xt) || !valid_dtype(yt))
+        return BL_ERR_DTYPE;
+    if (!valid_nk(N, K) || K > 65536)
+        return BL_ERR_SHAPE;
+    if (!aligned16(Wb) || !aligned16(x) || (reinterpret_cast<uintptr_t>(s_w) & 3u) ||
+        (reinterpret_cast<uintptr_t>(y) & (yt == BL_BF16 ? 1u : 3u)) ||
+        (reinterpret_cast<uintptr_t>(acc_dbg) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({Wb, s_w, x, y, acc_dbg})))
+        return st;
+    return launch_binary_gemv(Wb, s_w, N, K, x, xt, y, yt, acc_dbg,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_last_device_status(void *stream)
+{
+    const DeviceInfo *di = device_info();
+    if (!di)
+        return BL_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int st = cuda_status(cudaStreamSynchronize(s));
+    if (st)
+        return st;
+    int v = 0;
+    st = cuda_status(cudaMemcpy(&v, di->status, sizeof v, cudaMemcpyDeviceToHost));
+    if (st)
+        return st;
+    if (v != 0) {
+        int zero = 0;
+        st = cuda_status(cudaMemcpy(di->status, &zero, sizeof zero, cudaMemcpyHostToDevice));
+        if (st)
+            return st;
+    }
+    return v;
+}
+
+int bitlinear_device_sm_count(void)
+{
+    const DeviceInfo *di = device_info();
+    return di ? di->sm_count : 0;
+}
+
+}  // extern "C"

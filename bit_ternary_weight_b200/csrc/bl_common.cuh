@@ -1,0 +1,133 @@
+// bl_common.cuh -- device helpers shared by the sm_100a kernels of
+// libbitlinear.so: cache-hinted loads, integer dot products, reductions,
+// named barriers and the bounded-wait clock.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "bl_internal.h"
+
+namespace bl {
+
+constexpr float kEps = 1e-5f;      // floor of both absmax and absmean scales
+constexpr float kQb = 127.0f;      // int8 activation range used by the scale
+
+// Streamed, read-once data: bypass L1 allocation (weights are touched once).
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint2 ld_stream_v2(const void *p)
+{
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "l"(p));
+    return v;
+}
+
+// Read-only data that many threads re-read (activations): keep in L1.
+__device__ __forceinline__ uint4 ld_ro_v4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 4-way byte dot product, unsigned bytes of a times signed bytes of b.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ void named_barrier(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Eight input elements (one 16-byte bf16 vector or two fp32 vectors) as fp32.
+template <int XT>
+__device__ __forceinline__ void load8(const void *base, int64_t idx, float f[8]);
+
+template <>
+__device__ __forceinline__ void load8<BL_BF16>(const void *base, int64_t idx, float f[8])
+{
+    uint4 v = ld_ro_v4(static_cast<const __nv_bfloat16 *>(base) + idx);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+template <>
+__device__ __forceinline__ void load8<BL_F32>(const void *base, int64_t idx, float f[8])
+{
+    const float *p = static_cast<const float *>(base) + idx;
+    uint4 a = ld_ro_v4(p);
+    uint4 b = ld_ro_v4(p + 4);
+    f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y);
+    f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+    f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y);
+    f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+}
+
+// int8 quantisation of one value with the per-token scale s: rint(x * s)
+// (fp32 product, ties to even) clamped to [-128, 127].
+__device__ __forceinline__ int quant1(float x, float s)
+{
+    int t = __float2int_rn(__fmul_rn(x, s));
+    return max(-128, min(127, t));
+}
+
+// Final rescale: ((float)acc * d) * gamma, two round-to-nearest products.
+__device__ __forceinline__ float rescale1(int acc, float d, float gamma)
+{
+    return __fmul_rn(__fmul_rn(static_cast<float>(acc), d), gamma);
+}
+
+__device__ __forceinline__ void store_y(void *y, int yt, int64_t idx, float v)
+{
+    if (yt == BL_BF16)
+        static_cast<__nv_bfloat16 *>(y)[idx] = __float2bfloat16_rn(v);
+    else
+        static_cast<float *>(y)[idx] = v;
+}
+
+}  // namespace bl

@@ -1,0 +1,73 @@
+// bl_internal.h -- host-side declarations shared by the translation units of
+// libbitlinear.so (launchers, device properties, error bookkeeping).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/bitlinear.h"
+
+namespace bl {
+
+struct DeviceInfo {
+    int device = -1;
+    int sm_count = 0;
+    int max_smem_optin = 0;     // bytes per block with opt-in
+    int cc_major = 0, cc_minor = 0;
+    int *status = nullptr;      // device address of the status word
+};
+
+// Properties of the current device (cached per device).  nullptr on error.
+const DeviceInfo *device_info();
+
+// Records `e` as the last CUDA error of this thread and returns BL_ERR_CUDA,
+// or BL_OK when e == cudaSuccess.
+int cuda_status(cudaError_t e);
+
+// Launch-error check after a kernel launch.
+int launch_status();
+
+// Resident CTAs per SM of `func` at this block size and dynamic shared memory,
+// with the kernel's dynamic shared memory limit raised to the device maximum
+// on first use.  Cached per (device, func, threads, smem).
+int occupancy(const void *func, int threads, size_t smem, int *per_sm);
+
+// --- launchers (arguments already validated) ------------------------------
+
+int launch_quantize_act(const void *x, int xt, int64_t M, int64_t K,
+                        int64_t ldx, int8_t *q, float *d, int32_t *rowsum,
+                        cudaStream_t s);
+
+int launch_pack(const void *W, int wt, int64_t N, int64_t K, uint8_t *packed,
+                float *w_scale, double *row_sums, cudaStream_t s);
+
+struct GemvArgs {
+    const uint8_t *packed;
+    const float *w_scale;
+    int64_t N, K, M;
+    // exactly one of (q, d, rowsum) or (x, xt, ldx) is used
+    const int8_t *q;
+    const float *d;
+    const int32_t *rowsum;
+    const void *x;
+    int xt;
+    int64_t ldx;
+    void *y;
+    int yt;
+    int64_t ldy;
+    int32_t *acc_dbg;
+};
+
+int launch_gemv(const GemvArgs &a, bool fused, cudaStream_t s);
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int launch_gemm(const GemvArgs &a, void *ws, size_t ws_bytes, cudaStream_t s);
+
+int launch_binary_pack(const void *W, int wt, int64_t N, int64_t K,
+                       uint64_t *Wb, float *s_w, cudaStream_t s);
+int launch_binary_gemv(const uint64_t *Wb, const float *s_w, int64_t N,
+                       int64_t K, const void *x, int xt, void *y, int yt,
+                       int32_t *acc_dbg, cudaStream_t s);
+
+}  // namespace bl

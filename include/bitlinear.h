@@ -1,0 +1,213 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear.so, the B200 (sm_100a) BitNet b1.58
+ * BitLinear product.
+ *
+ * What the library computes (pages cited by title and section):
+ *   - per-token absmax int8 activation quantisation ("How to Run BitNet
+ *     Inference on GPU Using CUDA Kernels: A Complete Guide", section
+ *     "Understanding the Two-Phase Architecture": BitLinearKernel quantises its
+ *     inputs to INT8 with scaling factors before the INT2 kernel);
+ *   - a product with ternary {-1, 0, +1} weights stored two bits each, with
+ *     exact int32 accumulation (same guide, FAQ "Can I use the CUDA kernel for
+ *     models other than the default BitNet architecture?": an INT8 x INT2
+ *     GEMM; "BitCompute: 1.58-bit LLM Execution Engine", sections "Features"
+ *     and "Future Roadmap": add / subtract / skip, four weights per byte);
+ *   - the rescale by the per-tensor absmean weight scale and the per-token
+ *     activation scale ("bit-floor" README, section "The core math": no
+ *     floating point until the final scale multiply; section "What's inside":
+ *     mean-abs scale for ternary weights, absmax scale for binary weights);
+ *   - the binary 1-bit XNOR / popcount GEMV ("bit-floor" README, section "The
+ *     core math": y = scale_w * scale_x * (2 * POPCNT(XNOR(W, x)) - K)).
+ *
+ * Numerics (identical on the CPU oracle):
+ *   gamma     = (float)(sum_n sum_k |W[n][k]| / (N*K)), the sums in fp64, k
+ *               ascending inside a row, then rows ascending; gamma_eff =
+ *               max(gamma, 1e-5f).  Stored in *w_scale.
+ *   code      = clamp(rint(W / gamma_eff), -1, 1), fp32 division, ties to even.
+ *   a_m       = max(max_k |x[m][k]|, 1e-5f); s_m = 127 / a_m (fp32);
+ *   q[m][k]   = clamp(rint(x * s_m), -128, 127), fp32 product, ties to even;
+ *   d[m]      = a_m / 127 (fp32); rowsum[m] = sum_k q[m][k].
+ *   acc[m][n] = sum_k code[n][k] * q[m][k] (exact int32, |acc| <= 128 K).
+ *   y[m][n]   = ((float)acc * d[m]) * gamma_eff, two fp32 round-to-nearest
+ *               products in that order; bf16 output rounds y to nearest even.
+ *
+ * Packed ternary layout "TL" (the pages fix none; this library's choice):
+ *   stored value s = code + 1 in {0, 1, 2} (3 never appears), rows padded to
+ *   a multiple of 8 with code 0; byte of (n, k) =
+ *     ((n/8 * (K/64) + k/64) * 8 + n%8) * 16 + ((k%64)/16) * 4 + k%4,
+ *   bit offset 2 * ((k%16)/4).  A 16-byte chunk holds 64 consecutive k of one
+ *   row; a 32-bit word w of a chunk gives, after (w >> 2i) & 0x03030303, the
+ *   stored codes of four consecutive k in byte order.
+ * Binary layout: uint64 [N][K/64], bit j of word w <-> k = 64 w + j, bit set
+ *   when the value is negative (-0.0 counts as positive).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named as device pointers must be device (or managed) memory of
+ *     the current device; a host pointer gives BL_ERR_NOT_DEVICE_PTR.  There
+ *     is no CPU fallback.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous on it; the caller owns all memory
+ *     and keeps it alive until the stream has passed the call.
+ *   - The library allocates no device memory.  It keeps a device status word
+ *     and cached device properties only.
+ *   - Argument errors return before any launch, with nothing written.  A
+ *     failed launch returns BL_ERR_CUDA (text via bitlinear_last_cuda_error).
+ *     Device-side errors (a bounded wait that ran out) are reported by the next
+ *     bitlinear_last_device_status().
+ *   - Shapes: N >= 1, K >= 64 and K % 64 == 0, 1 <= M.
+ *   - Alignment: weight, packed, q, x and y base pointers 16-byte aligned;
+ *     row strides (ldx, ldy) in elements such that each row starts 16-byte
+ *     aligned.  Otherwise BL_ERR_ALIGN.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BL_OK = 0,
+    BL_ERR_NULL = 1,            /* a required pointer is NULL */
+    BL_ERR_DTYPE = 2,           /* unsupported element type */
+    BL_ERR_SHAPE = 3,           /* N, K, M, strides out of range */
+    BL_ERR_ALIGN = 4,           /* pointer or stride misaligned */
+    BL_ERR_NOT_DEVICE_PTR = 5,  /* a device pointer is host memory */
+    BL_ERR_WORKSPACE = 6,       /* workspace missing or too small */
+    BL_ERR_CUDA = 7,            /* CUDA runtime error */
+    BL_ERR_TIMEOUT = 8,         /* a device-side bounded wait ran out */
+    BL_ERR_UNSUPPORTED = 9      /* no sm_100 device */
+} bl_status;
+
+typedef enum { BL_F32 = 0, BL_BF16 = 1 } bl_dtype;
+
+/* Human-readable name of a status code (static string). */
+const char *bitlinear_status_string(int status);
+
+/* Text of the last CUDA runtime error seen by this library in this thread
+ * (static per-thread buffer; "" if none). */
+const char *bitlinear_last_cuda_error(void);
+
+/* Bytes of the TL packed array for an N x K weight (rows padded to 8). */
+size_t bitlinear_packed_bytes(int64_t N, int64_t K);
+
+/* Bytes of workspace bitlinear_pack needs: one fp64 partial sum per row. */
+size_t bitlinear_pack_workspace_bytes(int64_t N, int64_t K);
+
+/*
+ * Offline ternary packer: absmean scale, round-clip to {-1, 0, +1}, 2-bit
+ * pack into layout TL.  Source: "bit-floor" README, section "What's inside"
+ * (mean-abs scale for ternary weights, packing f32 weights); "BitCompute",
+ * section "Future Roadmap" (four weights per byte).
+ *   W        device, [N][K] row-major, dtype wt (BL_F32 or BL_BF16)
+ *   packed   device, bitlinear_packed_bytes(N, K) bytes, written
+ *   w_scale  device, 1 float, written with gamma_eff
+ *   ws       device workspace of at least bitlinear_pack_workspace_bytes;
+ *            contents on entry are ignored, on exit unspecified
+ */
+int bitlinear_pack(const void *W, int wt, int64_t N, int64_t K,
+                   uint8_t *packed, float *w_scale, void *ws, size_t ws_bytes,
+                   void *stream);
+
+/*
+ * Per-token absmax int8 activation quantisation.  Source: "How to Run BitNet
+ * Inference on GPU Using CUDA Kernels", section "Understanding the Two-Phase
+ * Architecture" (inputs quantised to INT8 with scaling factors).
+ *   x       device, [M][ldx] of dtype xt (BL_F32 or BL_BF16), ldx >= K
+ *   q       device, [M][K] int8, written
+ *   d       device, [M] float (dequantisation scale a_m / 127), written
+ *   rowsum  device, [M] int32 (sum of q over k), written
+ */
+int bitlinear_quantize_act(const void *x, int xt, int64_t M, int64_t K,
+                           int64_t ldx, int8_t *q, float *d, int32_t *rowsum,
+                           void *stream);
+
+/*
+ * Ternary GEMV for 1 <= M <= 16 tokens on pre-quantised activations.
+ * Source: "How to Run BitNet Inference on GPU Using CUDA Kernels", section
+ * "Key Components and Source Code Architecture" (the decode-phase INT8 x INT2
+ * linear); "bit-floor" README, section "The core math".
+ *   packed, w_scale   from bitlinear_pack (device)
+ *   q, d, rowsum      from bitlinear_quantize_act (device), q is [M][K]
+ *   y                 device, [M][ldy] of dtype yt (BL_F32 or BL_BF16), ldy >= N
+ *   acc_dbg           NULL, or device [M][N] int32 receiving acc (before rescale)
+ * M * K must not exceed 196608 (the activations are staged on chip).
+ */
+int bitlinear_gemv(const uint8_t *packed, const float *w_scale, int64_t N,
+                   int64_t K, const int8_t *q, const float *d,
+                   const int32_t *rowsum, int64_t M, void *y, int yt,
+                   int64_t ldy, int32_t *acc_dbg, void *stream);
+
+/*
+ * Ternary GEMV with the activation quantisation fused into the kernel: the
+ * whole decode BitLinear (quantise, product, rescale) in one launch.
+ *   x    device, [M][ldx] of dtype xt (BL_F32 or BL_BF16)
+ *   other arguments as for bitlinear_gemv.
+ */
+int bitlinear_gemv_fused(const uint8_t *packed, const float *w_scale,
+                         int64_t N, int64_t K, const void *x, int xt,
+                         int64_t ldx, int64_t M, void *y, int yt, int64_t ldy,
+                         int32_t *acc_dbg, void *stream);
+
+/* Bytes of workspace bitlinear_gemm needs for this problem (0 if none). */
+size_t bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Ternary GEMM for any M >= 1 (prefill), on the tcgen05 int8 tensor cores
+ * with int32 accumulators in tensor memory.  Source: "How to Run BitNet
+ * Inference on GPU Using CUDA Kernels", FAQ (a generic INT8 x INT2 GEMM);
+ * "BitCompute", section "Future Roadmap" (tensor-core execution of the
+ * ternary product).  Arguments as for bitlinear_gemv, plus
+ *   ws, ws_bytes   device workspace, at least bitlinear_gemm_workspace_bytes
+ *                  (may be NULL when that is 0).
+ * q must be 16-byte aligned and K % 64 == 0.
+ */
+int bitlinear_gemm(const uint8_t *packed, const float *w_scale, int64_t N,
+                   int64_t K, const int8_t *q, const float *d,
+                   const int32_t *rowsum, int64_t M, void *y, int yt,
+                   int64_t ldy, int32_t *acc_dbg, void *ws, size_t ws_bytes,
+                   void *stream);
+
+/* Bytes of the binary packed array: N * (K/64) * 8. */
+size_t bitlinear_binary_packed_bytes(int64_t N, int64_t K);
+
+/*
+ * Binary (1-bit) weight packer: sign bits and the absmax scale.  Source:
+ * "bit-floor" README, section "What's inside" (binary packing, absmax scale).
+ *   W     device [N][K] of dtype wt
+ *   Wb    device uint64 [N][K/64], written
+ *   s_w   device, 1 float, written with max |W|
+ */
+int bitlinear_binary_pack(const void *W, int wt, int64_t N, int64_t K,
+                          uint64_t *Wb, float *s_w, void *stream);
+
+/*
+ * Binary GEMV of one token: acc[n] = 2 * popcount(XNOR(Wb[n], xb)) - K,
+ * y[n] = (float)acc[n] * (s_w * s_x), s_x = max |x|, xb the sign bits of x.
+ * Source: "bit-floor" README, section "The core math".
+ *   x        device [K] of dtype xt
+ *   y        device [N] of dtype yt
+ *   acc_dbg  NULL or device [N] int32
+ */
+int bitlinear_binary_gemv(const uint64_t *Wb, const float *s_w, int64_t N,
+                          int64_t K, const void *x, int xt, void *y, int yt,
+                          int32_t *acc_dbg, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device: BL_OK, or BL_ERR_TIMEOUT if a kernel's bounded wait ran
+ * out since the last call.  BL_ERR_CUDA if the synchronisation failed.
+ */
+int bitlinear_last_device_status(void *stream);
+
+/* Number of SMs of the current device (0 on error); for callers sizing work. */
+int bitlinear_device_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

@@ -68,6 +68,7 @@ def _load():
             "oracle_binary_signs": (None, [vp, i64, i64, ctypes.c_int, vp]),
             "oracle_binary_acc": (None, [vp, vp, i64, i64, vp]),
             "oracle_binary_rescale": (None, [vp, f32, f32, i64, vp]),
+            "oracle_num_threads": (ctypes.c_int, []),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -103,6 +104,11 @@ def ternary_codes(W: np.ndarray, gamma_eff) -> np.ndarray:
     out = np.empty((N, K), np.int8)
     _load().oracle_ternary_codes(_p(W), N, K, float(np.float32(gamma_eff)), _p(out))
     return out
+
+
+def num_threads() -> int:
+    """Threads the oracle's parallel loops use."""
+    return int(_load().oracle_num_threads())
 
 
 def packed_bytes(N: int, K: int) -> int:

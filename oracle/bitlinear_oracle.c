@@ -296,3 +296,16 @@ void oracle_binary_rescale(const int32_t *acc, float s_w, float s_x, int64_t N,
     for (int64_t n = 0; n < N; ++n)
         y[n] = (float)acc[n] * s;
 }
+
+/* Threads the OpenMP loops above use (1 when built without OpenMP). */
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

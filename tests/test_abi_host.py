@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load and export every function that include/*.h declares;
+argument errors (null pointers, element types, shapes, alignment) must be
+reported with the documented status before any CUDA call, so they are
+testable on a machine without a device.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(bitlinear_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def bl():
+    import bit_ternary_weight_b200 as b
+    return b
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("bitlinear_pack", "bitlinear_quantize_act", "bitlinear_gemv",
+                     "bitlinear_gemm", "bitlinear_binary_gemv"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(bl):
+    raw = ctypes.CDLL(bl.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(raw, n)]
+    assert not missing, missing
+
+
+def test_status_strings(bl):
+    for s in range(10):
+        assert bl.lib.bitlinear_status_string(s).startswith(b"BL_")
+    assert bl.lib.bitlinear_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("N,K", [(1, 64), (8, 128), (13, 256), (640, 2560), (28672, 8192),
+                                 (8192, 28672)])
+def test_packed_sizes_match_layout(bl, N, K):
+    assert bl.packed_bytes(N, K) == oracle.packed_bytes(N, K)
+    assert bl.lib.bitlinear_binary_packed_bytes(N, K) == N * (K // 64) * 8
+    assert bl.lib.bitlinear_pack_workspace_bytes(N, K) == 8 * N
+
+
+@pytest.mark.parametrize("N,K", [(0, 64), (8, 0), (8, 100), (8, 32), (-1, 64)])
+def test_invalid_shapes_have_no_size(bl, N, K):
+    assert bl.packed_bytes(N, K) == 0
+    assert bl.lib.bitlinear_binary_packed_bytes(N, K) == 0
+
+
+# Fake device addresses: the argument checks must reject these calls before any
+# CUDA call, so the pointers are never dereferenced.
+A = 0x7f0000000000          # 16-byte aligned
+MIS = A + 4                 # misaligned for 16-byte vectors
+
+
+def _gemv(bl, packed=A, scale=A, N=256, K=256, q=A, d=A, r=A, M=1, y=A, yt=1, ldy=256,
+          acc=None):
+    return bl.lib.bitlinear_gemv(packed, scale, N, K, q, d, r, M, y, yt, ldy, acc, None)
+
+
+def test_gemv_argument_errors(bl):
+    assert _gemv(bl, packed=None) == bl.BL_ERR_NULL
+    assert _gemv(bl, q=None) == bl.BL_ERR_NULL
+    assert _gemv(bl, y=None) == bl.BL_ERR_NULL
+    assert _gemv(bl, yt=7) == bl.BL_ERR_DTYPE
+    assert _gemv(bl, K=100) == bl.BL_ERR_SHAPE
+    assert _gemv(bl, M=0) == bl.BL_ERR_SHAPE
+    assert _gemv(bl, M=17) == bl.BL_ERR_SHAPE
+    assert _gemv(bl, ldy=10) == bl.BL_ERR_SHAPE
+    assert _gemv(bl, M=16, K=16384) == bl.BL_ERR_SHAPE  # activations exceed on-chip staging
+    assert _gemv(bl, packed=MIS) == bl.BL_ERR_ALIGN
+    assert _gemv(bl, q=MIS) == bl.BL_ERR_ALIGN
+
+
+def test_fused_and_quant_argument_errors(bl):
+    L = bl.lib
+    assert L.bitlinear_gemv_fused(A, A, 256, 256, None, 1, 256, 1, A, 1, 256, None, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_gemv_fused(A, A, 256, 256, A, 5, 256, 1, A, 1, 256, None, None) == bl.BL_ERR_DTYPE
+    assert L.bitlinear_gemv_fused(A, A, 256, 256, A, 1, 100, 1, A, 1, 256, None, None) == bl.BL_ERR_SHAPE
+    # ldx of 260 bf16 elements = 520 bytes: rows not 16-byte aligned
+    assert L.bitlinear_gemv_fused(A, A, 256, 256, A, 1, 260, 1, A, 1, 256, None, None) == bl.BL_ERR_ALIGN
+    assert L.bitlinear_quantize_act(None, 1, 4, 256, 256, A, A, A, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_quantize_act(A, 3, 4, 256, 256, A, A, A, None) == bl.BL_ERR_DTYPE
+    assert L.bitlinear_quantize_act(A, 1, 0, 256, 256, A, A, A, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_quantize_act(A, 1, 4, 256, 128, A, A, A, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_quantize_act(MIS, 1, 4, 256, 256, A, A, A, None) == bl.BL_ERR_ALIGN
+
+
+def test_pack_and_binary_argument_errors(bl):
+    L = bl.lib
+    assert L.bitlinear_pack(None, 0, 8, 64, A, A, A, 64, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_pack(A, 2, 8, 64, A, A, A, 64, None) == bl.BL_ERR_DTYPE
+    assert L.bitlinear_pack(A, 0, 8, 96, A, A, A, 64, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_pack(MIS, 0, 8, 64, A, A, A, 64, None) == bl.BL_ERR_ALIGN
+    assert L.bitlinear_binary_pack(A, 0, 8, 64, None, A, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_binary_gemv(A, A, 8, 64, A, 9, A, 1, None, None) == bl.BL_ERR_DTYPE
+    assert L.bitlinear_binary_gemv(A, A, 8, 65, A, 1, A, 1, None, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_gemm(A, A, 8, 64, None, A, A, 4, A, 1, 8, None, None, 0, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_gemm(A, A, 8, 64, A, A, A, 0, A, 1, 8, None, None, 0, None) == bl.BL_ERR_SHAPE
+
+
+def test_valid_arguments_without_device_fail_cleanly(bl):
+    """On a machine with no GPU the checks pass and the device query fails."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    st = _gemv(bl)
+    assert st in (bl.BL_ERR_CUDA, bl.BL_ERR_UNSUPPORTED)

@@ -1,0 +1,223 @@
+"""GPU parity of the CUDA path against the CPU oracle, through the C ABI.
+
+Integers (packed bytes, q, rowsum, acc) must match bit for bit; the weight
+and activation scales must match bit for bit (they are defined with a fixed
+fp32/fp64 operation order); rescaled outputs must be within 1e-3 relative of
+the oracle and, by construction, bit-identical to it.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs as si
+from parity_helpers import (Guarded, assert_rel, bf16_bits_of, compare_outputs, dev,
+                            f32_bits, oracle_weight, seeded_problem)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bl():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import bit_ternary_weight_b200 as b
+    return b
+
+
+def _pack_gpu(bl, W):
+    return bl.pack(W.to(dev()))
+
+
+# ------------------------------------------------------------------ packer
+
+PACK_SHAPES = [(8, 64), (13, 128), (40, 2560), (512, 256), (1001, 192),
+               (2560, 2560), (640, 2560), (6912, 2560), (2560, 6912)]
+
+
+@pytest.mark.parametrize("N,K", PACK_SHAPES)
+@pytest.mark.parametrize("wdtype", [torch.float32, torch.bfloat16])
+def test_pack_parity(bl, N, K, wdtype):
+    W = si.weight(N, K, seed=N + K).to(wdtype)
+    g, codes, packed = oracle_weight(W.float())
+    w = _pack_gpu(bl, W)
+    torch.cuda.synchronize()
+    assert f32_bits(w.w_scale.cpu().numpy())[0] == f32_bits(np.float32([g]))[0]
+    np.testing.assert_array_equal(w.packed.cpu().numpy(), packed)
+
+
+@pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672)])
+def test_pack_parity_100b(bl, N, K):
+    W = si.weight(N, K, seed=7)
+    g, codes, packed = oracle_weight(W)
+    w = _pack_gpu(bl, W)
+    torch.cuda.synchronize()
+    assert f32_bits(w.w_scale.cpu().numpy())[0] == f32_bits(np.float32([g]))[0]
+    np.testing.assert_array_equal(w.packed.cpu().numpy(), packed)
+
+
+def test_pack_zero_weight(bl):
+    W = torch.zeros(16, 128)
+    w = _pack_gpu(bl, W)
+    assert w.w_scale.item() == np.float32(1e-5)
+    assert (w.packed.cpu().numpy() == 0x55).all()
+
+
+# ------------------------------------------------------------------ activation quant
+
+@pytest.mark.parametrize("M,K", [(1, 256), (3, 2560), (16, 6912), (128, 256), (512, 2560),
+                                 (2, 28672), (8192, 6912)])
+@pytest.mark.parametrize("xdtype", [torch.bfloat16, torch.float32])
+def test_quantize_parity(bl, M, K, xdtype):
+    x = si.activations(M, K, seed=M + K, dtype=xdtype)
+    q_o, d_o, r_o = oracle.quantize_act(x.float().numpy())
+    q, d, r = bl.quantize_act(x.to(dev()))
+    np.testing.assert_array_equal(q.cpu().numpy(), q_o)
+    np.testing.assert_array_equal(f32_bits(d.cpu().numpy()), f32_bits(d_o))
+    np.testing.assert_array_equal(r.cpu().numpy(), r_o)
+
+
+def test_quantize_edge_tokens(bl):
+    K = 512
+    x = torch.randn(6, K)
+    x[0] = 0.0                       # all-zero token
+    x[1, 17] = 1e4                   # one huge outlier
+    x[2] = 3.0                       # constant token: every q = 127
+    x[2, ::2] = -3.0
+    x[3] = 1e-30                     # below the 1e-5 floor
+    x[4] = torch.tensor([2.5, -1.5] * (K // 2))  # exact halves after scaling
+    x[4, 0] = 127.0
+    x[5, 5] = -x[5].abs().max() * 2  # negative extreme
+    for xd in (torch.float32, torch.bfloat16):
+        xx = x.to(xd)
+        q_o, d_o, r_o = oracle.quantize_act(xx.float().numpy())
+        q, d, r = bl.quantize_act(xx.to(dev()))
+        np.testing.assert_array_equal(q.cpu().numpy(), q_o)
+        np.testing.assert_array_equal(f32_bits(d.cpu().numpy()), f32_bits(d_o))
+        np.testing.assert_array_equal(r.cpu().numpy(), r_o)
+
+
+def test_quantize_strided_rows(bl):
+    M, K, ld = 5, 256, 384
+    base = si.activations(M, ld, seed=3, dtype=torch.bfloat16)
+    x = base[:, :K]
+    q_o, d_o, r_o = oracle.quantize_act(x.float().numpy())
+    q, d, r = bl.quantize_act(base.to(dev())[:, :K])
+    np.testing.assert_array_equal(q.cpu().numpy(), q_o)
+    np.testing.assert_array_equal(r.cpu().numpy(), r_o)
+
+
+# ------------------------------------------------------------------ ternary GEMV
+
+def _oracle_gemv(g, codes, x):
+    q, d, r = oracle.quantize_act(x.float().numpy())
+    acc = oracle.ternary_acc(codes, q)
+    return oracle.rescale(acc, d, g), acc
+
+
+def _check_gemv(bl, W, x, out_dtype, fused, guard=True):
+    N, K = W.shape
+    M = x.shape[0]
+    g, codes, _ = oracle_weight(W)
+    y_o, acc_o = _oracle_gemv(g, codes, x)
+    w = _pack_gpu(bl, W)
+    xd = x.to(dev())
+    yb = Guarded(M * N, out_dtype, dev())
+    ab = Guarded(M * N, torch.int32, dev())
+    y = yb.view.view(M, N)
+    acc = ab.view.view(M, N)
+    if fused:
+        bl.gemv_fused(w, xd, out=y, acc_dbg=acc)
+    else:
+        q, d, r = bl.quantize_act(xd)
+        bl.gemv(w, q, d, r, out=y, acc_dbg=acc)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+    compare_outputs(y, y_o)
+    if guard:
+        assert yb.intact() and ab.intact()
+
+
+@pytest.mark.parametrize("K,N", si.DECODE_SHAPES_2B)
+@pytest.mark.parametrize("fused", [True, False])
+def test_decode_gemv_2b_shapes(bl, K, N, fused):
+    W, x = seeded_problem(N, K, 1, seed=0)
+    _check_gemv(bl, W, x, torch.bfloat16, fused)
+
+
+@pytest.mark.parametrize("K,N", si.DECODE_SHAPES_2B)
+def test_decode_gemv_fp32_output(bl, K, N):
+    W, x = seeded_problem(N, K, 1, seed=1)
+    _check_gemv(bl, W, x, torch.float32, True)
+
+
+@pytest.mark.parametrize("K,N", si.DECODE_SHAPES_100B)
+def test_decode_gemv_100b_shapes(bl, K, N):
+    W, x = seeded_problem(N, K, 1, seed=0)
+    _check_gemv(bl, W, x, torch.bfloat16, True)
+
+
+@pytest.mark.parametrize("N,K,M", [(13, 64, 1), (1001, 192, 3), (8, 128, 16), (77, 320, 5),
+                                   (1, 64, 2), (4096, 64, 7), (24, 12288, 16)])
+@pytest.mark.parametrize("fused", [True, False])
+def test_gemv_ragged_and_edge(bl, N, K, M, fused):
+    W, x = seeded_problem(N, K, M, seed=N * 7 + K + M)
+    if M >= 2:
+        x[0] = 0.0
+    _check_gemv(bl, W, x, torch.bfloat16, fused)
+
+
+def test_gemv_fp32_input_and_strided_output(bl):
+    N, K, M = 300, 256, 4
+    W, x = seeded_problem(N, K, M, seed=11, xdtype=torch.float32)
+    g, codes, _ = oracle_weight(W)
+    y_o, _ = _oracle_gemv(g, codes, x)
+    w = _pack_gpu(bl, W)
+    big = torch.full((M, 320), -7.0, dtype=torch.float32, device=dev())
+    bl.gemv_fused(w, x.to(dev()), out=big[:, :N])
+    torch.cuda.synchronize()
+    compare_outputs(big[:, :N], y_o)
+    assert (big[:, N:] == -7.0).all()
+
+
+def test_small_batch_sweep_100_seeds(bl):
+    """Small-batch GEMV: M in {1,2,4,8,16} x the four 2.4B shapes x 100 seeds."""
+    for K, N in si.DECODE_SHAPES_2B:
+        for seed in range(100):
+            W = si.weight(N, K, seed=1000 + seed)
+            g, codes, _ = oracle_weight(W)
+            w = _pack_gpu(bl, W)
+            for M in si.SMALL_BATCH_M:
+                x = si.activations(M, K, seed=seed * 31 + M)
+                y_o, acc_o = _oracle_gemv(g, codes, x)
+                acc = torch.empty(M, N, dtype=torch.int32, device=dev())
+                y = bl.gemv_fused(w, x.to(dev()), acc_dbg=acc)
+                np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+                compare_outputs(y, y_o)
+
+
+def test_host_pointer_rejected(bl):
+    W = si.weight(16, 64)
+    w = _pack_gpu(bl, W)
+    x_host = torch.randn(1, 64, dtype=torch.bfloat16)
+    with pytest.raises(bl.BitLinearError) as e:
+        bl.gemv_fused(w, x_host, out=torch.empty(1, 16, dtype=torch.bfloat16, device=dev()))
+    assert e.value.status == bl.BL_ERR_NOT_DEVICE_PTR
+
+
+# ------------------------------------------------------------------ binary GEMV
+
+@pytest.mark.parametrize("N,K", [(28672, 8192), (1, 64), (333, 640), (64, 4096), (10, 40960)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_binary_gemv_parity(bl, N, K, out_dtype):
+    W = si.weight(N, K, seed=K)
+    x = si.activations(1, K, seed=K, dtype=torch.bfloat16)
+    ref = oracle.binary_gemv(W.numpy(), x.float().numpy())
+    bw = bl.binary_pack(W.to(dev()))
+    acc = torch.empty(N, dtype=torch.int32, device=dev())
+    y = bl.binary_gemv(bw, x.to(dev()), out_dtype=out_dtype, acc_dbg=acc)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bw.bits.cpu().numpy().view(np.uint64), ref["Wb"])
+    assert f32_bits(bw.s_w.cpu().numpy())[0] == f32_bits(np.float32([ref["s_w"]]))[0]
+    np.testing.assert_array_equal(acc.cpu().numpy(), ref["acc"])
+    compare_outputs(y.view(1, N), ref["y"].reshape(1, N))
