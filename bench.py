@@ -442,17 +442,20 @@ def run_ours(args, world, rank, local):
 
     extra = {}
     if rank == 0 and not args.no_extra:
-        extra["isolated_2b"] = [isolated_gemv(bl, K, N, device=device) for (K, N) in si.DECODE_SHAPES_2B]
-        extra["isolated_100b"] = [isolated_gemv(bl, K, N, iters=50, device=device)
-                                  for (K, N) in si.DECODE_SHAPES_100B]
-        extra["small_batch_2560x6912"] = [isolated_gemv(bl, 2560, 6912, M=m, iters=100, device=device)
-                                          for m in si.SMALL_BATCH_M]
-        extra["binary_100b"] = isolated_binary(bl, 8192, 28672, device=device)
-        try:
-            extra["prefill"] = [prefill_gemm(bl, K, N, M, device=device)
-                                for (K, N) in si.PREFILL_SHAPES for M in si.PREFILL_TOKENS]
-        except Exception as ex:  # GEMM not available: reported, never hidden
-            extra["prefill"] = {"error": str(ex)[:200]}
+        def measure(key, fn):
+            try:
+                extra[key] = fn()
+            except Exception as ex:  # reported in the line, never hidden
+                extra[key] = {"error": str(ex)[:300]}
+        measure("isolated_2b", lambda: [isolated_gemv(bl, K, N, device=device)
+                                        for (K, N) in si.DECODE_SHAPES_2B])
+        measure("isolated_100b", lambda: [isolated_gemv(bl, K, N, iters=50, device=device)
+                                          for (K, N) in si.DECODE_SHAPES_100B])
+        measure("small_batch_2560x6912", lambda: [
+            isolated_gemv(bl, 2560, 6912, M=m, iters=100, device=device) for m in si.SMALL_BATCH_M])
+        measure("binary_100b", lambda: isolated_binary(bl, 8192, 28672, device=device))
+        measure("prefill", lambda: [prefill_gemm(bl, K, N, M, device=device)
+                                    for (K, N) in si.PREFILL_SHAPES for M in si.PREFILL_TOKENS])
 
     if rank != 0:
         return

@@ -110,7 +110,9 @@ def _ptr(t):
 
 
 def _stream(device: torch.device):
-    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    # a CPU tensor still goes to the library, which rejects host pointers
+    dev = device if device.type == "cuda" else None
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
 
 
 @dataclass

@@ -129,8 +129,16 @@ int occupancy(const void *func, int threads, size_t smem, int *per_sm)
     }
     auto rk = std::make_pair(di->device, func);
     if (!raised.count(rk)) {
-        int st = cuda_status(cudaFuncSetAttribute(
-            func, cudaFuncAttributeMaxDynamicSharedMemorySize, di->max_smem_optin));
+        // the dynamic limit may take whatever the kernel's static shared memory leaves
+        cudaFuncAttributes fa;
+        int st = cuda_status(cudaFuncGetAttributes(&fa, func));
+        if (st)
+            return st;
+        const int dyn_max = di->max_smem_optin - int(fa.sharedSizeBytes);
+        if (smem > size_t(dyn_max > 0 ? dyn_max : 0))
+            return BL_ERR_SHAPE;
+        st = cuda_status(cudaFuncSetAttribute(
+            func, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max));
         if (st)
             return st;
         raised[rk] = true;

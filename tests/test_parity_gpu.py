@@ -221,3 +221,49 @@ def test_binary_gemv_parity(bl, N, K, out_dtype):
     assert f32_bits(bw.s_w.cpu().numpy())[0] == f32_bits(np.float32([ref["s_w"]]))[0]
     np.testing.assert_array_equal(acc.cpu().numpy(), ref["acc"])
     compare_outputs(y.view(1, N), ref["y"].reshape(1, N))
+
+
+# ------------------------------------------------------------------ prefill GEMM (tcgen05)
+
+def _check_gemm(bl, N, K, M, xdtype=torch.bfloat16, out_dtype=torch.bfloat16, seed=0,
+                outliers=True, sample=None):
+    W = si.weight(N, K, seed=seed)
+    x = si.activations(M, K, seed=seed, outliers=outliers, dtype=xdtype)
+    g, codes, _ = oracle_weight(W)
+    w = _pack_gpu(bl, W)
+    q, d, r = bl.quantize_act(x.to(dev()))
+    yb = Guarded(M * N, out_dtype, dev())
+    ab = Guarded(M * N, torch.int32, dev())
+    y = yb.view.view(M, N)
+    acc = ab.view.view(M, N)
+    bl.gemm(w, q, d, r, out=y, acc_dbg=acc)
+    torch.cuda.synchronize()
+    assert bl.last_device_status() == 0
+    rows = np.arange(M) if sample is None else sample
+    xs = x[torch.as_tensor(rows)].float().numpy()
+    q_o, d_o, r_o = oracle.quantize_act(xs)
+    acc_o = oracle.ternary_acc(codes, q_o)
+    y_o = oracle.rescale(acc_o, d_o, g)
+    np.testing.assert_array_equal(acc.cpu().numpy()[rows], acc_o)
+    compare_outputs(y[torch.as_tensor(rows, device=dev())], y_o)
+    assert yb.intact() and ab.intact()
+
+
+def test_gemm_config1_fp32(bl):
+    """X[128x256] fp32 ~N(0,1) (no outliers) x W[512x256]^T, fp32 output."""
+    _check_gemm(bl, 512, 256, 128, xdtype=torch.float32, out_dtype=torch.float32, outliers=False)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (160, 200, 2560), (130, 300, 192),
+                                   (256, 256, 64), (128, 1001, 320), (5, 77, 128),
+                                   (300, 129, 6912), (17, 8, 64)])
+def test_gemm_ragged_shapes(bl, M, N, K):
+    _check_gemm(bl, N, K, M, seed=M + N + K)
+
+
+@pytest.mark.parametrize("K,N", si.PREFILL_SHAPES)
+@pytest.mark.parametrize("M", si.PREFILL_TOKENS)
+def test_gemm_prefill_full_size(bl, K, N, M):
+    rng = np.random.default_rng(M + K)
+    sample = np.unique(np.concatenate([[0, M - 1, 127, 128], rng.integers(0, M, 60)]))
+    _check_gemm(bl, N, K, M, seed=3, sample=sample)
