@@ -493,8 +493,53 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_case(args):
+    """One kernel on one shape, --iters times (for profiling); prints a JSON line."""
+    import bit_ternary_weight_b200 as bl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(17)
+    K, N, M = args.K, args.N, args.M
+    W = torch.randn(N, K, generator=gen, device=dev) * 0.02
+    x = si.activations(M, K, seed=9).to(dev)
+    if args.case == "binary":
+        w = bl.binary_pack(W)
+        fn = lambda: bl.binary_gemv(w, x[0])  # noqa: E731
+        nbytes, ops = N * K // 8, 2 * N * K
+    else:
+        w = bl.pack(W)
+        if args.case == "gemv":
+            fn = lambda: bl.gemv_fused(w, x)  # noqa: E731
+        else:
+            q, d, r = bl.quantize_act(x)
+            ws = torch.empty(max(bl.gemm_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
+            fn = lambda: bl.gemm(w, q, d, r, workspace=ws)  # noqa: E731
+        nbytes, ops = bl.packed_bytes(N, K), 2 * M * N * K
+    del W
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.iters):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    t = s.elapsed_time(e) / 1000.0 / args.iters
+    print(json.dumps({"case": args.case, "K": K, "N": N, "M": M, "iters": args.iters,
+                      "us": t * 1e6, "weight_GBps": nbytes / t / 1e9, "TOPS": ops / t / 1e12,
+                      "note": "same weights every launch (L2-warm unless profiled)"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=["stream", "gemv", "gemm", "binary"], default="stream",
+                    help="stream: the benchmark; others: one kernel on one shape (profiling)")
+    ap.add_argument("--K", type=int, default=8192)
+    ap.add_argument("--N", type=int, default=28672)
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--iters", type=int, default=5)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
@@ -507,6 +552,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.case != "stream":
+        run_case(args)
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

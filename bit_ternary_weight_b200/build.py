@@ -1,6 +1,6 @@
 """Build libbitlinear.so in-tree: every CUDA source compiled for sm_100a only.
 
-    python -m bit_ternary_weight_b200.build [--force] [--verbose]
+    python bit_ternary_weight_b200/build.py [--force] [--verbose] [--ptxas-v]
 
 Objects go to ``bit_ternary_weight_b200/_build/``; the shared library lands
 next to this file so that it travels with the source tree.  The CUDA runtime
