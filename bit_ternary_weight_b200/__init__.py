@@ -4,8 +4,8 @@ Every function here only checks and marshals torch tensors (device pointers,
 sizes, dtypes and the current CUDA stream) into the C ABI of
 ``libbitlinear.so`` declared in ``include/bitlinear.h``; all arithmetic runs in
 the library's CUDA kernels.  There is no CPU fallback: importing this package
-fails if the library has not been built (``python -m
-bit_ternary_weight_b200.build``), and every call raises ``BitLinearError`` on a
+fails if the library has not been built (``python
+bit_ternary_weight_b200/build.py``), and every call raises ``BitLinearError`` on a
 non-zero status.
 
 Pages the operations follow (title, section):
@@ -59,7 +59,7 @@ class BitLinearError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m bit_ternary_weight_b200.build`")
+        f"{LIB_PATH} is missing: build it with `python bit_ternary_weight_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -70,6 +70,7 @@ _SIGNATURES = {
     "bitlinear_packed_bytes": (_sz, [_i64, _i64]),
     "bitlinear_pack_workspace_bytes": (_sz, [_i64, _i64]),
     "bitlinear_pack": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _vp, _sz, _vp]),
+    "bitlinear_pack_noalloc": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _vp]),
     "bitlinear_quantize_act": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
     "bitlinear_gemv": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int, _i64,
                               _vp, _vp]),
@@ -149,6 +150,21 @@ def pack(W: torch.Tensor) -> TernaryWeight:
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=W.device)
     _check(_lib.bitlinear_pack(_ptr(W), _dt(W.dtype), N, K, _ptr(packed), _ptr(w_scale),
                                _ptr(ws), ws.numel(), _stream(W.device)), "bitlinear_pack")
+    return TernaryWeight(packed, w_scale, N, K)
+
+
+PACK_NOALLOC_MAX_ROWS = 65536
+
+
+def pack_noalloc(W: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor) -> TernaryWeight:
+    """Like ``pack`` but into caller-given buffers and with no workspace: the
+    library keeps the scratch it needs in a device array of its own (N must
+    not exceed PACK_NOALLOC_MAX_ROWS).  For callers that cannot allocate
+    device memory when they pack; this function allocates nothing either."""
+    N, K = W.shape
+    _check(_lib.bitlinear_pack_noalloc(_ptr(W), _dt(W.dtype), N, K, _ptr(packed),
+                                       _ptr(w_scale), _stream(W.device)),
+           "bitlinear_pack_noalloc")
     return TernaryWeight(packed, w_scale, N, K)
 
 

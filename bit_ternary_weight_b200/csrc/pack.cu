@@ -14,6 +14,8 @@
 //   3. pack_kernel         one thread per 32-bit output word (16 codes).
 // The order of the fp64 additions is part of the definition of gamma, so the
 // result is bit-identical to a sequential CPU evaluation.
+#include <mutex>
+
 #include "bl_common.cuh"
 
 namespace bl {
@@ -129,4 +131,81 @@ int launch_pack(const void *W, int wt, int64_t N, int64_t K, uint8_t *packed,
     return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// Packing with no caller-provided workspace (bitlinear_pack_noalloc).
+//
+// The per-row fp64 sums live in this file-scope device array instead of a
+// workspace the caller allocates.  Every GPU that loads the library holds it
+// (512 KiB) until the process exits.  In host code the symbol is only a
+// host-side stand-in, so its device address is looked up once per device with
+// cudaGetSymbolAddress, with that device current, and passed to the kernels.
+constexpr int64_t kNoAllocMaxRows = BITLINEAR_PACK_NOALLOC_MAX_ROWS;
+static __device__ __align__(256) double g_pack_scratch[kNoAllocMaxRows];
+
+namespace {
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mutex;
+double *g_scratch_addr[kMaxScratchDevices] = {};
+
+// Device address of g_pack_scratch on the current device (set up on first use).
+int scratch_address(double **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_status(e);
+    if (dev < 0 || dev >= kMaxScratchDevices)
+        return BL_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_pack_scratch);
+        if (e != cudaSuccess)
+            return cuda_status(e);
+        g_scratch_addr[dev] = static_cast<double *>(p);
+    }
+    *out = g_scratch_addr[dev];
+    return BL_OK;
+}
+
+bool device_pointer(const void *p)
+{
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+}  // namespace
+
 }  // namespace bl
+
+extern "C" int bitlinear_pack_noalloc(const void *W, int wt, int64_t N, int64_t K,
+                                      uint8_t *packed, float *w_scale, void *stream)
+{
+    using namespace bl;
+    if (!W || !packed || !w_scale)
+        return BL_ERR_NULL;
+    if (wt != BL_F32 && wt != BL_BF16)
+        return BL_ERR_DTYPE;
+    if (N < 1 || K < 64 || K % 64 != 0 || K > (int64_t(1) << 22) || N > kNoAllocMaxRows)
+        return BL_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(W) & 15u) || (reinterpret_cast<uintptr_t>(packed) & 15u) ||
+        (reinterpret_cast<uintptr_t>(w_scale) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di = device_info();
+    if (!di)
+        return BL_ERR_CUDA;
+    if (di->cc_major != 10)
+        return BL_ERR_UNSUPPORTED;
+    if (!device_pointer(W) || !device_pointer(packed) || !device_pointer(w_scale))
+        return BL_ERR_NOT_DEVICE_PTR;
+    double *scratch = nullptr;
+    int st = scratch_address(&scratch);
+    if (st)
+        return st;
+    return launch_pack(W, wt, N, K, packed, w_scale, scratch, static_cast<cudaStream_t>(stream));
+}

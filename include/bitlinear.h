@@ -112,6 +112,32 @@ int bitlinear_pack(const void *W, int wt, int64_t N, int64_t K,
                    uint8_t *packed, float *w_scale, void *ws, size_t ws_bytes,
                    void *stream);
 
+/* Largest N that bitlinear_pack_noalloc accepts. */
+#define BITLINEAR_PACK_NOALLOC_MAX_ROWS 65536
+
+/*
+ * bitlinear_pack without a workspace argument: the same result, bit for bit,
+ * as bitlinear_pack, for callers that cannot allocate device memory at the
+ * time they pack weights -- for example a plain C host with no device
+ * allocator of its own, or a runtime whose memory pool already owns the GPU's
+ * memory, where a cudaMalloc would fail, fragment the pool or synchronise the
+ * device.  The pages have no counterpart of this entry point; it exists for
+ * such callers only.
+ *   W, wt, N, K, packed, w_scale, stream   as for bitlinear_pack
+ * Scratch: the per-row fp64 sums use a device array that lives inside the
+ * library, BITLINEAR_PACK_NOALLOC_MAX_ROWS doubles (512 KiB) on every GPU that
+ * loads the library, kept until the process exits.  N above
+ * BITLINEAR_PACK_NOALLOC_MAX_ROWS returns BL_ERR_SHAPE.  The first call on a
+ * device looks up that array's device address (once per device) and should
+ * come before any stream capture.  Every call on a device shares the array:
+ * calls whose work overlaps on the GPU (different streams with no ordering
+ * between them) race and may produce wrong scales.  Nothing in the array needs
+ * to start at zero, since every call writes each value it reads.  The call
+ * allocates nothing, and frees nothing.
+ */
+int bitlinear_pack_noalloc(const void *W, int wt, int64_t N, int64_t K,
+                           uint8_t *packed, float *w_scale, void *stream);
+
 /*
  * Per-token absmax int8 activation quantisation.  Source: "How to Run BitNet
  * Inference on GPU Using CUDA Kernels", section "Understanding the Two-Phase
