@@ -7,10 +7,17 @@ BitLinear products of a 2.4B-parameter BitNet b1.58 model -- per layer q/o
 (2560 -> 2560), k/v (2560 -> 640), gate/up (2560 -> 6912) and down
 (6912 -> 2560) -- for 30 layers, every product with its own packed ternary
 weight (521 MB of distinct weights per step, more than four times the 126 MB
-L2, so every step streams from HBM and no flush is needed).  Each product is
-one launch of the fused GEMV (absmax int8 quantisation of x, ternary product
-with int32 accumulation, rescale, bf16 out); the 210 launches of a step are
-replayed from a CUDA graph captured through the public Python API.
+L2, so every step streams from HBM and no flush is needed).  Each layer is
+four launches of the fused GEMV (absmax int8 quantisation of x, ternary
+product with int32 accumulation, rescale, bf16 out): q/k/v in one launch and
+gate/up in one, since each group shares its input, then o and down -- 120
+launches per step.  Each launch reads the output of the one before it, as in a
+decoder (o reads q, gate/up read o's output, down reads gate's output, the
+next layer reads down's output), so the chain is truly dependent; launches
+use programmatic dependent launch (a launch fetches its weights while the
+previous one finishes, and reads x only after it) and are replayed from a CUDA
+graph captured through the public Python API.  The end-to-end figure copies
+the token's input in and its final output back every step.
 
 Metric: effective weight bandwidth, packed weight bytes / device time, GB/s,
 against the measured HBM copy bandwidth.  Inputs are synthetic and seeded
@@ -44,7 +51,8 @@ import synth_inputs as si  # noqa: E402
 METRIC = "decode ternary GEMV effective weight GB/s (% of HBM peak); prefill int8 TOPS"
 WORKLOAD = ("decode GEMV M=1, BitNet b1.58 2.4B layer shapes (q/o 2560->2560, k/v 2560->640, "
             "gate/up 2560->6912, down 6912->2560) x 30 layers, distinct packed weights per "
-            "layer, fused int8 absmax quantisation, bf16 in/out")
+            "layer, fused int8 absmax quantisation, bf16 in/out; per layer 4 dependent launches "
+            "(qkv, o, gate+up, down; products sharing x fused) with programmatic dependent launch")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -154,40 +162,64 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- workload
 
+# One decoder layer's BitLinear launches: products that share their input are
+# fused into one launch (q/k/v; gate/up), as a decoder computes them.
+LAYER_LAUNCHES_2B = [("qkv", ["q", "k", "v"]), ("o", ["o"]), ("gate_up", ["gate", "up"]),
+                     ("down", ["down"])]
+
+
 def build_stream(bl, layers: int, seed: int, device):
-    """Pack distinct weights for every product of every layer; x and y buffers."""
+    """Pack distinct weights for every product of every layer and chain the
+    launches the way a decoder layer does: q/k/v read the layer input, o reads
+    q, gate/up read o's output, down reads gate's output, and the next layer
+    reads down's output.  Returns the launches, the token's input x0, the last
+    output, the host copy of x0 and the packed bytes per step."""
+    shapes = {name: (K, N) for (name, K, N) in si.LAYER_SHAPES_2B}
     gen = torch.Generator(device=device)
-    items = []
+    per_layer = []
     total_bytes = 0
     for layer in range(layers):
-        for j, (name, K, N) in enumerate(si.LAYER_SHAPES_2B):
-            gen.manual_seed(seed * 100003 + layer * 31 + j)
-            W = torch.randn(N, K, generator=gen, device=device, dtype=torch.float32) * 0.02
-            w = bl.pack(W)
-            del W
-            items.append((name, K, N, w))
-            total_bytes += w.packed.numel()
-    x_elems = sum(K for (_, K, _, _) in items)
-    y_elems = sum(N for (_, _, N, _) in items)
-    # all activations / outputs of a step live in one buffer each (one copy each way)
-    xs = torch.empty(x_elems, dtype=torch.bfloat16, device=device)
+        launches = []
+        for li, (lname, names) in enumerate(LAYER_LAUNCHES_2B):
+            ws = []
+            for j, name in enumerate(names):
+                K, N = shapes[name]
+                gen.manual_seed(seed * 100003 + layer * 31 + li * 7 + j)
+                W = torch.randn(N, K, generator=gen, device=device, dtype=torch.float32) * 0.02
+                ws.append(bl.pack(W))
+                del W
+                total_bytes += ws[-1].packed.numel()
+            launches.append(ws)
+        per_layer.append(launches)
+    y_elems = sum(w.N for launches in per_layer for ws in launches for w in ws)
     ys = torch.empty(y_elems, dtype=torch.bfloat16, device=device)
-    xo = yo = 0
-    views = []
-    for (name, K, N, w) in items:
-        views.append((w, xs[xo:xo + K].view(1, K), ys[yo:yo + N].view(1, N)))
-        xo += K
-        yo += N
-    host_x = torch.cat([si.activations(1, K, seed=seed + i).reshape(-1)
-                        for i, (_, K, _, _) in enumerate(items)])
-    xs.copy_(host_x)
+    x0 = torch.empty(1, si.HIDDEN_2B, dtype=torch.bfloat16, device=device)
+    chain = []
+    off = 0
+    h = x0
+    for launches in per_layer:
+        outs = []
+        for ws in launches:
+            o = []
+            for w in ws:
+                o.append(ys[off:off + w.N].view(1, w.N))
+                off += w.N
+            outs.append(o)
+        qkv, o_proj, gate_up, down = launches
+        chain.append((qkv, h, outs[0]))                 # q, k, v <- layer input
+        chain.append((o_proj, outs[0][0], outs[1]))     # o <- q
+        chain.append((gate_up, outs[1][0], outs[2]))    # gate, up <- o
+        chain.append((down, outs[2][0], outs[3]))       # down <- gate
+        h = outs[3][0]
+    host_x0 = si.activations(1, si.HIDDEN_2B, seed=seed)
+    x0.copy_(host_x0)
     torch.cuda.synchronize()
-    return items, views, xs, ys, host_x, total_bytes
+    return chain, x0, h, host_x0, total_bytes
 
 
-def run_step(bl, views):
-    for (w, x, y) in views:
-        bl.gemv_fused(w, x, out=y)
+def run_step(bl, launches, pdl=True):
+    for (ws, x, ys) in launches:
+        bl.gemv_fused_multi(ws, x, outs=ys, pdl=pdl)
 
 
 def time_graph(graph, steps, world):
@@ -385,15 +417,16 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", torch.cuda.current_device())
     hbm, bf16, bf16_sus, peak_kind = peaks()
 
-    items, views, xs, ys, host_x, step_bytes = build_stream(bl, args.layers, seed=rank, device=device)
-    launches_per_step = len(views)
+    launches, xs, ys, host_x, step_bytes = build_stream(bl, args.layers, seed=rank, device=device)
+    # xs: the token's input (copied in every e2e step); ys: its final output
+    launches_per_step = len(launches)
     # eager warm-up through the public API, then capture the step
     for _ in range(2):
-        run_step(bl, views)
+        run_step(bl, launches)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        run_step(bl, views)
+        run_step(bl, launches)
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
@@ -408,7 +441,7 @@ def run_ours(args, world, rank, local):
     # e2e: host activations in, host outputs back, every step, through the same
     # public-API launches (replayed from the graph captured above)
     pin_x = host_x.pin_memory()
-    pin_y = torch.empty(ys.numel(), dtype=ys.dtype).pin_memory()
+    pin_y = torch.empty(ys.shape, dtype=ys.dtype).pin_memory()
     for _ in range(3):
         xs.copy_(pin_x, non_blocking=True)
         graph.replay()
@@ -433,7 +466,7 @@ def run_ours(args, world, rank, local):
     s.record()
     for _ in range(eager_steps):
         xs.copy_(pin_x, non_blocking=True)
-        run_step(bl, views)
+        run_step(bl, launches)
         pin_y.copy_(ys, non_blocking=True)
     e.record()
     torch.cuda.synchronize()
@@ -476,15 +509,15 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": hbm, "unit": "GB/s",
                      "frac": value / world / hbm, "traffic": None,
                      "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                     "kernel": "gemv_kernel<1, bf16 fused>",
+                     "kernel": "gemv_kernel<1, bf16 fused> (4 launches per layer)",
                      "note": "algorithmic bytes = packed weight bytes per launch; duration = "
                              "step time / launches (CUDA events over the timed region)"},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "GB/s",
                 "h2d_bytes_per_step": xs.numel() * xs.element_size(),
                 "d2h_bytes_per_step": ys.numel() * ys.element_size(),
-                "how": "pinned host x -> device, graph of public-API gemv_fused calls, "
-                       "device y -> pinned host, CUDA events"},
+                "how": "pinned host token input -> device, graph of the public-API "
+                       "gemv_fused_multi chain, final output -> pinned host, CUDA events"},
         "e2e_eager_GBps": step_bytes * eager_steps / t_eager / 1e9,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,

@@ -76,6 +76,8 @@ _SIGNATURES = {
                               _vp, _vp]),
     "bitlinear_gemv_fused": (_int, [_vp, _vp, _i64, _i64, _vp, _int, _i64, _i64, _vp, _int,
                                     _i64, _vp, _vp]),
+    "bitlinear_gemv_fused_multi": (_int, [_int, _vp, _vp, _vp, _i64, _vp, _int, _i64, _i64,
+                                          _vp, _int, _vp, _vp, ctypes.c_uint, _vp]),
     "bitlinear_gemm_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bitlinear_gemm": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int, _i64,
                               _vp, _vp, _sz, _vp]),
@@ -212,6 +214,39 @@ def gemv_fused(w: TernaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16, out=
     return out
 
 
+GEMV_MAX_PROBLEMS = 8
+BL_FLAG_PDL = 1
+
+
+def gemv_fused_multi(weights, x: torch.Tensor, out_dtype=torch.bfloat16, outs=None,
+                     acc_dbgs=None, pdl: bool = False):
+    """Several decode BitLinears sharing the activations x, in one launch.
+
+    weights: list of TernaryWeight with the same K (q/k/v or gate/up of a layer).
+    pdl: allow the launch to overlap the preceding kernel's tail (programmatic
+    dependent launch); only when the weights were not written by that kernel.
+    """
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    n = len(weights)
+    M = x.shape[0]
+    if outs is None:
+        outs = [torch.empty(M, w.N, dtype=out_dtype, device=x.device) for w in weights]
+    P = ctypes.c_void_p * n
+    I64 = ctypes.c_int64 * n
+    packed = P(*[w.packed.data_ptr() for w in weights])
+    scales = P(*[w.w_scale.data_ptr() for w in weights])
+    Ns = I64(*[w.N for w in weights])
+    ys = P(*[o.data_ptr() for o in outs])
+    ldys = I64(*[o.stride(0) for o in outs])
+    accs = None if acc_dbgs is None else P(*[0 if a is None else a.data_ptr() for a in acc_dbgs])
+    _check(_lib.bitlinear_gemv_fused_multi(n, packed, scales, Ns, weights[0].K, _ptr(x),
+                                           _dt(x.dtype), x.stride(0), M, ys, _dt(outs[0].dtype),
+                                           ldys, accs, BL_FLAG_PDL if pdl else 0,
+                                           _stream(x.device)), "bitlinear_gemv_fused_multi")
+    return outs
+
+
 def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(_lib.bitlinear_gemm_workspace_bytes(M, N, K))
 
@@ -235,7 +270,7 @@ def gemm(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc
 def linear(w: TernaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16):
     """y = BitLinear(x): the fused GEMV for M <= 16 tokens, else quantise + GEMM."""
     x2 = x.reshape(-1, x.shape[-1])
-    if x2.shape[0] <= GEMV_MAX_M and x2.shape[0] * w.K <= 196608:
+    if x2.shape[0] <= GEMV_MAX_M and x2.shape[0] * w.K <= 163840:
         y = gemv_fused(w, x2, out_dtype)
     else:
         q, d, r = quantize_act(x2)

@@ -255,7 +255,7 @@ int check_gemv_common(const uint8_t *packed, const float *w_scale, int64_t N,
 }
 
 constexpr int64_t kGemvMaxM = 16;
-constexpr int64_t kGemvMaxMK = 196608;
+constexpr int64_t kGemvMaxMK = 163840;
 
 }  // namespace
 
@@ -305,6 +305,55 @@ int bitlinear_gemv_fused(const uint8_t *packed, const float *w_scale, int64_t N,
         return st;
     GemvArgs a{packed, w_scale, N, K, M, nullptr, nullptr, nullptr, x, xt, ldx, y, yt, ldy, acc_dbg};
     return launch_gemv(a, true, static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_gemv_fused_multi(int count, const uint8_t *const *packed,
+                               const float *const *w_scale, const int64_t *N, int64_t K,
+                               const void *x, int xt, int64_t ldx, int64_t M, void *const *y,
+                               int yt, const int64_t *ldy, int32_t *const *acc_dbg,
+                               unsigned flags, void *stream)
+{
+    if (!packed || !w_scale || !N || !y || !ldy || !x)
+        return BL_ERR_NULL;
+    if (count < 1 || count > kGemvMaxProblems)
+        return BL_ERR_SHAPE;
+    if (flags & ~BL_FLAG_PDL)
+        return BL_ERR_SHAPE;
+    if (!valid_dtype(xt) || !valid_dtype(yt))
+        return BL_ERR_DTYPE;
+    if (M * K > kGemvMaxMK || ldx < K)
+        return BL_ERR_SHAPE;
+    int st;
+    for (int i = 0; i < count; ++i) {
+        if ((st = check_gemv_common(packed[i], w_scale[i], N[i], K, M, y[i], yt, ldy[i],
+                                    kGemvMaxM)))
+            return st;
+        if (acc_dbg && (reinterpret_cast<uintptr_t>(acc_dbg[i]) & 3u))
+            return BL_ERR_ALIGN;
+    }
+    if (!aligned16(x) || (ldx * elem_bytes(xt)) % 16)
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    if ((st = need_device(&di)))
+        return st;
+    if ((st = check_dev_ptrs({x})))
+        return st;
+    GemvBatch b{};
+    b.count = count;
+    for (int i = 0; i < count; ++i) {
+        if ((st = check_dev_ptrs({packed[i], w_scale[i], y[i], acc_dbg ? acc_dbg[i] : nullptr})))
+            return st;
+        b.prob[i] = GemvProblem{packed[i], w_scale[i], N[i], y[i], ldy[i],
+                                acc_dbg ? acc_dbg[i] : nullptr};
+    }
+    b.K = K;
+    b.M = M;
+    b.x = x;
+    b.xt = xt;
+    b.ldx = ldx;
+    b.yt = yt;
+    b.flags = flags;
+    return launch_gemv_batch(b, true, static_cast<cudaStream_t>(stream));
 }
 
 size_t bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)

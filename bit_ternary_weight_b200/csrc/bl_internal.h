@@ -61,6 +61,34 @@ struct GemvArgs {
 
 int launch_gemv(const GemvArgs &a, bool fused, cudaStream_t s);
 
+// Several GEMVs that share their activations, in one launch.
+constexpr int kGemvMaxProblems = BITLINEAR_GEMV_MAX_PROBLEMS;
+
+struct GemvProblem {
+    const uint8_t *packed;
+    const float *w_scale;
+    int64_t N;
+    void *y;
+    int64_t ldy;
+    int32_t *acc_dbg;
+};
+
+struct GemvBatch {
+    int count;
+    GemvProblem prob[kGemvMaxProblems];
+    int64_t K, M;
+    const int8_t *q;        // pre-quantised activations (unfused), or
+    const float *d;
+    const int32_t *rowsum;
+    const void *x;          // raw activations (fused)
+    int xt;
+    int64_t ldx;
+    int yt;
+    unsigned flags;
+};
+
+int launch_gemv_batch(const GemvBatch &b, bool fused, cudaStream_t s);
+
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int launch_gemm(const GemvArgs &a, void *ws, size_t ws_bytes, cudaStream_t s);
 

@@ -7,26 +7,36 @@
 // integer inner loop, floating point only in the final scale multiply.
 //
 // Design (B200): the weight stream N*K/4 bytes is the whole cost.
-//   * Persistent grid, one or two 512-thread CTAs per SM.  Each CTA owns a
-//     contiguous range of 8-row groups, i.e. one contiguous byte range of the
-//     TL array, so the per-SM byte counts differ by at most one row group.
-//   * A row group's slab (K/64 chunks x 8 rows x 16 B) is split into 512-byte
-//     pieces; one warp-wide 16-byte load per lane reads one piece: lane l gets
-//     row l%8, chunk 4p + l/8.  Loads bypass L1 (read once) and are issued
-//     kUnroll pieces ahead of the math.
-//   * Teams of T warps share a row group (T chosen so that every warp of the
-//     grid has work); partial sums meet in shared memory behind a named
-//     barrier per team, double-buffered so there is one barrier per group.
-//   * The activations (int8, M*K bytes) sit in shared memory.  With the fused
-//     entry point the CTA quantises x itself in its prologue (absmax, scale,
-//     rint, row sum), so decode is one launch per BitLinear.
-//   * Inner loop: the stored codes s = code + 1 in {0,1,2} of four consecutive
-//     k are (word & (3 << 2i)) per byte; dp4a (unsigned x signed bytes) against
-//     four int8 activations gives 4^i * sum(s q).  For M <= 4 each of the four
-//     shifts keeps its own accumulator (one LOP3 + one dp4a per 4 weights per
-//     token), for M >= 8 the codes are shifted down once and shared by all
+//   * One launch may carry up to kGemvMaxProblems GEMVs that share the same
+//     activations x (the q/k/v or gate/up products of a decoder layer).  Their
+//     8-row groups are concatenated into one list.
+//   * Persistent grid of 512-thread CTAs: one per SM for small problems (so
+//     that the next launch's CTA fits beside it and can start its weight
+//     fetch early), two per SM for large ones.  Each CTA owns a contiguous
+//     range of row groups (host-computed), taken in phases of at most
+//     256 / M groups.  In a phase the 16 warps split the phase's 512-byte
+//     pieces into 16 contiguous runs that cross row-group boundaries; lane l
+//     of a warp always reads bytes 16l..16l+15 of a piece (row l%8, chunk
+//     4p + l/8 of the TL layout).
+//   * Weights stream through a per-warp ring of STAGES 512-byte slots in
+//     shared memory filled by cp.async (16 bytes per lane, L1 bypassed); each
+//     lane reads back only the bytes it copied, so no intra-warp sync is
+//     needed.  The ring is primed before the kernel waits on the preceding
+//     launch (programmatic dependent launch), so with BL_FLAG_PDL the weight
+//     fetch of one BitLinear overlaps the tail of the previous one.
+//   * The activations (int8, M*K bytes) sit in shared memory.  The fused
+//     entry points quantise x in the prologue (absmax, scale, rint, row sum;
+//     one register-resident pass for a single token).
+//   * Inner loop, stored codes s = code + 1 in {0,1,2}: for four consecutive
+//     k, (word & 0x03030303), (word & 0x0c0c0c0c), (word & 0x30303030) and
+//     (word & 0xc0c0c0c0) hold s, 4s, 16s, 64s per byte; dp4a (unsigned x
+//     signed bytes) against four int8 activations into four accumulators
+//     (two interleaved sets for one token) costs one LOP3 + one dp4a per four
+//     weights.  For M >= 8 the codes are shifted down once and shared by all
 //     tokens.  sum(code q) = sum(s q) - rowsum(q).
-//   * Epilogue: y = ((float)acc * d_m) * gamma_eff, bf16 or fp32.
+//   * At each row-group boundary a warp folds its partial sums into shared
+//     accumulators (warp shuffles + shared atomics); after the phase barrier
+//     y = ((float)acc * d_m) * gamma_eff is written, bf16 or fp32.
 #include "bl_common.cuh"
 
 namespace bl {
@@ -34,26 +44,33 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 4;
+
+// Bytes of the weight ring: STAGES 512-byte slots per warp.
+template <int STAGES>
+constexpr int ring_bytes() { return kWarps * STAGES * 512; }
 
 enum { MODE_Q = 0, MODE_X_BF16 = 1, MODE_X_F32 = 2 };
 
 struct Params {
-    const uint8_t *packed;
-    const float *w_scale;
-    int64_t N, K, NG;
+    GemvProblem prob[kGemvMaxProblems];
+    int64_t gstart[kGemvMaxProblems + 1];  // prefix sums of the problems' row groups
+    int count;
+    int64_t K;
     int M;
-    int T;  // warps per team: 1, 2, 4, 8 or 16
     const int8_t *q;
     const float *d;
     const int32_t *rowsum;
     const void *x;
     int64_t ldx;
-    void *y;
     int yt;
-    int64_t ldy;
-    int32_t *acc_dbg;
+    // CTA b owns row groups [b*gpc_base + min(b, gpc_rem), ...), gpc_base (+1) of them
+    int64_t gpc_base;
+    int gpc_rem;
 };
+
+// Row groups whose partial sums a CTA holds at once (8 KB of int32 sums).
+template <int MT>
+constexpr int groups_per_phase() { return 256 / MT; }
 
 template <int MT>
 struct Smem {
@@ -62,17 +79,108 @@ struct Smem {
     float scale[MT];
     float d[MT];
     int r[MT];
-    int red[2][kWarps][MT][8];
-    // followed by the int8 activations, M*K bytes, 16-byte aligned
+    int sacc[groups_per_phase<MT>()][MT][8];
+    // followed by the weight ring and the int8 activations (M*K)
 };
 
 template <int MT>
 constexpr size_t smem_header()
 {
-    return (sizeof(Smem<MT>) + 15) / 16 * 16;
+    return (sizeof(Smem<MT>) + 127) / 128 * 128;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void *g)
+{
+    asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(saddr), "l"(g)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t saddr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(saddr));
+    return v;
+}
+
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Problem and local row group of concatenated row group G.
+__device__ __forceinline__ int locate(const Params &p, int64_t G, int64_t &g_local)
+{
+    int pi = 0;
+#pragma unroll
+    for (int i = 1; i < kGemvMaxProblems; ++i)
+        if (i < p.count && G >= p.gstart[i])
+            pi = i;
+    g_local = G - p.gstart[pi];
+    return pi;
 }
 
 // Quantise the M tokens of x into shared memory (block-cooperative).
+// One token whose K/8 eight-element chunks fit two per thread: x is read once
+// into registers, one block reduction gives the absmax, the quantised values
+// go to shared memory and each warp leaves its partial row sum in bsum (the
+// epilogue adds them up), so the prologue needs a single barrier.
+template <int MT, int XT>
+__device__ __forceinline__ void quantize_prologue_1(const Params &p, Smem<MT> &sm, int8_t *qs)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int chunks = int(p.K / 8);
+    float f[2][8];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int c = tid + i * kThreads;
+        if (c < chunks) {
+            load8<XT>(p.x, int64_t(c) * 8, f[i]);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                amax = fmaxf(amax, fabsf(f[i][j]));
+        }
+    }
+    amax = warp_max(amax);
+    if (lane == 0)
+        sm.bmax[warp][0] = amax;
+    __syncthreads();
+    float a = sm.bmax[0][0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w)
+        a = fmaxf(a, sm.bmax[w][0]);
+    const float a_eff = fmaxf(a, kEps);
+    const float s = __fdiv_rn(kQb, a_eff);
+    if (tid == 0)
+        sm.d[0] = __fdiv_rn(a_eff, kQb);
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int c = tid + i * kThreads;
+        if (c < chunks) {
+            uint32_t lo = 0, hi = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int t0 = quant1(f[i][j], s), t1 = quant1(f[i][j + 4], s);
+                sum += t0 + t1;
+                lo |= (uint32_t(t0) & 0xffu) << (8 * j);
+                hi |= (uint32_t(t1) & 0xffu) << (8 * j);
+            }
+            *reinterpret_cast<uint2 *>(qs + int64_t(c) * 8) = make_uint2(lo, hi);
+        }
+    }
+    sum = warp_sum(sum);
+    if (lane == 0)
+        sm.bsum[warp][0] = sum;
+    // the barrier before the main loop publishes qs, d and bsum
+}
+
 template <int MT, int XT>
 __device__ __forceinline__ void quantize_prologue(const Params &p, Smem<MT> &sm, int8_t *qs)
 {
@@ -156,83 +264,184 @@ __device__ __forceinline__ void copy_prologue(const Params &p, Smem<MT> &sm, int
         sm.d[threadIdx.x] = p.d[threadIdx.x];
         sm.r[threadIdx.x] = p.rowsum[threadIdx.x];
     }
+    // the epilogue reads row sums as the sum over warps of bsum
+    for (int i = threadIdx.x; i < kWarps * MT; i += kThreads) {
+        const int w = i / MT, m = i % MT;
+        sm.bsum[w][m] = (w == 0 && m < p.M) ? p.rowsum[m] : 0;
+    }
     __syncthreads();
 }
 
-template <int MT>
-__device__ __forceinline__ void epilogue(const Params &p, const Smem<MT> &sm, float gamma,
-                                         int64_t g, int rr, int m, int total)
+// Work of one CTA: the row groups [g_begin, g_end), taken in phases of at
+// most groups_per_phase<MT>() groups.  In a phase the 16 warps split the
+// phase's 512-byte pieces into 16 contiguous runs; a warp streams its run
+// through its cp.async ring, crossing row-group boundaries, and at each
+// boundary (and at the end of its run) adds its partial row sums into the
+// phase's shared accumulators.  After a barrier the phase's rows are rescaled
+// and written.  The first ring fill is issued before the kernel waits on the
+// preceding launch, so the weight stream starts at once.
+template <int MT, int MODE, bool FULL, int STAGES>
+__global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p)
 {
-    const int64_t n = g * 8 + rr;
-    if (n >= p.N)
-        return;
-    const int a = total - sm.r[m];
-    if (p.acc_dbg)
-        p.acc_dbg[int64_t(m) * p.N + n] = a;
-    store_y(p.y, p.yt, int64_t(m) * p.ldy + n, rescale1(a, sm.d[m], gamma));
-}
-
-template <int MT, int MODE, int MINB>
-__global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const Params p)
-{
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+    extern __shared__ __align__(128) unsigned char smem_raw[];
     Smem<MT> &sm = *reinterpret_cast<Smem<MT> *>(smem_raw);
-    int8_t *qs = reinterpret_cast<int8_t *>(smem_raw + smem_header<MT>());
+    const uint32_t ring0 = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw + smem_header<MT>()));
+    int8_t *qs = reinterpret_cast<int8_t *>(smem_raw + smem_header<MT>() + ring_bytes<STAGES>());
+    const uint32_t qs_addr = static_cast<uint32_t>(__cvta_generic_to_shared(qs));
+    constexpr bool kMask = MT <= 4;
+    // two interleaved accumulator sets (even / odd words) halve the dp4a
+    // dependency chains when there are few tokens
+    constexpr int kSets = MT == 1 ? 2 : 1;
+    constexpr int kAcc = kMask ? 4 * kSets : 1;
+    constexpr int GP = groups_per_phase<MT>();
 
-    if constexpr (MODE == MODE_Q)
-        copy_prologue<MT>(p, sm, qs);
-    else if constexpr (MODE == MODE_X_BF16)
-        quantize_prologue<MT, BL_BF16>(p, sm, qs);
-    else
-        quantize_prologue<MT, BL_F32>(p, sm, qs);
-
-    constexpr bool kMaskVariant = MT <= 4;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int T = p.T, nteams = kWarps / T, team = warp / T, wt = warp % T;
-    const int64_t C = p.K / 64, P = (C + 3) / 4, slab = C * 128;
+    const int Ki = int(p.K);
+    const int C = Ki / 64, P = (C + 3) / 4;
+    const int64_t slab = int64_t(C) * 128;
     const int csub = lane >> 3;
-    const float gamma = p.w_scale[0];
-    const int64_t g_begin = int64_t(blockIdx.x) * p.NG / gridDim.x;
-    const int64_t g_end = int64_t(blockIdx.x + 1) * p.NG / gridDim.x;
-    int parity = 0;
+    const int64_t NGt = p.gstart[p.count];
+    const int bx = blockIdx.x;
+    const int64_t g_begin = bx * p.gpc_base + (bx < p.gpc_rem ? bx : p.gpc_rem);
+    const int64_t g_end = g_begin + p.gpc_base + (bx < p.gpc_rem ? 1 : 0);
+    const uint32_t ring = ring0 + uint32_t(warp) * (STAGES * 512) + lane * 16;
 
-    for (int64_t g = g_begin + team; g < g_end; g += nteams) {
-        int acc[MT][kMaskVariant ? 4 : 1];
+    auto group_ptr = [&](int64_t G) -> const uint8_t * {
+        int64_t gl;
+        const int pi = locate(p, G, gl);
+        return p.prob[pi].packed + gl * slab + lane * 16;
+    };
+
+    // this lane's slot 0 of its warp's ring, as a generic pointer for the
+    // loads (slot offsets then become immediates) and as a shared address for
+    // cp.async
+    const unsigned char *ring_g = smem_raw + smem_header<MT>() + warp * (STAGES * 512) + lane * 16;
+
+    // issue cursor (runs STAGES pieces ahead of the math)
+    int64_t i_group = 0;
+    int i_j = 0, i_left = 0, i_rem = 0;
+    const uint8_t *i_ptr = nullptr;
+    // With K % 256 == 0 (FULL) a problem's pieces are one contiguous byte
+    // stream, so the cursor only jumps when it moves on to the next problem.
+    int i_prob = 0;
+    int64_t i_to_jump = 0;
+    auto issue = [&](int slot) {
+        if (i_rem > 0) {
+            if constexpr (FULL) {
+                cp_async16(ring + slot * 512, i_ptr);
+                i_ptr += 512;
+                --i_rem;
+                if (--i_to_jump == 0 && i_rem > 0) {
+                    ++i_prob;
+                    i_ptr = p.prob[i_prob].packed + lane * 16;
+                    i_to_jump = (p.gstart[i_prob + 1] - p.gstart[i_prob]) * P;
+                }
+            } else {
+                if (4 * i_j + csub < C)
+                    cp_async16(ring + slot * 512, i_ptr);
+                --i_rem;
+                ++i_j;
+                i_ptr += 512;
+                if (--i_left == 0) {
+                    ++i_group;
+                    i_left = P;
+                    i_j = 0;
+                    if (i_rem > 0)
+                        i_ptr = group_ptr(i_group);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+    int acc[MT][kAcc];
+    // end of a row group, or of this warp's run: fold into the shared sums
+    auto flush = [&](int gi) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            int t;
+            if constexpr (kMask) {
+                t = 0;
+#pragma unroll
+                for (int b = 0; b < 4 * kSets; b += 4)
+                    t += acc[m][b] + (acc[m][b + 1] >> 2) + (acc[m][b + 2] >> 4) +
+                         (acc[m][b + 3] >> 6);
+            } else {
+                t = acc[m][0];
+            }
+#pragma unroll
+            for (int a = 0; a < kAcc; ++a)
+                acc[m][a] = 0;
+            t += __shfl_xor_sync(0xffffffffu, t, 8);
+            t += __shfl_xor_sync(0xffffffffu, t, 16);
+            if (lane < 8 && m < p.M)
+                atomicAdd(&sm.sacc[gi][m][lane], t);
+        }
+    };
+
+    bool first = true;
+    for (int64_t ph0 = g_begin; ph0 < g_end; ph0 += GP) {
+        const int64_t ph1 = ph0 + GP < g_end ? ph0 + GP : g_end;
+        const int nG = int(ph1 - ph0);
+        const int64_t TP = int64_t(nG) * P;
+        // kWarps is a power of two: the split needs no division
+        const int wb = int((int64_t(warp) * TP) >> 4);
+        const int n = int((int64_t(warp + 1) * TP) >> 4) - wb;
+        const int gi0 = wb / P, j0 = wb - gi0 * P;
+        static_assert(kWarps == 16, "the run split above assumes 16 warps");
+
+        i_group = ph0 + gi0;
+        i_j = j0;
+        i_left = P - j0;
+        i_rem = n;
+        i_ptr = n > 0 ? group_ptr(i_group) + int64_t(j0) * 512 : nullptr;
+        if constexpr (FULL) {
+            int64_t gl;
+            i_prob = locate(p, i_group, gl);
+            i_to_jump = (p.gstart[i_prob + 1] - i_group) * P - j0;
+        }
+        if (first)
+            pdl_launch_dependents();
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s)
+            issue(s);
+        if (first) {
+            // everything below may read what the preceding launch wrote
+            pdl_wait();
+            if constexpr (MODE == MODE_Q)
+                copy_prologue<MT>(p, sm, qs);
+            else if (MT == 1 && p.K <= int64_t(16) * kThreads)
+                quantize_prologue_1<MT, MODE == MODE_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
+            else
+                quantize_prologue<MT, MODE == MODE_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
+            first = false;
+        }
+        for (int i = tid; i < nG * MT * 8; i += kThreads)
+            (&sm.sacc[0][0][0])[i] = 0;
+        __syncthreads();
+
 #pragma unroll
         for (int m = 0; m < MT; ++m)
 #pragma unroll
-            for (int i = 0; i < (kMaskVariant ? 4 : 1); ++i)
-                acc[m][i] = 0;
-        const uint8_t *sp = p.packed + g * slab + lane * 16;
-
-        for (int64_t p0 = wt; p0 < P; p0 += int64_t(T) * kUnroll) {
-            uint4 wv[kUnroll];
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int64_t pp = p0 + int64_t(u) * T;
-                const int64_t c = 4 * pp + csub;
-                wv[u] = (pp < P && c < C) ? ld_stream_v4(sp + pp * 512) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int64_t pp = p0 + int64_t(u) * T;
-                const int64_t c = 4 * pp + csub;
-                if (!(pp < P && c < C))
-                    continue;
-                const uint32_t wd[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
-                if constexpr (kMaskVariant) {
+            for (int a = 0; a < kAcc; ++a)
+                acc[m][a] = 0;
+        // multiply one 16-byte piece (wv, this lane's 64 k of one row) into
+        // the accumulators against the activations at qp
+        auto mac = [&](const uint4 wv, const int8_t *qp) {
+                const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+                if constexpr (kMask) {
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
                         if (m >= p.M)
                             break;
-                        const uint4 *qp = reinterpret_cast<const uint4 *>(qs + m * p.K + c * 64);
+                        const uint4 *q4p = reinterpret_cast<const uint4 *>(qp + m * Ki);
 #pragma unroll
                         for (int w = 0; w < 4; ++w) {
-                            const uint4 q4 = qp[w];
-                            acc[m][0] = dp4a_us(wd[w] & 0x03030303u, q4.x, acc[m][0]);
-                            acc[m][1] = dp4a_us(wd[w] & 0x0c0c0c0cu, q4.y, acc[m][1]);
-                            acc[m][2] = dp4a_us(wd[w] & 0x30303030u, q4.z, acc[m][2]);
-                            acc[m][3] = dp4a_us(wd[w] & 0xc0c0c0c0u, q4.w, acc[m][3]);
+                            const uint4 q4 = q4p[w];
+                            const int b = 4 * (w % kSets);
+                            acc[m][b + 0] = dp4a_us(wd[w] & 0x03030303u, q4.x, acc[m][b + 0]);
+                            acc[m][b + 1] = dp4a_us(wd[w] & 0x0c0c0c0cu, q4.y, acc[m][b + 1]);
+                            acc[m][b + 2] = dp4a_us(wd[w] & 0x30303030u, q4.z, acc[m][b + 2]);
+                            acc[m][b + 3] = dp4a_us(wd[w] & 0xc0c0c0c0u, q4.w, acc[m][b + 3]);
                         }
                     }
                 } else {
@@ -246,8 +455,7 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const Params p)
                         for (int m = 0; m < MT; ++m) {
                             if (m >= p.M)
                                 break;
-                            const uint4 q4 =
-                                reinterpret_cast<const uint4 *>(qs + m * p.K + c * 64)[w];
+                            const uint4 q4 = reinterpret_cast<const uint4 *>(qp + m * Ki)[w];
                             int a = acc[m][0];
                             a = dp4a_us(c0, q4.x, a);
                             a = dp4a_us(c1, q4.y, a);
@@ -257,122 +465,172 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const Params p)
                         }
                     }
                 }
-            }
-        }
+                    };
 
-        int tot[MT];
+        int c_gi = gi0, c_j = j0, c_left = P - j0;
+        const int8_t *qp = qs + j0 * 256 + csub * 64;
+        for (int k0 = 0; k0 < n; k0 += STAGES) {
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            if constexpr (kMaskVariant)
-                tot[m] = acc[m][0] + (acc[m][1] >> 2) + (acc[m][2] >> 4) + (acc[m][3] >> 6);
-            else
-                tot[m] = acc[m][0];
-            tot[m] += __shfl_xor_sync(0xffffffffu, tot[m], 8);
-            tot[m] += __shfl_xor_sync(0xffffffffu, tot[m], 16);
-        }
-        if (T == 1) {
-            if (lane < 8) {
-#pragma unroll
-                for (int m = 0; m < MT; ++m)
-                    if (m < p.M)
-                        epilogue<MT>(p, sm, gamma, g, lane, m, tot[m]);
-            }
-        } else {
-            if (lane < 8) {
-#pragma unroll
-                for (int m = 0; m < MT; ++m)
-                    if (m < p.M)
-                        sm.red[parity][warp][m][lane] = tot[m];
-            }
-            named_barrier(1 + team, T * 32);
-            if (wt == 0) {
-                for (int idx = lane; idx < p.M * 8; idx += 32) {
-                    const int m = idx >> 3, rr = idx & 7;
-                    int s = 0;
-                    for (int t = 0; t < T; ++t)
-                        s += sm.red[parity][team * T + t][m][rr];
-                    epilogue<MT>(p, sm, gamma, g, rr, m, s);
+            for (int u = 0; u < STAGES; ++u) {
+                if (k0 + u >= n)
+                    break;
+                cp_async_wait<STAGES - 1>();
+                const uint4 wv = *reinterpret_cast<const uint4 *>(ring_g + u * 512);
+                if (FULL || 4 * c_j + csub < C)
+                    mac(wv, qp);
+                // the slot's data has been consumed: refill it
+                issue(u);
+                qp += 256;
+                if constexpr (!FULL)
+                    ++c_j;
+                if (--c_left == 0) {
+                    flush(c_gi);
+                    ++c_gi;
+                    c_left = P;
+                    c_j = 0;
+                    qp = qs + csub * 64;
                 }
             }
-            parity ^= 1;
         }
+        if (n > 0 && c_left != P)
+            flush(c_gi);  // the run ended inside a group
+        cp_async_wait<0>();
+        __syncthreads();
+        // rescale and write the phase's rows
+        for (int idx = tid; idx < nG * 8 * p.M; idx += kThreads) {
+            const int gi = idx / (8 * p.M), rem = idx % (8 * p.M);
+            const int m = rem >> 3, rr = rem & 7;
+            int64_t gl;
+            const int pi = locate(p, ph0 + gi, gl);
+            const GemvProblem &pr = p.prob[pi];
+            const int64_t row = gl * 8 + rr;
+            if (row < pr.N) {
+                int r = 0;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w)
+                    r += sm.bsum[w][m];
+                const int a = sm.sacc[gi][m][rr] - r;
+                if (pr.acc_dbg)
+                    pr.acc_dbg[int64_t(m) * pr.N + row] = a;
+                store_y(pr.y, p.yt, int64_t(m) * pr.ldy + row, rescale1(a, sm.d[m], pr.w_scale[0]));
+            }
+        }
+        __syncthreads();
+    }
+    if (first) {
+        // a CTA with no rows still honours the launch order
+        pdl_launch_dependents();
+        pdl_wait();
     }
 }
 
+
 template <int MT, int MODE>
-int launch_one(const Params &base, cudaStream_t s)
+int launch_one(const Params &base, unsigned flags, cudaStream_t s)
 {
-    constexpr int kMinBlocks = MT <= 4 ? 2 : 1;
-    auto kern = gemv_kernel<MT, MODE, kMinBlocks>;
     const DeviceInfo *di = device_info();
     if (!di)
         return BL_ERR_CUDA;
-    const size_t smem = smem_header<MT>() + size_t(base.M) * size_t(base.K);
+    const bool full = (base.K / 64) % 4 == 0;
+    const size_t act = size_t(base.M) * size_t(base.K);
+    // a deep ring while two CTAs (this launch and the next one) still fit on
+    // an SM, a shallow one for large activation tiles
+    const bool deep = smem_header<MT>() + ring_bytes<8>() + act <= 100 * 1024;
+    const size_t smem = smem_header<MT>() + (deep ? ring_bytes<8>() : ring_bytes<4>()) + act;
     if (smem > size_t(di->max_smem_optin))
         return BL_ERR_SHAPE;
+    auto kern = deep ? (full ? gemv_kernel<MT, MODE, true, 8> : gemv_kernel<MT, MODE, false, 8>)
+                     : (full ? gemv_kernel<MT, MODE, true, 4> : gemv_kernel<MT, MODE, false, 4>);
     int per_sm = 0;
     int st = occupancy(reinterpret_cast<const void *>(kern), kThreads, smem, &per_sm);
     if (st)
         return st;
     if (per_sm < 1)
         return BL_ERR_SHAPE;
-    Params p = base;
-    const int64_t warps_total = int64_t(di->sm_count) * per_sm * kWarps;
-    const int64_t P = (p.K / 64 + 3) / 4;
-    int tmax = 1;
-    while (tmax * 2 <= kWarps && tmax * 2 <= P)
-        tmax *= 2;
-    int T = 1;
-    while (T < tmax && p.NG * T < warps_total)
-        T *= 2;
-    p.T = T;
-    const int nteams = kWarps / T;
-    const int64_t want = (p.NG + nteams - 1) / nteams;
-    const int64_t grid = want < int64_t(di->sm_count) * per_sm ? want : int64_t(di->sm_count) * per_sm;
-    kern<<<unsigned(grid), kThreads, smem, s>>>(p);
-    return launch_status();
+    // one persistent CTA per SM (a second slot stays free for the next launch)
+    const int64_t NGt = base.gstart[base.count];
+    // large problems: up to two CTAs per SM for more warps in flight; small
+    // ones keep one so that the next launch's CTA fits beside it
+    const int64_t per = NGt >= 4 * int64_t(di->sm_count) && per_sm >= 2 ? 2 : 1;
+    const int64_t cap = int64_t(di->sm_count) * per;
+    const unsigned grid = unsigned(NGt < cap ? NGt : cap);
+    Params pp = base;
+    pp.gpc_base = NGt / grid;
+    pp.gpc_rem = int(NGt % grid);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    if (flags & BL_FLAG_PDL) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, pp));
 }
 
 template <int MODE>
-int dispatch_m(const Params &p, cudaStream_t s)
+int dispatch_m(const Params &p, unsigned flags, cudaStream_t s)
 {
     if (p.M <= 1)
-        return launch_one<1, MODE>(p, s);
+        return launch_one<1, MODE>(p, flags, s);
     if (p.M <= 2)
-        return launch_one<2, MODE>(p, s);
+        return launch_one<2, MODE>(p, flags, s);
     if (p.M <= 4)
-        return launch_one<4, MODE>(p, s);
+        return launch_one<4, MODE>(p, flags, s);
     if (p.M <= 8)
-        return launch_one<8, MODE>(p, s);
-    return launch_one<16, MODE>(p, s);
+        return launch_one<8, MODE>(p, flags, s);
+    return launch_one<16, MODE>(p, flags, s);
 }
 
 }  // namespace
 
-int launch_gemv(const GemvArgs &a, bool fused, cudaStream_t s)
+int launch_gemv_batch(const GemvBatch &b, bool fused, cudaStream_t s)
 {
     Params p{};
-    p.packed = a.packed;
-    p.w_scale = a.w_scale;
-    p.N = a.N;
-    p.K = a.K;
-    p.NG = (a.N + 7) / 8;
-    p.M = int(a.M);
-    p.T = 1;
-    p.q = a.q;
-    p.d = a.d;
-    p.rowsum = a.rowsum;
-    p.x = a.x;
-    p.ldx = a.ldx;
-    p.y = a.y;
-    p.yt = a.yt;
-    p.ldy = a.ldy;
-    p.acc_dbg = a.acc_dbg;
+    p.count = b.count;
+    p.gstart[0] = 0;
+    for (int i = 0; i < b.count; ++i) {
+        p.prob[i] = b.prob[i];
+        p.gstart[i + 1] = p.gstart[i] + (b.prob[i].N + 7) / 8;
+    }
+    for (int i = b.count; i < kGemvMaxProblems; ++i)
+        p.gstart[i + 1] = p.gstart[b.count];
+    p.K = b.K;
+    p.M = int(b.M);
+    p.q = b.q;
+    p.d = b.d;
+    p.rowsum = b.rowsum;
+    p.x = b.x;
+    p.ldx = b.ldx;
+    p.yt = b.yt;
     if (!fused)
-        return dispatch_m<MODE_Q>(p, s);
-    if (a.xt == BL_BF16)
-        return dispatch_m<MODE_X_BF16>(p, s);
-    return dispatch_m<MODE_X_F32>(p, s);
+        return dispatch_m<MODE_Q>(p, b.flags, s);
+    if (b.xt == BL_BF16)
+        return dispatch_m<MODE_X_BF16>(p, b.flags, s);
+    return dispatch_m<MODE_X_F32>(p, b.flags, s);
+}
+
+int launch_gemv(const GemvArgs &a, bool fused, cudaStream_t s)
+{
+    GemvBatch b{};
+    b.count = 1;
+    b.prob[0] = GemvProblem{a.packed, a.w_scale, a.N, a.y, a.ldy, a.acc_dbg};
+    b.K = a.K;
+    b.M = a.M;
+    b.q = a.q;
+    b.d = a.d;
+    b.rowsum = a.rowsum;
+    b.x = a.x;
+    b.xt = a.xt;
+    b.ldx = a.ldx;
+    b.yt = a.yt;
+    b.flags = 0;
+    return launch_gemv_batch(b, fused, s);
 }
 
 }  // namespace bl

@@ -160,7 +160,7 @@ int bitlinear_quantize_act(const void *x, int xt, int64_t M, int64_t K,
  *   q, d, rowsum      from bitlinear_quantize_act (device), q is [M][K]
  *   y                 device, [M][ldy] of dtype yt (BL_F32 or BL_BF16), ldy >= N
  *   acc_dbg           NULL, or device [M][N] int32 receiving acc (before rescale)
- * M * K must not exceed 196608 (the activations are staged on chip).
+ * M * K must not exceed 163840 (the activations are staged on chip).
  */
 int bitlinear_gemv(const uint8_t *packed, const float *w_scale, int64_t N,
                    int64_t K, const int8_t *q, const float *d,
@@ -177,6 +177,41 @@ int bitlinear_gemv_fused(const uint8_t *packed, const float *w_scale,
                          int64_t N, int64_t K, const void *x, int xt,
                          int64_t ldx, int64_t M, void *y, int yt, int64_t ldy,
                          int32_t *acc_dbg, void *stream);
+
+/* Most GEMVs one bitlinear_gemv_fused_multi call may carry. */
+#define BITLINEAR_GEMV_MAX_PROBLEMS 8
+
+/* Launch flag: the kernel may start while the work before it in the stream is
+ * still running, and fetch its packed weights early (programmatic dependent
+ * launch).  It still waits for that work to finish before it reads x or
+ * writes anything, so a chain of dependent BitLinears stays correct.  The
+ * caller promises that the packed weights and scales were not written by the
+ * kernel immediately before this call in the stream. */
+#define BL_FLAG_PDL 1u
+
+/*
+ * Decode BitLinear for `count` weights that share the same activations x
+ * (for instance the q, k and v products, or the gate and up products, of one
+ * decoder layer), quantising x once and running all products in one launch.
+ * Source: "How to Run BitNet Inference on GPU Using CUDA Kernels", sections
+ * "Understanding the Two-Phase Architecture" (Attention and FeedForward use the
+ * BitLinear kernel) and "Key Components and Source Code Architecture" (CUDA
+ * graphs to remove launch overhead in decode).
+ *   count            1 .. BITLINEAR_GEMV_MAX_PROBLEMS
+ *   packed[i], w_scale[i], N[i]   the i-th packed weight (all share K)
+ *   x, xt, ldx, M    as for bitlinear_gemv_fused (1 <= M <= 16)
+ *   y[i], ldy[i]     device outputs [M][ldy[i]] of dtype yt
+ *   acc_dbg          NULL, or a host array of `count` device pointers (each
+ *                    NULL or [M][N[i]] int32)
+ *   flags            0 or BL_FLAG_PDL
+ * The pointer arrays are host memory, read during the call only.
+ */
+int bitlinear_gemv_fused_multi(int count, const uint8_t *const *packed,
+                               const float *const *w_scale, const int64_t *N,
+                               int64_t K, const void *x, int xt, int64_t ldx,
+                               int64_t M, void *const *y, int yt,
+                               const int64_t *ldy, int32_t *const *acc_dbg,
+                               unsigned flags, void *stream);
 
 /* Bytes of workspace bitlinear_gemm needs for this problem (0 if none). */
 size_t bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);

@@ -158,7 +158,7 @@ def test_decode_gemv_100b_shapes(bl, K, N):
 
 
 @pytest.mark.parametrize("N,K,M", [(13, 64, 1), (1001, 192, 3), (8, 128, 16), (77, 320, 5),
-                                   (1, 64, 2), (4096, 64, 7), (24, 12288, 16)])
+                                   (1, 64, 2), (4096, 64, 7), (24, 10240, 16)])
 @pytest.mark.parametrize("fused", [True, False])
 def test_gemv_ragged_and_edge(bl, N, K, M, fused):
     W, x = seeded_problem(N, K, M, seed=N * 7 + K + M)
@@ -267,3 +267,54 @@ def test_gemm_prefill_full_size(bl, K, N, M):
     rng = np.random.default_rng(M + K)
     sample = np.unique(np.concatenate([[0, M - 1, 127, 128], rng.integers(0, M, 60)]))
     _check_gemm(bl, N, K, M, seed=3, sample=sample)
+
+
+# ------------------------------------------------------------------ shared-input multi GEMV, PDL chains
+
+@pytest.mark.parametrize("M", [1, 3, 16])
+def test_multi_gemv_qkv_shapes(bl, M):
+    """q/k/v of one 2.4B layer in one launch, each output against the oracle."""
+    K = si.HIDDEN_2B
+    shapes = [si.HIDDEN_2B, si.KV_2B, si.KV_2B]
+    x = si.activations(M, K, seed=40 + M)
+    ws, refs = [], []
+    for i, N in enumerate(shapes):
+        W = si.weight(N, K, seed=50 + i)
+        g, codes, _ = oracle_weight(W)
+        refs.append(_oracle_gemv(g, codes, x))
+        ws.append(_pack_gpu(bl, W))
+    accs = [torch.empty(M, N, dtype=torch.int32, device=dev()) for N in shapes]
+    outs = bl.gemv_fused_multi(ws, x.to(dev()), acc_dbgs=accs)
+    torch.cuda.synchronize()
+    for (y_o, acc_o), y, acc in zip(refs, outs, accs):
+        np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+        compare_outputs(y, y_o)
+
+
+def test_pdl_dependent_chain(bl):
+    """A chain where each launch reads the previous launch's output, all with
+    BL_FLAG_PDL, inside a CUDA graph: the result must equal the oracle chain."""
+    K = 2560
+    Ws = [si.weight(K, K, seed=70 + i) for i in range(6)]
+    oracles = [oracle_weight(W) for W in Ws]
+    ws = [_pack_gpu(bl, W) for W in Ws]
+    x0 = si.activations(1, K, seed=77)
+    xs = [x0.to(dev())] + [torch.empty(1, K, dtype=torch.bfloat16, device=dev()) for _ in Ws]
+    for _ in range(2):  # warm-up, eager
+        for i, w in enumerate(ws):
+            bl.gemv_fused_multi([w], xs[i], outs=[xs[i + 1]], pdl=True)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i, w in enumerate(ws):
+            bl.gemv_fused_multi([w], xs[i], outs=[xs[i + 1]], pdl=True)
+    for i in range(1, len(xs)):
+        xs[i].zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    x = x0
+    for i, (gam, codes, _) in enumerate(oracles):
+        y_o, _ = _oracle_gemv(gam, codes, x)
+        compare_outputs(xs[i + 1], y_o)
+        x = torch.from_numpy(oracle.to_bf16_bits(y_o).view(np.int16)).view(torch.bfloat16)
+    assert bl.last_device_status() == 0
