@@ -68,6 +68,25 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+def profiled_traffic():
+    """DRAM bytes per GEMV launch from the committed ncu summary, or None when
+    the kernel source has changed since those counters were taken."""
+    import hashlib
+    import re
+    prof = os.path.join(ROOT, "profiles", "decode_stream_2b_gemv_launches.md")
+    src = os.path.join(ROOT, "bit_ternary_weight_b200", "csrc", "gemv.cu")
+    try:
+        text = open(prof).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        m = re.search(r"sha256 prefix `([0-9a-f]+)`", text)
+        t = re.search(r"traffic_per_launch_bytes: (\d+)", text)
+        if m and t and sha.startswith(m.group(1)):
+            return int(t.group(1))
+    except OSError:
+        pass
+    return None
+
+
 # ---------------------------------------------------------------- distributed
 
 def dist_init(n_gpus: int):
@@ -507,7 +526,7 @@ def run_ours(args, world, rank, local):
                    "l2": "inputs larger than L2: 521 MB of distinct packed weights per step",
                    "parallelism": f"{world} independent replicas (weak scaling)"},
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": hbm, "unit": "GB/s",
-                     "frac": value / world / hbm, "traffic": None,
+                     "frac": value / world / hbm, "traffic": profiled_traffic(),
                      "peak_kind": f"{peak_kind} HBM copy bandwidth",
                      "kernel": "gemv_kernel<1, bf16 fused> (4 launches per layer)",
                      "note": "algorithmic bytes = packed weight bytes per launch; duration = "
