@@ -10,8 +10,9 @@
 // unsigned stored values by the signed activations; the epilogue subtracts the
 // row sum and rescales.
 //
-// Tile: 128 weight rows (MMA M) x 128 tokens (MMA N), 128 k per stage, four
-// stages.  Operands:
+// Persistent kernel, one CTA per SM, walking output tiles of 128 weight rows
+// (MMA M) x 128 tokens (MMA N); k advances 128 per pipeline stage through an
+// eight-slot ring.  Operands:
 //   A (weights)  TL bytes of the tile arrive in shared memory by TMA (a 2-D
 //                view [row groups][K/64 * 128 B], box 16 groups x 256 B); four
 //                expansion warps turn each thread's row (one TMEM lane) into
@@ -20,17 +21,30 @@
 //                with tcgen05.st, so expanded weights never touch shared memory.
 //   B (tokens)   int8 activations [M][K], TMA with 128-byte swizzle into the
 //                canonical K-major layout the MMA descriptor describes.
-//   D            int32 accumulators in tensor memory, 128 lanes x 128 columns.
-// Warp roles (192 threads): warp 0 issues TMA, warp 1 allocates tensor memory
-// and issues tcgen05.mma.kind::i8 (one thread), warps 2-5 expand and then run
-// the epilogue (tcgen05.ld, subtract row sum, rescale, store).  Two CTAs fit
-// per SM (tensor memory 2 x 256 columns, shared memory 2 x ~82 KB), so one
-// CTA's epilogue overlaps the other's main loop.
+//   D            int32 accumulators in tensor memory, two buffers of 128 lanes
+//                x 128 columns: the epilogue drains one tile while the MMAs of
+//                the next accumulate into the other.
+// Tensor memory: D 2 x 128 columns + A 8 stages x 32 columns = 512 columns.
+//
+// Warp roles (416 threads):
+//   warps 0-3    TMA producers.  Warp w owns the ring slots s = w (mod 4); its
+//                lane 0 copies the activation tile and lane 1 the packed weight
+//                tile of the slot, so the two copies run side by side.  TMA
+//                copies issued by one thread complete one after another, so
+//                the ring is spread over several threads; and the slots are
+//                spread over warps, not lanes of one warp, because lanes that
+//                wait on different barriers move in lockstep.
+//   warp 4       tensor memory allocation; lane 0 issues tcgen05.mma.kind::i8.
+//   warps 5-8    expansion of the packed weights into tensor memory.
+//   warps 9-12   epilogue: tcgen05.ld, subtract the row sum, rescale, store.
+//                Per-token d and row sums are staged in shared memory per warp.
 //
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA
-// records BL_ERR_TIMEOUT in the device status word, lets copies and MMAs in
-// flight drain (bounded again), frees its tensor memory and returns.  No TMA
-// multicast is used anywhere.
+// records BL_ERR_TIMEOUT in the device status word, every role leaves its
+// loop, copies and MMAs in flight drain (bounded again), tensor memory is
+// freed and the CTA returns.  No TMA multicast is used anywhere.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -42,18 +56,15 @@ namespace {
 constexpr int kBM = 128;     // weight rows per tile (MMA M)
 constexpr int kBN = 128;     // tokens per tile (MMA N)
 constexpr int kBK = 128;     // k per pipeline stage
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kStages = 8;
+constexpr int kProducerWarps = 4;
+constexpr int kThreads = 32 * (kProducerWarps + 1 + 4 + 4);
 constexpr int kMmaK = 32;    // k per tcgen05.mma.kind::i8
-constexpr uint32_t kTmemCols = 256;  // D: 128 columns; A: kStages x 32 columns
+constexpr uint32_t kTmemCols = 512;  // D: 2 x 128 columns; A: kStages x 32 columns
 constexpr uint32_t kQStage = kBN * kBK;        // 16 KB of int8 activations
 constexpr uint32_t kPStage = kBM * kBK / 4;    // 4 KB of packed weights
-constexpr uint32_t kSmemQ = 0;
-constexpr uint32_t kSmemP = kSmemQ + kStages * kQStage;
-constexpr uint32_t kSmemBar = kSmemP + kStages * kPStage;
-constexpr uint32_t kNumBars = 3 * kStages + 2;
-constexpr uint32_t kSmemMisc = kSmemBar + kNumBars * 8;
-constexpr uint32_t kSmemBytes = kSmemMisc + 16 + 1024;  // + alignment slack
+static_assert(2 * kBN + kStages * (kBK / 4) == int(kTmemCols), "tensor memory budget");
+static_assert(kStages % kProducerWarps == 0, "producer warp w owns the slots congruent to w");
 
 struct GemmParams {
     const float *w_scale;
@@ -106,6 +117,20 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// Non-blocking test of an mbarrier phase (true once the phase with this parity completed).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar)
@@ -168,164 +193,284 @@ constexpr uint32_t kIdesc = (2u << 4) | (0u << 7) | (1u << 10) | (uint32_t(kBN >
 
 // ---------------------------------------------------------------- kernel
 
+struct Smem {
+    // ring of operand stages (1024-byte aligned for the 128-byte swizzle)
+    unsigned char q[kStages][kQStage];
+    unsigned char p[kStages][kPStage];
+    // per epilogue warp: d and row sums of the current tile's 128 tokens
+    float ep_d[4][kBN];
+    int32_t ep_r[4][kBN];
+    uint64_t full[kStages];      // TMA landed
+    uint64_t afull[kStages];     // A expanded into tensor memory
+    uint64_t empty[kStages];     // MMAs of the stage completed
+    uint64_t tfull[2];           // accumulator buffer complete
+    uint64_t tempty[2];          // accumulator buffer drained
+    uint64_t drain;              // teardown after an abort
+    uint32_t tmem_base;
+    int abort_flag;
+};
+constexpr uint32_t kSmemBytes = uint32_t(sizeof(Smem)) + 1024;  // + alignment slack
+static_assert(kSmemBytes > 116 * 1024, "one CTA per SM: its 512 tensor-memory columns are the whole SM's");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+
+struct TileMap {
+    int tiles_m;                 // token tiles
+    int num_tiles;
+    __device__ void coords(int t, int64_t &n0, int64_t &m0) const
+    {
+        n0 = int64_t(t / tiles_m) * kBM;
+        m0 = int64_t(t % tiles_m) * kBN;
+    }
+};
+
+template <typename T>
+__device__ __forceinline__ void store_out(T *y, int64_t idx, float v);
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16 *y, int64_t idx, float v)
+{
+    y[idx] = __float2bfloat16_rn(v);
+}
+template <>
+__device__ __forceinline__ void store_out<float>(float *y, int64_t idx, float v)
+{
+    y[idx] = v;
+}
+
+// One 32-token chunk of the epilogue for this thread's weight row n.
+template <typename T, bool FULL>
+__device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], const float *sd, const int32_t *sr,
+                                               int64_t n, int64_t m0, const GemmParams &p, float gamma)
+{
+    T *y = static_cast<T *>(p.y);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const int64_t m = m0 + j;
+        if (FULL || m < p.M) {
+            const int a = int(v[j]) - sr[j];
+            if (p.acc_dbg)
+                p.acc_dbg[m * p.N + n] = a;
+            store_out<T>(y, m * p.ldy + n, rescale1(a, sd[j], gamma));
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap pmap,
-            const GemmParams p)
+            const GemmParams p, const TileMap tm)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
-    unsigned char *sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    const uint32_t sbase = smem_u32(sm);
-    const uint32_t bar_full = sbase + kSmemBar;                  // TMA landed     [kStages]
-    const uint32_t bar_afull = bar_full + 8 * kStages;          // A expanded     [kStages]
-    const uint32_t bar_empty = bar_afull + 8 * kStages;         // MMA consumed   [kStages]
-    const uint32_t bar_dfull = bar_empty + 8 * kStages;         // accumulators ready
-    const uint32_t bar_drain = bar_dfull + 8;                   // teardown after an abort
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kSmemMisc);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kSmemMisc + 4);
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
+    volatile int *abort_flag = &sm.abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t n0 = int64_t(blockIdx.x) * kBM;
-    const int64_t m0 = int64_t(blockIdx.y) * kBN;
     const int KB = int((p.K + kBK - 1) / kBK);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar_full + 8 * s, 1);
-            mbar_init(bar_afull + 8 * s, 128);
-            mbar_init(bar_empty + 8 * s, 1);
+            mbar_init(smem_u32(&sm.full[s]), 2);
+            mbar_init(smem_u32(&sm.afull[s]), 128);
+            mbar_init(smem_u32(&sm.empty[s]), 1);
         }
-        mbar_init(bar_dfull, 1);
-        mbar_init(bar_drain, 1);
-        *abort_flag = 0;
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&sm.tfull[b]), 1);
+            mbar_init(smem_u32(&sm.tempty[b]), 128);
+        }
+        mbar_init(smem_u32(&sm.drain), 1);
+        sm.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&qmap)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&pmap)) : "memory");
     }
-    if (warp == 1)
-        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    if (warp == kProducerWarps)
+        tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t d_tmem = tmem;                 // columns [0, 128)
-    const uint32_t a_tmem0 = tmem + kBN;          // columns [128, 256): kStages x 32
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t a_tmem0 = tmem + 2 * kBN;    // columns [256, 512): kStages x 32
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t ph = uint32_t(kb / kStages) & 1u;
-                if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort_flag, p.status))
-                    break;
-                mbar_arrive_tx(bar_full + 8 * s, kQStage + kPStage);
-                tma_load_2d(sbase + kSmemQ + s * kQStage, &qmap, bar_full + 8 * s, kb * kBK,
-                            int32_t(m0));
-                tma_load_2d(sbase + kSmemP + s * kPStage, &pmap, bar_full + 8 * s, kb * (kBK * 2),
-                            int32_t(n0 / 8));
-                issued = kb + 1;
-            }
-            if (*abort_flag) {
-                // let every copy this thread started land before the CTA exits
-                for (int kb = issued > kStages ? issued - kStages : 0; kb < issued; ++kb) {
-                    volatile int no_abort = 0;
-                    mbar_wait(bar_full + 8 * (kb % kStages), uint32_t(kb / kStages) & 1u,
-                              &no_abort, p.status, 100000000ull);
+    if (warp < kProducerWarps) {
+        // ------------------------------------------------ TMA producers
+        if (lane < 2) {
+            const bool is_q = lane == 0;
+            int last = -1;   // global stage index of this thread's last issued copy
+            int base = 0;    // global stage index of the current tile's first k block
+            bool ok = true;
+            for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, base += KB) {
+                int64_t n0, m0;
+                tm.coords(t, n0, m0);
+                for (int kb = ((warp - base) % kProducerWarps + kProducerWarps) % kProducerWarps; kb < KB;
+                     kb += kProducerWarps) {
+                    const int g = base + kb;
+                    const int s = g % kStages;
+                    const uint32_t full = smem_u32(&sm.full[s]);
+                    if (!mbar_wait(smem_u32(&sm.empty[s]), (uint32_t(g / kStages) & 1u) ^ 1u, abort_flag,
+                                   p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    if (is_q) {
+                        mbar_arrive_tx(full, kQStage);
+                        tma_load_2d(smem_u32(sm.q[s]), &qmap, full, kb * kBK, int32_t(m0));
+                    } else {
+                        mbar_arrive_tx(full, kPStage);
+                        tma_load_2d(smem_u32(sm.p[s]), &pmap, full, kb * (kBK * 2), int32_t(n0 / 8));
+                    }
+                    last = g;
                 }
             }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            int issued = 0;
-            for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t ph = uint32_t(kb / kStages) & 1u;
-                if (!mbar_wait(bar_full + 8 * s, ph, abort_flag, p.status))
-                    break;
-                if (!mbar_wait(bar_afull + 8 * s, ph, abort_flag, p.status))
-                    break;
-                tc_fence_after();
-                const uint32_t qaddr = sbase + kSmemQ + s * kQStage;
-#pragma unroll
-                for (int j = 0; j < kBK / kMmaK; ++j) {
-                    const uint64_t bdesc = smem_desc_sw128(qaddr + j * kMmaK);
-                    mma_i8_ts(d_tmem, a_tmem0 + s * (kBK / 4) + j * (kMmaK / 4), bdesc, kIdesc,
-                              (kb > 0 || j > 0) ? 1u : 0u);
-                }
-                mma_commit(bar_empty + 8 * s);
-                issued = kb + 1;
-            }
-            if (issued == KB) {
-                mma_commit(bar_dfull);
-            } else if (issued > 0) {
-                // drain the MMAs in flight before tensor memory is released
-                mma_commit(bar_drain);
+            if (last >= 0) {
+                // this thread's last copy has landed before the CTA exits (at
+                // once unless another role gave up before consuming it)
                 volatile int no_abort = 0;
-                mbar_wait(bar_drain, 0, &no_abort, p.status, 100000000ull);
+                mbar_wait(smem_u32(&sm.full[last % kStages]), uint32_t(last / kStages) & 1u, &no_abort, p.status,
+                          100000000ull);
             }
         }
-    } else {
-        // ------------------------------------------------ expansion, then epilogue
+    } else if (warp == kProducerWarps) {
+        // ------------------------------------------------ MMA issuer
+        // The tensor pipe queues about one MMA ahead of the issuing thread, so a
+        // barrier wait between stages leaves it idle for the wait's shared
+        // memory round trip.  The thread therefore tests the next stage's
+        // barriers (non-blocking) right after the first MMA of the current
+        // stage, while the remaining MMAs of the stage queue, and blocks only
+        // when that test found the next stage not yet ready.
+        if (lane == 0) {
+            int g = 0, it = 0;
+            bool ok = true, issued_any = false, ready = false;
+            for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, ++it) {
+                const int b = it & 1;
+                if (it >= 2 &&
+                    !mbar_wait(smem_u32(&sm.tempty[b]), (uint32_t(it >> 1) & 1u) ^ 1u, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t d_tmem = tmem + uint32_t(b * kBN);
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int s = g % kStages;
+                    const uint32_t ph = uint32_t(g / kStages) & 1u;
+                    if (!ready && (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, p.status) ||
+                                   !mbar_wait(smem_u32(&sm.afull[s]), ph, abort_flag, p.status))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t qaddr = smem_u32(sm.q[s]);
+                    const uint32_t a_stage = a_tmem0 + s * (kBK / 4);
+                    mma_i8_ts(d_tmem, a_stage, smem_desc_sw128(qaddr), kIdesc, kb > 0 ? 1u : 0u);
+                    const int s1 = (g + 1) % kStages;
+                    const uint32_t ph1 = uint32_t((g + 1) / kStages) & 1u;
+                    const bool next_full = mbar_test(smem_u32(&sm.full[s1]), ph1);
+                    const bool next_afull = mbar_test(smem_u32(&sm.afull[s1]), ph1);
+#pragma unroll
+                    for (int j = 1; j < kBK / kMmaK; ++j)
+                        mma_i8_ts(d_tmem, a_stage + j * (kMmaK / 4), smem_desc_sw128(qaddr + j * kMmaK), kIdesc, 1u);
+                    mma_commit(smem_u32(&sm.empty[s]));
+                    issued_any = true;
+                    ready = next_full && next_afull;
+                }
+                if (ok)
+                    mma_commit(smem_u32(&sm.tfull[b]));
+            }
+            if (issued_any) {
+                // every MMA has completed before tensor memory is released (at
+                // once unless the epilogue gave up before draining them)
+                mma_commit(smem_u32(&sm.drain));
+                volatile int no_abort = 0;
+                mbar_wait(smem_u32(&sm.drain), 0, &no_abort, p.status, 100000000ull);
+            }
+        }
+    } else if (warp < kProducerWarps + 5) {
+        // ------------------------------------------------ expansion into tensor memory
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
         const int rl = quarter * 32 + lane;           // weight row within the tile
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+        int g = 0;
         bool ok = true;
-        for (int kb = 0; kb < KB; ++kb) {
-            const int s = kb % kStages;
-            const uint32_t ph = uint32_t(kb / kStages) & 1u;
-            // warp-uniform outcome: the tcgen05.st below is .sync.aligned
-            if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, ph, abort_flag, p.status))) {
-                ok = false;
-                break;
-            }
-            const unsigned char *ps = sm + kSmemP + s * kPStage + (rl >> 3) * 256 + (rl & 7) * 16;
-            const uint4 c0 = *reinterpret_cast<const uint4 *>(ps);
-            const uint4 c1 = *reinterpret_cast<const uint4 *>(ps + 128);
-            const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-            uint32_t v[32];
+        for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x) {
+            for (int kb = 0; kb < KB; ++kb, ++g) {
+                const int s = g % kStages;
+                const uint32_t ph = uint32_t(g / kStages) & 1u;
+                // warp-uniform outcome: the tcgen05.st below is .sync.aligned
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, p.status))) {
+                    ok = false;
+                    break;
+                }
+                const unsigned char *ps = sm.p[s] + (rl >> 3) * 256 + (rl & 7) * 16;
+                const uint4 c0 = *reinterpret_cast<const uint4 *>(ps);
+                const uint4 c1 = *reinterpret_cast<const uint4 *>(ps + 128);
+                const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                uint32_t v[32];
 #pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                v[4 * w + 0] = wd[w] & 0x03030303u;
-                v[4 * w + 1] = (wd[w] >> 2) & 0x03030303u;
-                v[4 * w + 2] = (wd[w] >> 4) & 0x03030303u;
-                v[4 * w + 3] = (wd[w] >> 6) & 0x03030303u;
+                for (int w = 0; w < 8; ++w) {
+                    v[4 * w + 0] = wd[w] & 0x03030303u;
+                    v[4 * w + 1] = (wd[w] >> 2) & 0x03030303u;
+                    v[4 * w + 2] = (wd[w] >> 4) & 0x03030303u;
+                    v[4 * w + 3] = (wd[w] >> 6) & 0x03030303u;
+                }
+                tmem_st32(a_tmem0 + lane_addr + s * (kBK / 4), v);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_u32(&sm.afull[s]));
             }
-            tmem_st32(a_tmem0 + lane_addr + s * (kBK / 4), v);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar_afull + 8 * s);
         }
-        if (ok && __all_sync(0xffffffffu, mbar_wait(bar_dfull, 0, abort_flag, p.status))) {
+    } else {
+        // ------------------------------------------------ epilogue
+        const int quarter = warp & 3;
+        const int ew = warp - (kProducerWarps + 5);   // this warp's staging slice
+        const int rl = quarter * 32 + lane;
+        const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
+        const float gamma = p.w_scale[0];
+        float *sd = sm.ep_d[ew];
+        int32_t *sr = sm.ep_r[ew];
+        int it = 0;
+        for (int t = blockIdx.x; t < tm.num_tiles; t += gridDim.x, ++it) {
+            const int b = it & 1;
+            int64_t n0, m0;
+            tm.coords(t, n0, m0);
+            __syncwarp();
+#pragma unroll
+            for (int c = 0; c < kBN / 32; ++c) {
+                const int64_t m = m0 + c * 32 + lane;
+                sd[c * 32 + lane] = m < p.M ? __ldg(p.d + m) : 0.0f;
+                sr[c * 32 + lane] = m < p.M ? __ldg(p.rowsum + m) : 0;
+            }
+            __syncwarp();
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(smem_u32(&sm.tfull[b]), uint32_t(it >> 1) & 1u, abort_flag, p.status)))
+                break;
             tc_fence_after();
             const int64_t n = n0 + rl;
-            const float gamma = p.w_scale[0];
+            const bool full_m = m0 + kBN <= p.M;
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
                 uint32_t v[32];
-                tmem_ld32(d_tmem + lane_addr + c * 32, v);
+                tmem_ld32(tmem + lane_addr + uint32_t(b * kBN + c * 32), v);
                 tmem_wait_ld();
                 if (n < p.N) {
-#pragma unroll 4
-                    for (int j = 0; j < 32; ++j) {
-                        const int64_t m = m0 + c * 32 + j;
-                        if (m < p.M) {
-                            const int a = int(v[j]) - __ldg(p.rowsum + m);
-                            if (p.acc_dbg)
-                                p.acc_dbg[m * p.N + n] = a;
-                            store_y(p.y, p.yt, m * p.ldy + n, rescale1(a, __ldg(p.d + m), gamma));
-                        }
+                    const int64_t mc = m0 + c * 32;
+                    if (p.yt == BL_BF16) {
+                        if (full_m)
+                            epilogue_chunk<__nv_bfloat16, true>(v, sd + c * 32, sr + c * 32, n, mc, p, gamma);
+                        else
+                            epilogue_chunk<__nv_bfloat16, false>(v, sd + c * 32, sr + c * 32, n, mc, p, gamma);
+                    } else {
+                        if (full_m)
+                            epilogue_chunk<float, true>(v, sd + c * 32, sr + c * 32, n, mc, p, gamma);
+                        else
+                            epilogue_chunk<float, false>(v, sd + c * 32, sr + c * 32, n, mc, p, gamma);
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&sm.tempty[b]));
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kProducerWarps) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -396,8 +541,14 @@ int launch_gemm(const GemvArgs &a, void *, size_t, cudaStream_t s)
     if (per_sm < 1)
         return BL_ERR_UNSUPPORTED;
     GemmParams p{a.w_scale, a.d, a.rowsum, a.M, a.N, a.K, a.y, a.yt, a.ldy, a.acc_dbg, di->status};
-    dim3 grid(unsigned((a.N + kBM - 1) / kBM), unsigned((a.M + kBN - 1) / kBN));
-    gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(qmap, pmap, p);
+    TileMap tm;
+    tm.tiles_m = int((a.M + kBN - 1) / kBN);
+    const int64_t tiles = int64_t(tm.tiles_m) * ((a.N + kBM - 1) / kBM);
+    if (tiles > (int64_t(1) << 30))
+        return BL_ERR_SHAPE;
+    tm.num_tiles = int(tiles);
+    const int grid = int(std::min<int64_t>(tiles, di->sm_count));
+    gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(qmap, pmap, p, tm);
     return launch_status();
 }
 

@@ -261,6 +261,14 @@ def test_gemm_ragged_shapes(bl, M, N, K):
     _check_gemm(bl, N, K, M, seed=M + N + K)
 
 
+@pytest.mark.parametrize("M,N,K", [(1200, 4000, 320), (1024, 2560, 1024), (2048, 2048, 128),
+                                   (1100, 2900, 192)])
+def test_gemm_several_tiles_per_cta(bl, M, N, K):
+    """More output tiles than SMs: each persistent CTA walks several tiles,
+    alternating its two accumulator buffers; every output is checked."""
+    _check_gemm(bl, N, K, M, seed=M ^ N ^ K)
+
+
 @pytest.mark.parametrize("K,N", si.PREFILL_SHAPES)
 @pytest.mark.parametrize("M", si.PREFILL_TOKENS)
 def test_gemm_prefill_full_size(bl, K, N, M):
