@@ -11,30 +11,38 @@
 // row sum and rescales.
 //
 // Persistent kernel, one CTA per SM, walking output tiles of 128 weight rows
-// (MMA M) x 128 tokens (MMA N); k advances 128 per pipeline stage through an
-// eight-slot ring.  Operands:
+// (MMA M) x 128 tokens (MMA N); k advances 256 per pipeline stage through a
+// four-slot ring.  A stage is eight MMAs (128x128x32, 64 tensor cycles each):
+// an issuing thread that waits on a barrier once per stage cannot issue
+// faster than about one stage per 480 cycles, so a stage carries at least
+// that much tensor work.  Operands:
 //   A (weights)  TL bytes of the tile arrive in shared memory by TMA (a 2-D
-//                view [row groups][K/64 * 128 B], box 16 groups x 256 B); four
+//                view [row groups][K/64 * 128 B], two boxes of 16 groups x
+//                256 B per stage); four
 //                expansion warps turn each thread's row (one TMEM lane) into
 //                int8 {0,1,2} -- (word >> 2i) & 0x03030303 gives four
 //                consecutive k -- and write them straight into tensor memory
 //                with tcgen05.st, so expanded weights never touch shared memory.
-//   B (tokens)   int8 activations [M][K], TMA with 128-byte swizzle into the
-//                canonical K-major layout the MMA descriptor describes.
+//   B (tokens)   int8 activations [M][K], two TMA boxes of 128 tokens x 128 k
+//                per stage with 128-byte swizzle, the canonical K-major layout
+//                the MMA descriptor describes.
 //   D            int32 accumulators in tensor memory, two buffers of 128 lanes
 //                x 128 columns: the epilogue drains one tile while the MMAs of
 //                the next accumulate into the other.
-// Tensor memory: D 2 x 128 columns + A 8 stages x 32 columns = 512 columns.
+// Tensor memory: D 2 x 128 columns + A 4 stages x 64 columns = 512 columns.
 //
 // Warp roles (416 threads):
-//   warps 0-3    TMA producers.  Warp w owns the ring slots s = w (mod 4); its
-//                lane 0 copies the activation tile and lane 1 the packed weight
-//                tile of the slot, so the two copies run side by side.  TMA
-//                copies issued by one thread complete one after another, so
-//                the ring is spread over several threads; and the slots are
-//                spread over warps, not lanes of one warp, because lanes that
-//                wait on different barriers move in lockstep.
+//   warps 0-3    TMA producers.  Warp w owns ring slot w; lanes 0-1 copy the
+//                two activation boxes and lanes 2-3 the two packed weight boxes
+//                of the slot, so the four copies run side by side.  TMA copies
+//                issued by one thread complete one after another, so the ring
+//                is spread over several threads; and the slots are spread over
+//                warps, not lanes of one warp, because lanes that wait on
+//                different barriers move in lockstep.
 //   warp 4       tensor memory allocation; lane 0 issues tcgen05.mma.kind::i8.
+//                It waits only on the expansion barrier of a stage: the
+//                expansion warps arrive there after they have seen the stage's
+//                copies land, which orders the activation tile before the MMAs.
 //   warps 5-8    expansion of the packed weights into tensor memory.
 //   warps 9-12   epilogue: tcgen05.ld, subtract the row sum, rescale, store.
 //                Per-token d and row sums are staged in shared memory per warp.
@@ -55,16 +63,19 @@ namespace {
 
 constexpr int kBM = 128;     // weight rows per tile (MMA M)
 constexpr int kBN = 128;     // tokens per tile (MMA N)
-constexpr int kBK = 128;     // k per pipeline stage
-constexpr int kStages = 8;
-constexpr int kProducerWarps = 4;
+constexpr int kBK = 256;     // k per pipeline stage: eight MMAs between barrier waits
+constexpr int kBoxK = 128;   // k per TMA box (one 128-byte swizzle span of activations)
+constexpr int kBoxes = kBK / kBoxK;
+constexpr int kStages = 4;
+constexpr int kProducerWarps = kStages;   // producer warp w owns ring slot w
 constexpr int kThreads = 32 * (kProducerWarps + 1 + 4 + 4);
 constexpr int kMmaK = 32;    // k per tcgen05.mma.kind::i8
-constexpr uint32_t kTmemCols = 512;  // D: 2 x 128 columns; A: kStages x 32 columns
-constexpr uint32_t kQStage = kBN * kBK;        // 16 KB of int8 activations
-constexpr uint32_t kPStage = kBM * kBK / 4;    // 4 KB of packed weights
-static_assert(2 * kBN + kStages * (kBK / 4) == int(kTmemCols), "tensor memory budget");
-static_assert(kStages % kProducerWarps == 0, "producer warp w owns the slots congruent to w");
+constexpr uint32_t kTmemCols = 512;  // D: 2 x 128 columns; A: kStages x 64 columns
+constexpr uint32_t kQBox = kBN * kBoxK;        // 16 KB of int8 activations per box
+constexpr uint32_t kPBox = kBM * kBoxK / 4;    // 4 KB of packed weights per box
+constexpr uint32_t kACols = kBK / 4;           // TMEM columns of one expanded A stage
+static_assert(2 * kBN + kStages * int(kACols) == int(kTmemCols), "tensor memory budget");
+static_assert(2 * kBoxes <= 32, "one producer lane per TMA box of a stage");
 
 struct GemmParams {
     const float *w_scale;
@@ -117,20 +128,6 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
-}
-
-// Non-blocking test of an mbarrier phase (true once the phase with this parity completed).
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar)
@@ -195,8 +192,8 @@ constexpr uint32_t kIdesc = (2u << 4) | (0u << 7) | (1u << 10) | (uint32_t(kBN >
 
 struct Smem {
     // ring of operand stages (1024-byte aligned for the 128-byte swizzle)
-    unsigned char q[kStages][kQStage];
-    unsigned char p[kStages][kPStage];
+    unsigned char q[kStages][kBoxes][kQBox];
+    unsigned char p[kStages][kBoxes][kPBox];
     // per epilogue warp: d and row sums of the current tile's 128 tokens
     float ep_d[4][kBN];
     int32_t ep_r[4][kBN];
@@ -268,7 +265,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(smem_u32(&sm.full[s]), 2);
+            mbar_init(smem_u32(&sm.full[s]), 2 * kBoxes);
             mbar_init(smem_u32(&sm.afull[s]), 128);
             mbar_init(smem_u32(&sm.empty[s]), 1);
         }
@@ -288,34 +285,35 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t a_tmem0 = tmem + 2 * kBN;    // columns [256, 512): kStages x 32
+    const uint32_t a_tmem0 = tmem + 2 * kBN;    // columns [256, 512): kStages x 64
 
     if (warp < kProducerWarps) {
         // ------------------------------------------------ TMA producers
-        if (lane < 2) {
-            const bool is_q = lane == 0;
+        if (lane < 2 * kBoxes) {
+            const bool is_q = lane < kBoxes;
+            const int box = lane % kBoxes;
+            const int s = warp;
+            const uint32_t full = smem_u32(&sm.full[s]);
             int last = -1;   // global stage index of this thread's last issued copy
             int base = 0;    // global stage index of the current tile's first k block
             bool ok = true;
             for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, base += KB) {
                 int64_t n0, m0;
                 tm.coords(t, n0, m0);
-                for (int kb = ((warp - base) % kProducerWarps + kProducerWarps) % kProducerWarps; kb < KB;
-                     kb += kProducerWarps) {
+                for (int kb = ((s - base) % kStages + kStages) % kStages; kb < KB; kb += kStages) {
                     const int g = base + kb;
-                    const int s = g % kStages;
-                    const uint32_t full = smem_u32(&sm.full[s]);
                     if (!mbar_wait(smem_u32(&sm.empty[s]), (uint32_t(g / kStages) & 1u) ^ 1u, abort_flag,
                                    p.status)) {
                         ok = false;
                         break;
                     }
+                    const int k0 = kb * kBK + box * kBoxK;
                     if (is_q) {
-                        mbar_arrive_tx(full, kQStage);
-                        tma_load_2d(smem_u32(sm.q[s]), &qmap, full, kb * kBK, int32_t(m0));
+                        mbar_arrive_tx(full, kQBox);
+                        tma_load_2d(smem_u32(sm.q[s][box]), &qmap, full, k0, int32_t(m0));
                     } else {
-                        mbar_arrive_tx(full, kPStage);
-                        tma_load_2d(smem_u32(sm.p[s]), &pmap, full, kb * (kBK * 2), int32_t(n0 / 8));
+                        mbar_arrive_tx(full, kPBox);
+                        tma_load_2d(smem_u32(sm.p[s][box]), &pmap, full, k0 * 2, int32_t(n0 / 8));
                     }
                     last = g;
                 }
@@ -324,21 +322,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                 // this thread's last copy has landed before the CTA exits (at
                 // once unless another role gave up before consuming it)
                 volatile int no_abort = 0;
-                mbar_wait(smem_u32(&sm.full[last % kStages]), uint32_t(last / kStages) & 1u, &no_abort, p.status,
-                          100000000ull);
+                mbar_wait(full, uint32_t(last / kStages) & 1u, &no_abort, p.status, 100000000ull);
             }
         }
     } else if (warp == kProducerWarps) {
         // ------------------------------------------------ MMA issuer
-        // The tensor pipe queues about one MMA ahead of the issuing thread, so a
-        // barrier wait between stages leaves it idle for the wait's shared
-        // memory round trip.  The thread therefore tests the next stage's
-        // barriers (non-blocking) right after the first MMA of the current
-        // stage, while the remaining MMAs of the stage queue, and blocks only
-        // when that test found the next stage not yet ready.
         if (lane == 0) {
             int g = 0, it = 0;
-            bool ok = true, issued_any = false, ready = false;
+            bool ok = true, issued_any = false;
             for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, ++it) {
                 const int b = it & 1;
                 if (it >= 2 &&
@@ -349,26 +340,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                 const uint32_t d_tmem = tmem + uint32_t(b * kBN);
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStages;
-                    const uint32_t ph = uint32_t(g / kStages) & 1u;
-                    if (!ready && (!mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, p.status) ||
-                                   !mbar_wait(smem_u32(&sm.afull[s]), ph, abort_flag, p.status))) {
+                    if (!mbar_wait(smem_u32(&sm.afull[s]), uint32_t(g / kStages) & 1u, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t qaddr = smem_u32(sm.q[s]);
-                    const uint32_t a_stage = a_tmem0 + s * (kBK / 4);
-                    mma_i8_ts(d_tmem, a_stage, smem_desc_sw128(qaddr), kIdesc, kb > 0 ? 1u : 0u);
-                    const int s1 = (g + 1) % kStages;
-                    const uint32_t ph1 = uint32_t((g + 1) / kStages) & 1u;
-                    const bool next_full = mbar_test(smem_u32(&sm.full[s1]), ph1);
-                    const bool next_afull = mbar_test(smem_u32(&sm.afull[s1]), ph1);
+                    const uint32_t a_stage = a_tmem0 + s * kACols;
 #pragma unroll
-                    for (int j = 1; j < kBK / kMmaK; ++j)
-                        mma_i8_ts(d_tmem, a_stage + j * (kMmaK / 4), smem_desc_sw128(qaddr + j * kMmaK), kIdesc, 1u);
+                    for (int j = 0; j < kBK / kMmaK; ++j) {
+                        const uint32_t qaddr = smem_u32(sm.q[s][j / (kBoxK / kMmaK)]) + (j % (kBoxK / kMmaK)) * kMmaK;
+                        mma_i8_ts(d_tmem, a_stage + j * (kMmaK / 4), smem_desc_sw128(qaddr), kIdesc,
+                                  (kb > 0 || j > 0) ? 1u : 0u);
+                    }
                     mma_commit(smem_u32(&sm.empty[s]));
                     issued_any = true;
-                    ready = next_full && next_afull;
                 }
                 if (ok)
                     mma_commit(smem_u32(&sm.tfull[b]));
@@ -397,19 +382,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                     ok = false;
                     break;
                 }
-                const unsigned char *ps = sm.p[s] + (rl >> 3) * 256 + (rl & 7) * 16;
-                const uint4 c0 = *reinterpret_cast<const uint4 *>(ps);
-                const uint4 c1 = *reinterpret_cast<const uint4 *>(ps + 128);
-                const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint32_t v[32];
 #pragma unroll
-                for (int w = 0; w < 8; ++w) {
-                    v[4 * w + 0] = wd[w] & 0x03030303u;
-                    v[4 * w + 1] = (wd[w] >> 2) & 0x03030303u;
-                    v[4 * w + 2] = (wd[w] >> 4) & 0x03030303u;
-                    v[4 * w + 3] = (wd[w] >> 6) & 0x03030303u;
+                for (int box = 0; box < kBoxes; ++box) {
+                    const unsigned char *ps = sm.p[s][box] + (rl >> 3) * 256 + (rl & 7) * 16;
+                    const uint4 c0 = *reinterpret_cast<const uint4 *>(ps);
+                    const uint4 c1 = *reinterpret_cast<const uint4 *>(ps + 128);
+                    const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    uint32_t v[32];
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        v[4 * w + 0] = wd[w] & 0x03030303u;
+                        v[4 * w + 1] = (wd[w] >> 2) & 0x03030303u;
+                        v[4 * w + 2] = (wd[w] >> 4) & 0x03030303u;
+                        v[4 * w + 3] = (wd[w] >> 6) & 0x03030303u;
+                    }
+                    tmem_st32(a_tmem0 + lane_addr + s * kACols + box * 32, v);
                 }
-                tmem_st32(a_tmem0 + lane_addr + s * (kBK / 4), v);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_u32(&sm.afull[s]));
@@ -525,13 +513,13 @@ int launch_gemm(const GemvArgs &a, void *, size_t, cudaStream_t s)
     if (a.M > (int64_t(1) << 30) || a.N > (int64_t(1) << 30))
         return BL_ERR_SHAPE;
     CUtensorMap qmap, pmap;
-    // activations: [M][K] int8, 128 x 128 boxes, 128-byte swizzle
-    int st = make_map_2d(&qmap, a.q, uint64_t(a.K), uint64_t(a.M), uint64_t(a.K), kBK, kBN, true);
+    // activations: [M][K] int8, boxes of 128 k x 128 tokens, 128-byte swizzle
+    int st = make_map_2d(&qmap, a.q, uint64_t(a.K), uint64_t(a.M), uint64_t(a.K), kBoxK, kBN, true);
     if (st)
         return st;
-    // packed weights as [row groups][K/64 * 128 B]: 16 groups x 256 B per stage
+    // packed weights as [row groups][K/64 * 128 B]: boxes of 16 groups x 256 B (128 k)
     const uint64_t rg_bytes = uint64_t(a.K / 64) * 128;
-    st = make_map_2d(&pmap, a.packed, rg_bytes, uint64_t((a.N + 7) / 8), rg_bytes, 2 * kBK,
+    st = make_map_2d(&pmap, a.packed, rg_bytes, uint64_t((a.N + 7) / 8), rg_bytes, 2 * kBoxK,
                      kBM / 8, false);
     if (st)
         return st;
