@@ -11,40 +11,42 @@
 // row sum and rescales.
 //
 // Persistent kernel, one CTA per SM, walking output tiles of 128 weight rows
-// (MMA M) x 128 tokens (MMA N); k advances 256 per pipeline stage through a
-// four-slot ring.  A stage is eight MMAs (128x128x32, 64 tensor cycles each):
-// an issuing thread that waits on a barrier once per stage cannot issue
-// faster than about one stage per 480 cycles, so a stage carries at least
-// that much tensor work.  Operands:
-//   A (weights)  TL bytes of the tile arrive in shared memory by TMA (a 2-D
-//                view [row groups][K/64 * 128 B], two boxes of 16 groups x
-//                256 B per stage); four
-//                expansion warps turn each thread's row (one TMEM lane) into
-//                int8 {0,1,2} -- (word >> 2i) & 0x03030303 gives four
-//                consecutive k -- and write them straight into tensor memory
-//                with tcgen05.st, so expanded weights never touch shared memory.
-//   B (tokens)   int8 activations [M][K], two TMA boxes of 128 tokens x 128 k
-//                per stage with 128-byte swizzle, the canonical K-major layout
-//                the MMA descriptor describes.
+// (MMA M) x 128 tokens (MMA N); k advances 256 per pipeline stage.  A stage is
+// eight MMAs (128x128x32, 64 tensor cycles each): an issuing thread that waits
+// on a barrier once per stage cannot issue faster than about one stage per
+// 480 cycles, so a stage carries at least that much tensor work.  Operands:
+//   B (tokens)   int8 activations [M][K]: two TMA boxes of 128 tokens x 128 k
+//                per stage with 128-byte swizzle (the canonical K-major layout
+//                of the MMA descriptor), in a five-slot shared-memory ring.
+//   A (weights)  TL bytes of the tile arrive in the same ring slot by TMA (a
+//                2-D view [row groups][K/64 * 128 B], two boxes of 16 groups x
+//                256 B); each expansion thread owns one weight row (one TMEM
+//                lane) and turns its bytes into int8 {0,1,2} -- (word >> 2i) &
+//                0x03030303 gives four consecutive k -- written straight into a
+//                four-stage ring in tensor memory with tcgen05.st.
 //   D            int32 accumulators in tensor memory, two buffers of 128 lanes
 //                x 128 columns: the epilogue drains one tile while the MMAs of
 //                the next accumulate into the other.
 // Tensor memory: D 2 x 128 columns + A 4 stages x 64 columns = 512 columns.
 //
-// Warp roles (416 threads):
-//   warps 0-3    TMA producers.  Warp w owns ring slot w; lanes 0-1 copy the
-//                two activation boxes and lanes 2-3 the two packed weight boxes
-//                of the slot, so the four copies run side by side.  TMA copies
-//                issued by one thread complete one after another, so the ring
-//                is spread over several threads; and the slots are spread over
-//                warps, not lanes of one warp, because lanes that wait on
-//                different barriers move in lockstep.
-//   warp 4       tensor memory allocation; lane 0 issues tcgen05.mma.kind::i8.
-//                It waits only on the expansion barrier of a stage: the
-//                expansion warps arrive there after they have seen the stage's
-//                copies land, which orders the activation tile before the MMAs.
-//   warps 5-8    expansion of the packed weights into tensor memory.
-//   warps 9-12   epilogue: tcgen05.ld, subtract the row sum, rescale, store.
+// Warp roles (480 threads):
+//   warps 0-1    TMA producers.  Warp w copies the stages g = w (mod 2): lanes
+//                0-1 the two activation boxes, lanes 2-3 the two packed weight
+//                boxes, side by side.  TMA copies issued
+//                by one thread complete one after another, so the ring is
+//                spread over several threads, and over warps rather than lanes
+//                of one warp, because lanes that wait on different barriers
+//                move in lockstep.
+//   warp 2       tensor memory allocation; lane 0 issues tcgen05.mma.kind::i8.
+//                It waits on one barrier per stage, the expansion barrier: the
+//                expansion warps arrive there once the A stage is written and
+//                they have seen the stage's activation copies land.
+//   warps 3-10   expansion of the packed weights into tensor memory, two groups
+//                of four warps (one per TMEM lane quarter) taking alternate
+//                stages: an mbarrier check costs a couple of hundred cycles
+//                even when the phase has completed, and one stage's expansion
+//                with its checks takes longer than the stage's MMAs.
+//   warps 11-14  epilogue: tcgen05.ld, subtract the row sum, rescale, store.
 //                Per-token d and row sums are staged in shared memory per warp.
 //
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA
@@ -66,16 +68,20 @@ constexpr int kBN = 128;     // tokens per tile (MMA N)
 constexpr int kBK = 256;     // k per pipeline stage: eight MMAs between barrier waits
 constexpr int kBoxK = 128;   // k per TMA box (one 128-byte swizzle span of activations)
 constexpr int kBoxes = kBK / kBoxK;
-constexpr int kStages = 4;
-constexpr int kProducerWarps = kStages;   // producer warp w owns ring slot w
-constexpr int kThreads = 32 * (kProducerWarps + 1 + 4 + 4);
+constexpr int kQStages = 5;  // operand ring (shared memory): activations and packed weights
+constexpr int kAStages = 4;  // expanded weight ring (tensor memory)
+constexpr int kExpGroups = 2;  // expansion groups, taking alternate stages
+constexpr int kProducerWarps = 2;
+constexpr int kMmaWarp = kProducerWarps;
+constexpr int kExpWarp0 = kMmaWarp + 1;
+constexpr int kEpiWarp0 = kExpWarp0 + 4 * kExpGroups;
+constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 constexpr int kMmaK = 32;    // k per tcgen05.mma.kind::i8
-constexpr uint32_t kTmemCols = 512;  // D: 2 x 128 columns; A: kStages x 64 columns
+constexpr uint32_t kTmemCols = 512;  // D: 2 x 128 columns; A: kAStages x 64 columns
 constexpr uint32_t kQBox = kBN * kBoxK;        // 16 KB of int8 activations per box
 constexpr uint32_t kPBox = kBM * kBoxK / 4;    // 4 KB of packed weights per box
 constexpr uint32_t kACols = kBK / 4;           // TMEM columns of one expanded A stage
-static_assert(2 * kBN + kStages * int(kACols) == int(kTmemCols), "tensor memory budget");
-static_assert(2 * kBoxes <= 32, "one producer lane per TMA box of a stage");
+static_assert(2 * kBN + kAStages * int(kACols) == int(kTmemCols), "tensor memory budget");
 
 struct GemmParams {
     const float *w_scale;
@@ -90,16 +96,6 @@ struct GemmParams {
 };
 
 // ---------------------------------------------------------------- PTX wrappers
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int32_t c0, int32_t c1)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
-        : "memory");
-}
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -118,22 +114,49 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
                  : "memory");
 }
 
+// The MMA role runs on a whole warp in warp-uniform control flow and issues
+// each tcgen05 operation from one lane chosen by elect.sync (the lowest active
+// lane, so always the same thread: tcgen05.commit tracks the operations of the
+// thread that executes it).  Issued from a single-lane divergent region
+// instead, back-to-back 128x128x32 MMAs measured ~120 cycles apiece once the
+// loop also waited on an mbarrier, against 64 in warp-uniform code.
+
 // D[tmem] (+)= A[tmem] * B[smem]^T, int8 inputs, int32 accumulate.
 __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate)
 {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+        : "memory");
+}
+
+// TMA load issued by lane `who` of a warp that runs in warp-uniform control
+// flow, together with that lane's expect-tx arrival on the stage barrier.
+__device__ __forceinline__ void tma_load_2d_lane(uint32_t who, uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                                 uint32_t bytes, int32_t c0, int32_t c1)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 l;\n\t"
+        "mov.u32 l, %%laneid;\n\t"
+        "setp.eq.u32 e, l, %0;\n\t"
+        "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%3], %4;\n\t"
+        "@e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%1], [%2, {%5, %6}], [%3];\n\t}" ::"r"(who),
+        "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(bytes), "r"(c0), "r"(c1)
+        : "memory");
 }
 
 // Thirty-two consecutive 32-bit TMEM columns of this thread's lane.
@@ -191,15 +214,16 @@ constexpr uint32_t kIdesc = (2u << 4) | (0u << 7) | (1u << 10) | (uint32_t(kBN >
 // ---------------------------------------------------------------- kernel
 
 struct Smem {
-    // ring of operand stages (1024-byte aligned for the 128-byte swizzle)
-    unsigned char q[kStages][kBoxes][kQBox];
-    unsigned char p[kStages][kBoxes][kPBox];
+    // activation ring (1024-byte aligned for the 128-byte swizzle)
+    unsigned char q[kQStages][kBoxes][kQBox];
+    unsigned char p[kQStages][kBoxes][kPBox];
     // per epilogue warp: d and row sums of the current tile's 128 tokens
     float ep_d[4][kBN];
     int32_t ep_r[4][kBN];
-    uint64_t full[kStages];      // TMA landed
-    uint64_t afull[kStages];     // A expanded into tensor memory
-    uint64_t empty[kStages];     // MMAs of the stage completed
+    uint64_t full[kQStages];     // activation and packed boxes landed
+    uint64_t empty[kQStages];    // the slot's bytes are no longer needed (MMAs completed)
+    uint64_t afull[kAStages];    // A expanded into tensor memory (and its activations landed)
+    uint64_t aempty[kAStages];   // MMAs reading the A stage completed
     uint64_t tfull[2];           // accumulator buffer complete
     uint64_t tempty[2];          // accumulator buffer drained
     uint64_t drain;              // teardown after an abort
@@ -264,10 +288,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
     const int KB = int((p.K + kBK - 1) / kBK);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kQStages; ++s) {
             mbar_init(smem_u32(&sm.full[s]), 2 * kBoxes);
-            mbar_init(smem_u32(&sm.afull[s]), 128);
             mbar_init(smem_u32(&sm.empty[s]), 1);
+        }
+        for (int a = 0; a < kAStages; ++a) {
+            mbar_init(smem_u32(&sm.afull[a]), 128);
+            mbar_init(smem_u32(&sm.aempty[a]), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&sm.tfull[b]), 1);
@@ -279,95 +306,96 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&qmap)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&pmap)) : "memory");
     }
-    if (warp == kProducerWarps)
+    if (warp == kMmaWarp)
         tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t a_tmem0 = tmem + 2 * kBN;    // columns [256, 512): kStages x 64
+    const uint32_t a_tmem0 = tmem + 2 * kBN;    // columns [256, 512): kAStages x 64
 
     if (warp < kProducerWarps) {
         // ------------------------------------------------ TMA producers
-        if (lane < 2 * kBoxes) {
-            const bool is_q = lane < kBoxes;
-            const int box = lane % kBoxes;
-            const int s = warp;
-            const uint32_t full = smem_u32(&sm.full[s]);
-            int last = -1;   // global stage index of this thread's last issued copy
-            int base = 0;    // global stage index of the current tile's first k block
-            bool ok = true;
-            for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, base += KB) {
-                int64_t n0, m0;
-                tm.coords(t, n0, m0);
-                for (int kb = ((s - base) % kStages + kStages) % kStages; kb < KB; kb += kStages) {
-                    const int g = base + kb;
-                    if (!mbar_wait(smem_u32(&sm.empty[s]), (uint32_t(g / kStages) & 1u) ^ 1u, abort_flag,
-                                   p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    const int k0 = kb * kBK + box * kBoxK;
-                    if (is_q) {
-                        mbar_arrive_tx(full, kQBox);
-                        tma_load_2d(smem_u32(sm.q[s][box]), &qmap, full, k0, int32_t(m0));
-                    } else {
-                        mbar_arrive_tx(full, kPBox);
-                        tma_load_2d(smem_u32(sm.p[s][box]), &pmap, full, k0 * 2, int32_t(n0 / 8));
-                    }
-                    last = g;
-                }
-            }
-            if (last >= 0) {
-                // this thread's last copy has landed before the CTA exits (at
-                // once unless another role gave up before consuming it)
-                volatile int no_abort = 0;
-                mbar_wait(full, uint32_t(last / kStages) & 1u, &no_abort, p.status, 100000000ull);
-            }
-        }
-    } else if (warp == kProducerWarps) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            int g = 0, it = 0;
-            bool ok = true, issued_any = false;
-            for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, ++it) {
-                const int b = it & 1;
-                if (it >= 2 &&
-                    !mbar_wait(smem_u32(&sm.tempty[b]), (uint32_t(it >> 1) & 1u) ^ 1u, abort_flag, p.status)) {
+        // lanes 0..kBoxes-1 copy the activation boxes of a stage, the next
+        // kBoxes lanes its packed weight boxes; the warp waits as a whole
+        int last = -1;   // global stage index of this warp's last issued stage
+        int base = 0;    // global stage index of the current tile's first k block
+        bool ok = true;
+        for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, base += KB) {
+            int64_t n0, m0;
+            tm.coords(t, n0, m0);
+            for (int kb = ((warp - base) % kProducerWarps + kProducerWarps) % kProducerWarps; kb < KB;
+                 kb += kProducerWarps) {
+                const int g = base + kb;
+                const int s = g % kQStages;
+                const uint32_t full = smem_u32(&sm.full[s]);
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.empty[s]), (uint32_t(g / kQStages) & 1u) ^ 1u,
+                                                       abort_flag, p.status))) {
                     ok = false;
                     break;
                 }
-                const uint32_t d_tmem = tmem + uint32_t(b * kBN);
-                for (int kb = 0; kb < KB; ++kb, ++g) {
-                    const int s = g % kStages;
-                    if (!mbar_wait(smem_u32(&sm.afull[s]), uint32_t(g / kStages) & 1u, abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a_stage = a_tmem0 + s * kACols;
 #pragma unroll
-                    for (int j = 0; j < kBK / kMmaK; ++j) {
-                        const uint32_t qaddr = smem_u32(sm.q[s][j / (kBoxK / kMmaK)]) + (j % (kBoxK / kMmaK)) * kMmaK;
-                        mma_i8_ts(d_tmem, a_stage + j * (kMmaK / 4), smem_desc_sw128(qaddr), kIdesc,
-                                  (kb > 0 || j > 0) ? 1u : 0u);
-                    }
-                    mma_commit(smem_u32(&sm.empty[s]));
-                    issued_any = true;
+                for (int box = 0; box < kBoxes; ++box) {
+                    const int k0 = kb * kBK + box * kBoxK;
+                    tma_load_2d_lane(box, smem_u32(sm.q[s][box]), &qmap, full, kQBox, k0, int32_t(m0));
+                    tma_load_2d_lane(kBoxes + box, smem_u32(sm.p[s][box]), &pmap, full, kPBox, k0 * 2,
+                                     int32_t(n0 / 8));
                 }
-                if (ok)
-                    mma_commit(smem_u32(&sm.tfull[b]));
-            }
-            if (issued_any) {
-                // every MMA has completed before tensor memory is released (at
-                // once unless the epilogue gave up before draining them)
-                mma_commit(smem_u32(&sm.drain));
-                volatile int no_abort = 0;
-                mbar_wait(smem_u32(&sm.drain), 0, &no_abort, p.status, 100000000ull);
+                last = g;
             }
         }
-    } else if (warp < kProducerWarps + 5) {
+        if (last >= 0) {
+            // the last stage's copies have landed before the CTA exits (at
+            // once unless another role gave up before consuming them)
+            volatile int no_abort = 0;
+            mbar_wait(smem_u32(&sm.full[last % kQStages]), uint32_t(last / kQStages) & 1u, &no_abort, p.status,
+                      100000000ull);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------ MMA issuer (whole warp, elected lane issues)
+        int g = 0, it = 0;
+        bool ok = true, issued_any = false;
+        for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, ++it) {
+            const int b = it & 1;
+            if (it >= 2 &&
+                !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.tempty[b]), (uint32_t(it >> 1) & 1u) ^ 1u,
+                                                   abort_flag, p.status))) {
+                ok = false;
+                break;
+            }
+            const uint32_t d_tmem = tmem + uint32_t(b * kBN);
+            for (int kb = 0; kb < KB; ++kb, ++g) {
+                const int s = g % kQStages, a = g % kAStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.afull[a]), uint32_t(g / kAStages) & 1u,
+                                                       abort_flag, p.status))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_stage = a_tmem0 + a * kACols;
+#pragma unroll
+                for (int j = 0; j < kBK / kMmaK; ++j) {
+                    const uint32_t qaddr = smem_u32(sm.q[s][j / (kBoxK / kMmaK)]) + (j % (kBoxK / kMmaK)) * kMmaK;
+                    mma_i8_ts(d_tmem, a_stage + j * (kMmaK / 4), smem_desc_sw128(qaddr), kIdesc,
+                              (kb > 0 || j > 0) ? 1u : 0u);
+                }
+                mma_commit(smem_u32(&sm.empty[s]));
+                mma_commit(smem_u32(&sm.aempty[a]));
+                issued_any = true;
+            }
+            if (ok)
+                mma_commit(smem_u32(&sm.tfull[b]));
+        }
+        if (issued_any) {
+            // every MMA has completed before tensor memory is released (at
+            // once unless the epilogue gave up before draining them)
+            mma_commit(smem_u32(&sm.drain));
+            volatile int no_abort = 0;
+            mbar_wait(smem_u32(&sm.drain), 0, &no_abort, p.status, 100000000ull);
+        }
+    } else if (warp < kEpiWarp0) {
         // ------------------------------------------------ expansion into tensor memory
+        const int grp = (warp - kExpWarp0) / 4;       // takes the stages g = grp (mod 2)
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
         const int rl = quarter * 32 + lane;           // weight row within the tile
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
@@ -375,38 +403,54 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
         bool ok = true;
         for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x) {
             for (int kb = 0; kb < KB; ++kb, ++g) {
-                const int s = g % kStages;
-                const uint32_t ph = uint32_t(g / kStages) & 1u;
-                // warp-uniform outcome: the tcgen05.st below is .sync.aligned
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.full[s]), ph, abort_flag, p.status))) {
+                if ((g & 1) != grp)
+                    continue;
+                const int s = g % kQStages, a = g % kAStages;
+                // warp-uniform outcomes: the tcgen05.st below is .sync.aligned
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.full[s]), uint32_t(g / kQStages) & 1u,
+                                                       abort_flag, p.status))) {
                     ok = false;
                     break;
                 }
+                uint4 c4[2 * kBoxes];
 #pragma unroll
                 for (int box = 0; box < kBoxes; ++box) {
                     const unsigned char *ps = sm.p[s][box] + (rl >> 3) * 256 + (rl & 7) * 16;
-                    const uint4 c0 = *reinterpret_cast<const uint4 *>(ps);
-                    const uint4 c1 = *reinterpret_cast<const uint4 *>(ps + 128);
-                    const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    c4[2 * box] = *reinterpret_cast<const uint4 *>(ps);
+                    c4[2 * box + 1] = *reinterpret_cast<const uint4 *>(ps + 128);
+                }
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.aempty[a]), (uint32_t(g / kAStages) & 1u) ^ 1u,
+                                                       abort_flag, p.status))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
                     uint32_t v[32];
 #pragma unroll
-                    for (int w = 0; w < 8; ++w) {
-                        v[4 * w + 0] = wd[w] & 0x03030303u;
-                        v[4 * w + 1] = (wd[w] >> 2) & 0x03030303u;
-                        v[4 * w + 2] = (wd[w] >> 4) & 0x03030303u;
-                        v[4 * w + 3] = (wd[w] >> 6) & 0x03030303u;
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        const uint4 cw = c4[2 * half + c2];
+                        const uint32_t wd[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            v[16 * c2 + 4 * w + 0] = wd[w] & 0x03030303u;
+                            v[16 * c2 + 4 * w + 1] = (wd[w] >> 2) & 0x03030303u;
+                            v[16 * c2 + 4 * w + 2] = (wd[w] >> 4) & 0x03030303u;
+                            v[16 * c2 + 4 * w + 3] = (wd[w] >> 6) & 0x03030303u;
+                        }
                     }
-                    tmem_st32(a_tmem0 + lane_addr + s * kACols + box * 32, v);
+                    tmem_st32(a_tmem0 + lane_addr + a * kACols + half * 32, v);
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(smem_u32(&sm.afull[s]));
+                mbar_arrive(smem_u32(&sm.afull[a]));
             }
         }
     } else {
         // ------------------------------------------------ epilogue
         const int quarter = warp & 3;
-        const int ew = warp - (kProducerWarps + 5);   // this warp's staging slice
+        const int ew = warp - kEpiWarp0;              // this warp's staging slice
         const int rl = quarter * 32 + lane;
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
         const float gamma = p.w_scale[0];
@@ -458,7 +502,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kProducerWarps) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
