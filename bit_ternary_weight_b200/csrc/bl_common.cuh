@@ -184,6 +184,18 @@ static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, vol
     }
 }
 
+// mbar_wait with its first test inline: when the phase has already completed
+// (the common case in a warp-specialised pipeline that runs ahead) no call is
+// made.  A function call in the issuing warp of tcgen05.mma was measured to
+// stall it for hundreds of cycles per stage.
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                               int *status)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    return mbar_wait(bar, parity, abort_flag, status);
+}
+
 // Bulk (non-tensor) TMA copy global -> shared, completion counted on `bar`.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
 {

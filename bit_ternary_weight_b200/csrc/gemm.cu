@@ -329,8 +329,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                 const int g = base + kb;
                 const int s = g % kQStages;
                 const uint32_t full = smem_u32(&sm.full[s]);
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.empty[s]), (uint32_t(g / kQStages) & 1u) ^ 1u,
-                                                       abort_flag, p.status))) {
+                if (!__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.empty[s]), (uint32_t(g / kQStages) & 1u) ^ 1u,
+                                                            abort_flag, p.status))) {
                     ok = false;
                     break;
                 }
@@ -358,16 +358,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
         for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, ++it) {
             const int b = it & 1;
             if (it >= 2 &&
-                !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.tempty[b]), (uint32_t(it >> 1) & 1u) ^ 1u,
-                                                   abort_flag, p.status))) {
+                !__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.tempty[b]), (uint32_t(it >> 1) & 1u) ^ 1u,
+                                                        abort_flag, p.status))) {
                 ok = false;
                 break;
             }
             const uint32_t d_tmem = tmem + uint32_t(b * kBN);
             for (int kb = 0; kb < KB; ++kb, ++g) {
                 const int s = g % kQStages, a = g % kAStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.afull[a]), uint32_t(g / kAStages) & 1u,
-                                                       abort_flag, p.status))) {
+                if (!__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.afull[a]), uint32_t(g / kAStages) & 1u,
+                                                            abort_flag, p.status))) {
                     ok = false;
                     break;
                 }
@@ -407,8 +407,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                     continue;
                 const int s = g % kQStages, a = g % kAStages;
                 // warp-uniform outcomes: the tcgen05.st below is .sync.aligned
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.full[s]), uint32_t(g / kQStages) & 1u,
-                                                       abort_flag, p.status))) {
+                if (!__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.full[s]), uint32_t(g / kQStages) & 1u,
+                                                            abort_flag, p.status))) {
                     ok = false;
                     break;
                 }
@@ -419,8 +419,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                     c4[2 * box] = *reinterpret_cast<const uint4 *>(ps);
                     c4[2 * box + 1] = *reinterpret_cast<const uint4 *>(ps + 128);
                 }
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.aempty[a]), (uint32_t(g / kAStages) & 1u) ^ 1u,
-                                                       abort_flag, p.status))) {
+                if (!__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.aempty[a]), (uint32_t(g / kAStages) & 1u) ^ 1u,
+                                                            abort_flag, p.status))) {
                     ok = false;
                     break;
                 }
@@ -470,7 +470,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
             }
             __syncwarp();
             if (!__all_sync(0xffffffffu,
-                            mbar_wait(smem_u32(&sm.tfull[b]), uint32_t(it >> 1) & 1u, abort_flag, p.status)))
+                            mbar_wait_fast(smem_u32(&sm.tfull[b]), uint32_t(it >> 1) & 1u, abort_flag, p.status)))
                 break;
             tc_fence_after();
             const int64_t n = n0 + rl;
