@@ -29,7 +29,7 @@
 //                the next accumulate into the other.
 // Tensor memory: D 2 x 128 columns + A 4 stages x 64 columns = 512 columns.
 //
-// Warp roles (480 threads):
+// Warp roles (608 threads):
 //   warps 0-1    TMA producers.  Warp w copies the stages g = w (mod 2): lanes
 //                0-1 the two activation boxes, lanes 2-3 the two packed weight
 //                boxes, side by side.  TMA copies issued
@@ -37,17 +37,19 @@
 //                spread over several threads, and over warps rather than lanes
 //                of one warp, because lanes that wait on different barriers
 //                move in lockstep.
-//   warp 2       tensor memory allocation; lane 0 issues tcgen05.mma.kind::i8.
-//                It waits on one barrier per stage, the expansion barrier: the
-//                expansion warps arrive there once the A stage is written and
-//                they have seen the stage's activation copies land.
+//   warp 2       tensor memory allocation; lane 0 issues tcgen05.mma.kind::i8
+//                after the stage's expansion barrier and its TMA barrier, the
+//                whole warp running the loop.
 //   warps 3-10   expansion of the packed weights into tensor memory, two groups
 //                of four warps (one per TMEM lane quarter) taking alternate
 //                stages: an mbarrier check costs a couple of hundred cycles
 //                even when the phase has completed, and one stage's expansion
 //                with its checks takes longer than the stage's MMAs.
-//   warps 11-14  epilogue: tcgen05.ld, subtract the row sum, rescale, store.
-//                Per-token d and row sums are staged in shared memory per warp.
+//   warps 11-18  epilogue: tcgen05.ld, subtract the row sum, rescale, store;
+//                two warps per TMEM lane quarter, each draining 64 token
+//                columns, so a tile's epilogue fits in the next tile's main
+//                loop even at K = 2560.  Per-token d and row sums are staged
+//                in shared memory per warp.
 //
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA
 // records BL_ERR_TIMEOUT in the device status word, every role leaves its
@@ -75,13 +77,16 @@ constexpr int kProducerWarps = 2;
 constexpr int kMmaWarp = kProducerWarps;
 constexpr int kExpWarp0 = kMmaWarp + 1;
 constexpr int kEpiWarp0 = kExpWarp0 + 4 * kExpGroups;
-constexpr int kThreads = 32 * (kEpiWarp0 + 4);
+constexpr int kEpiSplit = 2;                 // epilogue warps per TMEM lane quarter
+constexpr int kEpiCols = kBN / kEpiSplit;    // token columns one epilogue warp drains
+constexpr int kThreads = 32 * (kEpiWarp0 + 4 * kEpiSplit);
 constexpr int kMmaK = 32;    // k per tcgen05.mma.kind::i8
 constexpr uint32_t kTmemCols = 512;  // D: 2 x 128 columns; A: kAStages x 64 columns
 constexpr uint32_t kQBox = kBN * kBoxK;        // 16 KB of int8 activations per box
 constexpr uint32_t kPBox = kBM * kBoxK / 4;    // 4 KB of packed weights per box
 constexpr uint32_t kACols = kBK / 4;           // TMEM columns of one expanded A stage
 static_assert(2 * kBN + kAStages * int(kACols) == int(kTmemCols), "tensor memory budget");
+static_assert(kBoxK == 128 && kMmaK == 32, "descriptor steps of mma_stage8");
 
 struct GemmParams {
     const float *w_scale;
@@ -114,23 +119,44 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
                  : "memory");
 }
 
-// The MMA role runs on a whole warp in warp-uniform control flow and issues
-// each tcgen05 operation from one lane chosen by elect.sync (the lowest active
-// lane, so always the same thread: tcgen05.commit tracks the operations of the
-// thread that executes it).  Issued from a single-lane divergent region
-// instead, back-to-back 128x128x32 MMAs measured ~120 cycles apiece once the
-// loop also waited on an mbarrier, against 64 in warp-uniform code.
+// The MMA role runs on a whole warp in warp-uniform control flow; each
+// tcgen05.mma and tcgen05.commit is an instruction predicated on lane 0 inside
+// that uniform code.  Two points matter:
+//   - issued from a single-lane divergent region instead, back-to-back
+//     128x128x32 MMAs measured ~120 cycles apiece once the loop also waited on
+//     an mbarrier, against 64 in warp-uniform code;
+//   - the issuing lane is fixed, not chosen by elect.sync: tcgen05.commit
+//     tracks only the MMAs of the thread that executes it, and leaders elected
+//     separately for the MMAs and for the commit were seen to differ, which let
+//     a ring slot be released while its MMAs still read it.
 
-// D[tmem] (+)= A[tmem] * B[smem]^T, int8 inputs, int32 accumulate.
-__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate)
+// One pipeline stage: eight MMAs (k = 0..255) issued by lane 0.
+// b_desc0 describes the stage's first 32 k of activations; the start address
+// field advances by 32 B (2 units) per MMA within a 128-k box and by one box
+// (16 KB, 1024 units) after four MMAs.  A advances 8 TMEM columns per MMA.
+// accumulate_first = 0 makes the first MMA overwrite D (first stage of a tile).
+__device__ __forceinline__ void mma_stage8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc0, uint32_t idesc,
+                                           uint32_t accumulate_first)
 {
+    static_assert(kBK / kMmaK == 8 && kBoxK / kMmaK == 4, "stage shape");
     asm volatile(
-        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
-        "elect.sync r|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred e, p, t;\n\t.reg .b32 r;\n\t"
+        "mov.u32 r, %%laneid;\n\t"
+        "setp.eq.u32 e, r, 0;\n\t"
+        "setp.ne.b32 p, %12, 0;\n\t"
+        "setp.ne.b32 t, %19, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %3, %11, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%2], %4, %11, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%13], %5, %11, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%14], %6, %11, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%15], %7, %11, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%16], %8, %11, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%17], %9, %11, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%18], %10, %11, t;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(a_tmem + 8), "l"(b_desc0), "l"(b_desc0 + 2), "l"(b_desc0 + 4), "l"(b_desc0 + 6),
+        "l"(b_desc0 + 1024), "l"(b_desc0 + 1026), "l"(b_desc0 + 1028), "l"(b_desc0 + 1030), "r"(idesc),
+        "r"(accumulate_first), "r"(a_tmem + 16), "r"(a_tmem + 24), "r"(a_tmem + 32), "r"(a_tmem + 40),
+        "r"(a_tmem + 48), "r"(a_tmem + 56), "r"(1u)
         : "memory");
 }
 
@@ -138,7 +164,8 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
 {
     asm volatile(
         "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
-        "elect.sync r|e, 0xffffffff;\n\t"
+        "mov.u32 r, %%laneid;\n\t"
+        "setp.eq.u32 e, r, 0;\n\t"
         "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
         : "memory");
 }
@@ -159,39 +186,33 @@ __device__ __forceinline__ void tma_load_2d_lane(uint32_t who, uint32_t dst, con
         : "memory");
 }
 
-// Thirty-two consecutive 32-bit TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
+// tcgen05.ld and tcgen05.st move registers asynchronously: the destination
+// registers of a load are valid only after tcgen05.wait::ld, and the source
+// registers of a store must stay unchanged until tcgen05.wait::st.  Each
+// access is therefore written together with its wait in one asm statement,
+// so that the compiler neither reads a loaded register early nor reuses a
+// stored one while the store is in flight.
+
+// Sixty-four consecutive 32-bit TMEM columns of this thread's lane, stored.
+__device__ __forceinline__ void tmem_st64_wait(uint32_t taddr, const uint32_t (&v)[64])
 {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-        "%28, %29, %30, %31, %32};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
-        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
-        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]), "r"(v[32]), "r"(v[33]), "r"(v[34]), "r"(v[35]), "r"(v[36]), "r"(v[37]), "r"(v[38]), "r"(v[39]), "r"(v[40]), "r"(v[41]), "r"(v[42]), "r"(v[43]), "r"(v[44]), "r"(v[45]), "r"(v[46]), "r"(v[47]), "r"(v[48]), "r"(v[49]), "r"(v[50]), "r"(v[51]), "r"(v[52]), "r"(v[53]), "r"(v[54]), "r"(v[55]), "r"(v[56]), "r"(v[57]), "r"(v[58]), "r"(v[59]), "r"(v[60]), "r"(v[61]), "r"(v[62]), "r"(v[63])
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
+// Thirty-two consecutive 32-bit TMEM columns of this thread's lane, loaded.
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&v)[32])
 {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-        "%28, %29, %30, %31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
-          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
-          "=r"(v[31])
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
         : "r"(taddr)
         : "memory");
 }
-
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms of
 // 1024 bytes stacked along the token dimension (stride byte offset 1024).
@@ -218,8 +239,8 @@ struct Smem {
     unsigned char q[kQStages][kBoxes][kQBox];
     unsigned char p[kQStages][kBoxes][kPBox];
     // per epilogue warp: d and row sums of the current tile's 128 tokens
-    float ep_d[4][kBN];
-    int32_t ep_r[4][kBN];
+    float ep_d[4 * kEpiSplit][kEpiCols];
+    int32_t ep_r[4 * kEpiSplit][kEpiCols];
     uint64_t full[kQStages];     // activation and packed boxes landed
     uint64_t empty[kQStages];    // the slot's bytes are no longer needed (MMAs completed)
     uint64_t afull[kAStages];    // A expanded into tensor memory (and its activations landed)
@@ -258,21 +279,30 @@ __device__ __forceinline__ void store_out<float>(float *y, int64_t idx, float v)
 }
 
 // One 32-token chunk of the epilogue for this thread's weight row n.
-template <typename T, bool FULL>
+template <typename T, bool FULL, bool DBG>
 __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], const float *sd, const int32_t *sr,
                                                int64_t n, int64_t m0, const GemmParams &p, float gamma)
 {
-    T *y = static_cast<T *>(p.y);
+    T *y = static_cast<T *>(p.y) + m0 * p.ldy + n;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-        const int64_t m = m0 + j;
-        if (FULL || m < p.M) {
+        if (FULL || m0 + j < p.M) {
             const int a = int(v[j]) - sr[j];
-            if (p.acc_dbg)
-                p.acc_dbg[m * p.N + n] = a;
-            store_out<T>(y, m * p.ldy + n, rescale1(a, sd[j], gamma));
+            if (DBG)
+                p.acc_dbg[(m0 + j) * p.N + n] = a;
+            store_out<T>(y, int64_t(j) * p.ldy, rescale1(a, sd[j], gamma));
         }
     }
+}
+
+template <typename T, bool DBG>
+__device__ __forceinline__ void epilogue_chunk_any(const uint32_t (&v)[32], const float *sd, const int32_t *sr,
+                                                   int64_t n, int64_t m0, const GemmParams &p, float gamma)
+{
+    if (m0 + 32 <= p.M)
+        epilogue_chunk<T, true, DBG>(v, sd, sr, n, m0, p, gamma);
+    else
+        epilogue_chunk<T, false, DBG>(v, sd, sr, n, m0, p, gamma);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -298,7 +328,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&sm.tfull[b]), 1);
-            mbar_init(smem_u32(&sm.tempty[b]), 128);
+            mbar_init(smem_u32(&sm.tempty[b]), 128 * kEpiSplit);
         }
         mbar_init(smem_u32(&sm.drain), 1);
         sm.abort_flag = 0;
@@ -352,7 +382,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                       100000000ull);
         }
     } else if (warp == kMmaWarp) {
-        // ------------------------------------------------ MMA issuer (whole warp, elected lane issues)
+        // ------------------------------------------------ MMA issuer (whole warp, lane 0 issues)
+        const uint64_t q_desc0 = smem_desc_sw128(smem_u32(sm.q[0][0]));   // slot s adds s * 40 KB >> 4
         int g = 0, it = 0;
         bool ok = true, issued_any = false;
         for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, ++it) {
@@ -366,19 +397,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
             const uint32_t d_tmem = tmem + uint32_t(b * kBN);
             for (int kb = 0; kb < KB; ++kb, ++g) {
                 const int s = g % kQStages, a = g % kAStages;
+                // the tensor core reads the activation tile through the async
+                // proxy: wait on the barrier its TMA completes, not only on the
+                // expansion barrier that follows it
                 if (!__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.afull[a]), uint32_t(g / kAStages) & 1u,
-                                                            abort_flag, p.status))) {
+                                                            abort_flag, p.status) &&
+                                                 mbar_wait_fast(smem_u32(&sm.full[s]), uint32_t(g / kQStages) & 1u,
+                                                                abort_flag, p.status))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a_stage = a_tmem0 + a * kACols;
-#pragma unroll
-                for (int j = 0; j < kBK / kMmaK; ++j) {
-                    const uint32_t qaddr = smem_u32(sm.q[s][j / (kBoxK / kMmaK)]) + (j % (kBoxK / kMmaK)) * kMmaK;
-                    mma_i8_ts(d_tmem, a_stage + j * (kMmaK / 4), smem_desc_sw128(qaddr), kIdesc,
-                              (kb > 0 || j > 0) ? 1u : 0u);
-                }
+                mma_stage8(d_tmem, a_tmem0 + a * kACols, q_desc0 + uint64_t(s) * (kBoxes * kQBox >> 4), kIdesc,
+                           kb > 0 ? 1u : 0u);
                 mma_commit(smem_u32(&sm.empty[s]));
                 mma_commit(smem_u32(&sm.aempty[a]));
                 issued_any = true;
@@ -425,32 +456,28 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                     break;
                 }
                 tc_fence_after();
+                uint32_t v[64];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t v[32];
+                for (int c = 0; c < 2 * kBoxes; ++c) {
+                    const uint32_t wd[4] = {c4[c].x, c4[c].y, c4[c].z, c4[c].w};
 #pragma unroll
-                    for (int c2 = 0; c2 < 2; ++c2) {
-                        const uint4 cw = c4[2 * half + c2];
-                        const uint32_t wd[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            v[16 * c2 + 4 * w + 0] = wd[w] & 0x03030303u;
-                            v[16 * c2 + 4 * w + 1] = (wd[w] >> 2) & 0x03030303u;
-                            v[16 * c2 + 4 * w + 2] = (wd[w] >> 4) & 0x03030303u;
-                            v[16 * c2 + 4 * w + 3] = (wd[w] >> 6) & 0x03030303u;
-                        }
+                    for (int w = 0; w < 4; ++w) {
+                        v[16 * c + 4 * w + 0] = wd[w] & 0x03030303u;
+                        v[16 * c + 4 * w + 1] = (wd[w] >> 2) & 0x03030303u;
+                        v[16 * c + 4 * w + 2] = (wd[w] >> 4) & 0x03030303u;
+                        v[16 * c + 4 * w + 3] = (wd[w] >> 6) & 0x03030303u;
                     }
-                    tmem_st32(a_tmem0 + lane_addr + a * kACols + half * 32, v);
                 }
-                tmem_wait_st();
+                tmem_st64_wait(a_tmem0 + lane_addr + a * kACols, v);
                 tc_fence_before();
                 mbar_arrive(smem_u32(&sm.afull[a]));
             }
         }
     } else {
         // ------------------------------------------------ epilogue
-        const int quarter = warp & 3;
         const int ew = warp - kEpiWarp0;              // this warp's staging slice
+        const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+        const int c0 = (ew / 4) * kEpiCols;           // first token column this warp drains
         const int rl = quarter * 32 + lane;
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
         const float gamma = p.w_scale[0];
@@ -463,8 +490,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
             tm.coords(t, n0, m0);
             __syncwarp();
 #pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) {
-                const int64_t m = m0 + c * 32 + lane;
+            for (int c = 0; c < kEpiCols / 32; ++c) {
+                const int64_t m = m0 + c0 + c * 32 + lane;
                 sd[c * 32 + lane] = m < p.M ? __ldg(p.d + m) : 0.0f;
                 sr[c * 32 + lane] = m < p.M ? __ldg(p.rowsum + m) : 0;
             }
@@ -474,24 +501,24 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                 break;
             tc_fence_after();
             const int64_t n = n0 + rl;
-            const bool full_m = m0 + kBN <= p.M;
 #pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
+            for (int c = 0; c < kEpiCols / 32; ++c) {
                 uint32_t v[32];
-                tmem_ld32(tmem + lane_addr + uint32_t(b * kBN + c * 32), v);
-                tmem_wait_ld();
+                tmem_ld32_wait(tmem + lane_addr + uint32_t(b * kBN + c0 + c * 32), v);
                 if (n < p.N) {
-                    const int64_t mc = m0 + c * 32;
+                    const int64_t mc = m0 + c0 + c * 32;
+                    const float *d32 = sd + c * 32;
+                    const int32_t *r32 = sr + c * 32;
                     if (p.yt == BL_BF16) {
-                        if (full_m)
-                            epilogue_chunk<__nv_bfloat16, true>(v, sd + c * 32, sr + c * 32, n, mc, p, gamma);
+                        if (p.acc_dbg)
+                            epilogue_chunk_any<__nv_bfloat16, true>(v, d32, r32, n, mc, p, gamma);
                         else
-                            epilogue_chunk<__nv_bfloat16, false>(v, sd + c * 32, sr + c * 32, n, mc, p, gamma);
+                            epilogue_chunk_any<__nv_bfloat16, false>(v, d32, r32, n, mc, p, gamma);
                     } else {
-                        if (full_m)
-                            epilogue_chunk<float, true>(v, sd + c * 32, sr + c * 32, n, mc, p, gamma);
+                        if (p.acc_dbg)
+                            epilogue_chunk_any<float, true>(v, d32, r32, n, mc, p, gamma);
                         else
-                            epilogue_chunk<float, false>(v, sd + c * 32, sr + c * 32, n, mc, p, gamma);
+                            epilogue_chunk_any<float, false>(v, d32, r32, n, mc, p, gamma);
                     }
                 }
             }
