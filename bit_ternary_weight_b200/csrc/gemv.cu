@@ -79,6 +79,7 @@ struct Smem {
     float scale[MT];
     float d[MT];
     int r[MT];
+    float wscale[kGemvMaxProblems];   // each problem's gamma_eff, read before the dependency wait
     int sacc[groups_per_phase<MT>()][MT][8];
     // followed by the weight ring and the int8 activations (M*K)
 };
@@ -399,8 +400,16 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p)
             i_prob = locate(p, i_group, gl);
             i_to_jump = (p.gstart[i_prob + 1] - i_group) * P - j0;
         }
-        if (first)
+        if (first) {
             pdl_launch_dependents();
+            // independent of the preceding launch: weight scales, accumulators
+#pragma unroll
+            for (int i = 0; i < kGemvMaxProblems; ++i)
+                if (tid == i && i < p.count)
+                    sm.wscale[i] = __ldg(p.prob[i].w_scale);
+            for (int i = tid; i < nG * MT * 8; i += kThreads)
+                (&sm.sacc[0][0][0])[i] = 0;
+        }
 #pragma unroll
         for (int s = 0; s < STAGES; ++s)
             issue(s);
@@ -413,11 +422,22 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p)
                 quantize_prologue_1<MT, MODE == MODE_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
             else
                 quantize_prologue<MT, MODE == MODE_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
+        } else {
+            for (int i = tid; i < nG * MT * 8; i += kThreads)
+                (&sm.sacc[0][0][0])[i] = 0;
+        }
+        __syncthreads();
+        if (first) {
+            // the activations' row sums, folded once for the epilogues
+            if (tid < MT) {
+                int r = 0;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w)
+                    r += sm.bsum[w][tid];
+                sm.r[tid] = r;
+            }
             first = false;
         }
-        for (int i = tid; i < nG * MT * 8; i += kThreads)
-            (&sm.sacc[0][0][0])[i] = 0;
-        __syncthreads();
 
 #pragma unroll
         for (int m = 0; m < MT; ++m)
@@ -505,14 +525,10 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p)
             const GemvProblem &pr = p.prob[pi];
             const int64_t row = gl * 8 + rr;
             if (row < pr.N) {
-                int r = 0;
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w)
-                    r += sm.bsum[w][m];
-                const int a = sm.sacc[gi][m][rr] - r;
+                const int a = sm.sacc[gi][m][rr] - sm.r[m];
                 if (pr.acc_dbg)
                     pr.acc_dbg[int64_t(m) * pr.N + row] = a;
-                store_y(pr.y, p.yt, int64_t(m) * pr.ldy + row, rescale1(a, sm.d[m], pr.w_scale[0]));
+                store_y(pr.y, p.yt, int64_t(m) * pr.ldy + row, rescale1(a, sm.d[m], sm.wscale[pi]));
             }
         }
         __syncthreads();
