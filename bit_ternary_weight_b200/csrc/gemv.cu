@@ -148,14 +148,19 @@ __device__ __forceinline__ void quantize_prologue_1(const Params &p, Smem<MT> &s
                 amax = fmaxf(amax, fabsf(f[i][j]));
         }
     }
-    amax = warp_max(amax);
+    // per-thread maxima are finite and >= 0 (fmaxf from 0 drops NaN), so
+    // their bit patterns order like the values: one redux per warp
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
     if (lane == 0)
-        sm.bmax[warp][0] = amax;
+        sm.bmax[warp][0] = __uint_as_float(wmax);
     __syncthreads();
-    float a = sm.bmax[0][0];
+    static_assert(MT == 1 && kWarps % 4 == 0, "bmax of one token is kWarps contiguous floats");
+    float a = 0.0f;
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w)
-        a = fmaxf(a, sm.bmax[w][0]);
+    for (int w = 0; w < kWarps; w += 4) {
+        const float4 b4 = *reinterpret_cast<const float4 *>(&sm.bmax[w][0]);
+        a = fmaxf(fmaxf(a, b4.x), fmaxf(b4.y, fmaxf(b4.z, b4.w)));
+    }
     const float a_eff = fmaxf(a, kEps);
     const float s = __fdiv_rn(kQb, a_eff);
     if (tid == 0)
@@ -176,7 +181,7 @@ __device__ __forceinline__ void quantize_prologue_1(const Params &p, Smem<MT> &s
             *reinterpret_cast<uint2 *>(qs + int64_t(c) * 8) = make_uint2(lo, hi);
         }
     }
-    sum = warp_sum(sum);
+    sum = __reduce_add_sync(0xffffffffu, sum);
     if (lane == 0)
         sm.bsum[warp][0] = sum;
     // the barrier before the main loop publishes qs, d and bsum
@@ -301,7 +306,6 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p)
     const int C = Ki / 64, P = (C + 3) / 4;
     const int64_t slab = int64_t(C) * 128;
     const int csub = lane >> 3;
-    const int64_t NGt = p.gstart[p.count];
     const int bx = blockIdx.x;
     const int64_t g_begin = bx * p.gpc_base + (bx < p.gpc_rem ? bx : p.gpc_rem);
     const int64_t g_end = g_begin + p.gpc_base + (bx < p.gpc_rem ? 1 : 0);
@@ -418,10 +422,14 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p)
             pdl_wait();
             if constexpr (MODE == MODE_Q)
                 copy_prologue<MT>(p, sm, qs);
-            else if (MT == 1 && p.K <= int64_t(16) * kThreads)
-                quantize_prologue_1<MT, MODE == MODE_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
-            else
+            else if constexpr (MT == 1) {
+                if (p.K <= int64_t(16) * kThreads)
+                    quantize_prologue_1<MT, MODE == MODE_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
+                else
+                    quantize_prologue<MT, MODE == MODE_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
+            } else {
                 quantize_prologue<MT, MODE == MODE_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
+            }
         } else {
             for (int i = tid; i < nG * MT * 8; i += kThreads)
                 (&sm.sacc[0][0][0])[i] = 0;
@@ -518,8 +526,17 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_kernel(const Params p)
         __syncthreads();
         // rescale and write the phase's rows
         for (int idx = tid; idx < nG * 8 * p.M; idx += kThreads) {
-            const int gi = idx / (8 * p.M), rem = idx % (8 * p.M);
-            const int m = rem >> 3, rr = rem & 7;
+            int gi, m, rr;
+            if constexpr (MT == 1) {
+                gi = idx >> 3;
+                m = 0;
+                rr = idx & 7;
+            } else {
+                gi = idx / (8 * p.M);
+                const int rem = idx % (8 * p.M);
+                m = rem >> 3;
+                rr = rem & 7;
+            }
             int64_t gl;
             const int pi = locate(p, ph0 + gi, gl);
             const GemvProblem &pr = p.prob[pi];
