@@ -111,12 +111,20 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest of the ranks' values (device times are reported as the max)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(bytes_per_step_per_rank: float, steps: int, world: int, t_max: float) -> float:
+    """Whole-job GB/s: every rank streams its own weights (weak scaling); the
+    job takes as long as its slowest rank."""
+    return bytes_per_step_per_rank * steps * world / t_max / 1e9
 
 
 # ---------------------------------------------------------------- clocks
@@ -454,7 +462,7 @@ def run_ours(args, world, rank, local):
         t = time_graph(graph, args.steps, world)
     clocks = clk.summary()
     t = max_over_ranks(t, world)
-    value = step_bytes * args.steps * world / t / 1e9
+    value = job_throughput(step_bytes, args.steps, world, t)
     ms_per_step = t / args.steps * 1000
 
     # e2e: host activations in, host outputs back, every step, through the same
@@ -476,7 +484,7 @@ def run_ours(args, world, rank, local):
     e.record()
     torch.cuda.synchronize()
     t_e2e = max_over_ranks(s.elapsed_time(e) / 1000.0, world)
-    e2e_value = step_bytes * args.steps * world / t_e2e / 1e9
+    e2e_value = job_throughput(step_bytes, args.steps, world, t_e2e)
 
     # eager (no graph) public-API loop, for context
     torch.cuda.synchronize()
