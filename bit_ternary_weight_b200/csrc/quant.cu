@@ -7,17 +7,30 @@
 //   d_m = a_m / 127;  rowsum_m = sum_k q.
 //
 // One CTA per token.  The token's row is read once into registers (16-byte
-// vectors, eight elements each), reduced for the absmax, quantised from the
-// registers and written as 8-byte int8 vectors; a second block reduction gives
-// the row sum.  Rows longer than the register budget are read a second time
-// (from L1/L2).  HBM-bound: M*K*(2 + 1) bytes for bf16 input.
+// vectors: raw bf16, eight elements each, or fp32 as floats), reduced for the
+// absmax, quantised from the registers and written as 8-byte int8 vectors; a
+// second block reduction gives the row sum.  Rows longer than the register
+// budget are read a second time (from L1/L2).  HBM-bound: M*K*(2 + 1) bytes
+// for bf16 input.  Keeping bf16 rows raw halves their registers, so more CTAs
+// (and more bytes of x) are in flight per SM: the kernel's time per token is
+// mostly load latency.
 #include "bl_common.cuh"
 
 namespace bl {
 namespace {
 
-constexpr int kQuantThreads = 256;
-constexpr int kQuantRegChunks = 4;  // 8-element chunks kept in registers per thread
+constexpr int kQuantThreads = 128;
+constexpr int kQuantRegChunks = 8;  // 8-element chunks kept in registers per thread (K <= 8192)
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float f[8])
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
 
 template <int XT>
 __global__ void __launch_bounds__(kQuantThreads)
@@ -32,17 +45,38 @@ quantize_act_kernel(const void *__restrict__ x, int64_t K, int64_t ldx,
     const int64_t chunks = K / 8;
     const int64_t xrow = m * ldx;
     const bool in_regs = chunks <= int64_t(kQuantThreads) * kQuantRegChunks;
+    // register copy of the row: raw bf16 vectors, or eight floats per chunk
+    constexpr int kRegF = XT == BL_BF16 ? 1 : 8;
+    uint4 raw[XT == BL_BF16 ? kQuantRegChunks : 1];
+    float v[XT == BL_BF16 ? 1 : kQuantRegChunks][kRegF];
+    auto chunk_f32 = [&](int i, float f[8]) {
+        if constexpr (XT == BL_BF16) {
+            bf16x8_to_f32(raw[i], f);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                f[j] = v[i][j];
+        }
+    };
 
-    float v[kQuantRegChunks][8];
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < kQuantRegChunks; ++i) {
         const int64_t c = tid + int64_t(i) * kQuantThreads;
         if (in_regs && c < chunks) {
-            load8<XT>(x, xrow + c * 8, v[i]);
+            float f[8];
+            if constexpr (XT == BL_BF16) {
+                raw[i] = ld_ro_v4(static_cast<const __nv_bfloat16 *>(x) + xrow + c * 8);
+                bf16x8_to_f32(raw[i], f);
+            } else {
+                load8<XT>(x, xrow + c * 8, f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    v[i][j] = f[j];
+            }
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-                amax = fmaxf(amax, fabsf(v[i][j]));
+                amax = fmaxf(amax, fabsf(f[j]));
         }
     }
     if (!in_regs) {
@@ -54,7 +88,9 @@ quantize_act_kernel(const void *__restrict__ x, int64_t K, int64_t ldx,
                 amax = fmaxf(amax, fabsf(f[j]));
         }
     }
-    amax = warp_max(amax);
+    // per-thread maxima are finite and >= 0 (fmaxf from 0 drops NaN), so
+    // their bit patterns order like the values
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
     if (lane == 0)
         s_red[warp] = amax;
     __syncthreads();
@@ -82,8 +118,11 @@ quantize_act_kernel(const void *__restrict__ x, int64_t K, int64_t ldx,
 #pragma unroll
         for (int i = 0; i < kQuantRegChunks; ++i) {
             const int64_t c = tid + int64_t(i) * kQuantThreads;
-            if (c < chunks)
-                emit(c, v[i]);
+            if (c < chunks) {
+                float f[8];
+                chunk_f32(i, f);
+                emit(c, f);
+            }
         }
     } else {
         for (int64_t c = tid; c < chunks; c += kQuantThreads) {
@@ -92,7 +131,7 @@ quantize_act_kernel(const void *__restrict__ x, int64_t K, int64_t ldx,
             emit(c, f);
         }
     }
-    sum = warp_sum(sum);
+    sum = __reduce_add_sync(0xffffffffu, sum);
     if (lane == 0)
         s_sum[warp] = sum;
     __syncthreads();
