@@ -278,13 +278,26 @@ def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda"):
         del W
     x = si.activations(M, K, seed=5).to(device)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+    # the path bl.linear takes: fused dp4a GEMV for few tokens, else quantise +
+    # tensor-core GEMM (both launches timed)
+    fused = M <= bl.GEMV_FUSED_MAX_M
+    if fused:
+        call = lambda wt: bl.gemv_fused(wt, x, out=y)  # noqa: E731
+    else:
+        q = torch.empty(M, K, dtype=torch.int8, device=device)
+        d = torch.empty(M, dtype=torch.float32, device=device)
+        r = torch.empty(M, dtype=torch.int32, device=device)
+
+        def call(wt):
+            bl.quantize_act(x, out=(q, d, r))
+            bl.gemm(wt, q, d, r, out=y)
     for i in range(min(copies, 8)):
-        bl.gemv_fused(ws[i], x, out=y)
+        call(ws[i])
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(iters):
-            bl.gemv_fused(ws[i % copies], x, out=y)
+            call(ws[i % copies])
     g.replay()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -295,7 +308,8 @@ def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda"):
     t = s.elapsed_time(e) / 1000.0 / iters
     del g, ws
     return {"K": K, "N": N, "M": M, "us": t * 1e6, "GBps": nbytes / t / 1e9,
-            "weight_copies": copies}
+            "weight_copies": copies,
+            "path": "fused dp4a GEMV" if fused else "quantise + tcgen05 GEMM (32-token tiles)"}
 
 
 def isolated_binary(bl, K, N, iters=100, device="cuda"):

@@ -170,14 +170,18 @@ def pack_noalloc(W: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor) -
     return TernaryWeight(packed, w_scale, N, K)
 
 
-def quantize_act(x: torch.Tensor):
-    """Per-token absmax int8: returns (q int8 [M,K], d fp32 [M], rowsum int32 [M])."""
+def quantize_act(x: torch.Tensor, out=None):
+    """Per-token absmax int8: returns (q int8 [M,K], d fp32 [M], rowsum int32 [M]),
+    written into out=(q, d, rowsum) when given."""
     if x.dim() == 1:
         x = x.unsqueeze(0)
     M, K = x.shape
-    q = torch.empty(M, K, dtype=torch.int8, device=x.device)
-    d = torch.empty(M, dtype=torch.float32, device=x.device)
-    r = torch.empty(M, dtype=torch.int32, device=x.device)
+    if out is None:
+        q = torch.empty(M, K, dtype=torch.int8, device=x.device)
+        d = torch.empty(M, dtype=torch.float32, device=x.device)
+        r = torch.empty(M, dtype=torch.int32, device=x.device)
+    else:
+        q, d, r = out
     _check(_lib.bitlinear_quantize_act(_ptr(x), _dt(x.dtype), M, K, x.stride(0), _ptr(q),
                                        _ptr(d), _ptr(r), _stream(x.device)),
            "bitlinear_quantize_act")
@@ -267,10 +271,14 @@ def gemm(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc
     return out
 
 
+GEMV_FUSED_MAX_M = 7   # from 8 tokens on, quantise + tensor-core GEMM is faster
+
+
 def linear(w: TernaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16):
-    """y = BitLinear(x): the fused GEMV for M <= 16 tokens, else quantise + GEMM."""
+    """y = BitLinear(x): the fused dp4a GEMV for up to 7 tokens, else quantise +
+    tensor-core GEMM."""
     x2 = x.reshape(-1, x.shape[-1])
-    if x2.shape[0] <= GEMV_MAX_M and x2.shape[0] * w.K <= 163840:
+    if x2.shape[0] <= GEMV_FUSED_MAX_M and x2.shape[0] * w.K <= 163840:
         y = gemv_fused(w, x2, out_dtype)
     else:
         q, d, r = quantize_act(x2)

@@ -255,6 +255,7 @@ int check_gemv_common(const uint8_t *packed, const float *w_scale, int64_t N,
 }
 
 constexpr int64_t kGemvMaxM = 16;
+constexpr int64_t kGemvTensorM = 8;     // bitlinear_gemv runs on the tcgen05 path from here on
 constexpr int64_t kGemvMaxMK = 163840;
 
 }  // namespace
@@ -279,6 +280,10 @@ int bitlinear_gemv(const uint8_t *packed, const float *w_scale, int64_t N, int64
     if ((st = check_dev_ptrs({packed, w_scale, q, d, rowsum, y, acc_dbg})))
         return st;
     GemvArgs a{packed, w_scale, N, K, M, q, d, rowsum, nullptr, BL_F32, 0, y, yt, ldy, acc_dbg};
+    // from kGemvTensorM tokens on, dp4a work grows with M while the tensor
+    // cores are idle: the product runs on the tcgen05 path (same results)
+    if (M >= kGemvTensorM)
+        return launch_gemm(a, nullptr, 0, static_cast<cudaStream_t>(stream));
     return launch_gemv(a, false, static_cast<cudaStream_t>(stream));
 }
 

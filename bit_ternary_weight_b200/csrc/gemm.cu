@@ -66,7 +66,6 @@ namespace bl {
 namespace {
 
 constexpr int kBM = 128;     // weight rows per tile (MMA M)
-constexpr int kBN = 128;     // tokens per tile (MMA N)
 constexpr int kBK = 256;     // k per pipeline stage: eight MMAs between barrier waits
 constexpr int kBoxK = 128;   // k per TMA box (one 128-byte swizzle span of activations)
 constexpr int kBoxes = kBK / kBoxK;
@@ -77,16 +76,29 @@ constexpr int kProducerWarps = 2;
 constexpr int kMmaWarp = kProducerWarps;
 constexpr int kExpWarp0 = kMmaWarp + 1;
 constexpr int kEpiWarp0 = kExpWarp0 + 4 * kExpGroups;
-constexpr int kEpiSplit = 2;                 // epilogue warps per TMEM lane quarter
-constexpr int kEpiCols = kBN / kEpiSplit;    // token columns one epilogue warp drains
-constexpr int kThreads = 32 * (kEpiWarp0 + 4 * kEpiSplit);
 constexpr int kMmaK = 32;    // k per tcgen05.mma.kind::i8
-constexpr uint32_t kTmemCols = 512;  // D: 2 x 128 columns; A: kAStages x 64 columns
-constexpr uint32_t kQBox = kBN * kBoxK;        // 16 KB of int8 activations per box
+constexpr uint32_t kTmemCols = 512;  // D: 2 x BN columns in [0, 256); A: kAStages x 64 columns in [256, 512)
+constexpr uint32_t kDCols = 256;
 constexpr uint32_t kPBox = kBM * kBoxK / 4;    // 4 KB of packed weights per box
 constexpr uint32_t kACols = kBK / 4;           // TMEM columns of one expanded A stage
-static_assert(2 * kBN + kAStages * int(kACols) == int(kTmemCols), "tensor memory budget");
-static_assert(kBoxK == 128 && kMmaK == 32, "descriptor steps of mma_stage8");
+static_assert(kDCols + kAStages * kACols == kTmemCols, "tensor memory budget");
+
+// Shapes that depend on the token tile BN (MMA N): 128 for prefill, 32 for
+// small batches (M <= 32), where a 128-token tile would be mostly padding.
+template <int BN>
+struct TileCfg {
+    static_assert(BN == 32 || BN == 128, "token tile");
+    static constexpr int kEpiSplit = BN >= 64 ? 2 : 1;      // epilogue warps per TMEM lane quarter
+    static constexpr int kEpiCols = BN / kEpiSplit;         // token columns one epilogue warp drains
+    static constexpr int kThreads = 32 * (kEpiWarp0 + 4 * kEpiSplit);
+    static constexpr uint32_t kQBox = uint32_t(BN) * kBoxK; // int8 activations per box
+    // Instruction descriptor: D int32, A unsigned 8-bit (stored codes), B
+    // signed 8-bit (activations), both K-major, M = 128, N = BN.
+    static constexpr uint32_t kIdesc = (2u << 4) | (0u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
+                                       (uint32_t(kBM >> 4) << 24);
+    static_assert(2 * BN <= int(kDCols), "two accumulator buffers");
+    static_assert(kEpiCols % 32 == 0, "epilogue drains 32-column chunks");
+};
 
 struct GemmParams {
     const float *w_scale;
@@ -133,12 +145,13 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 // One pipeline stage: eight MMAs (k = 0..255) issued by lane 0.
 // b_desc0 describes the stage's first 32 k of activations; the start address
 // field advances by 32 B (2 units) per MMA within a 128-k box and by one box
-// (16 KB, 1024 units) after four MMAs.  A advances 8 TMEM columns per MMA.
+// (BOX16 units of 16 B) after four MMAs.  A advances 8 TMEM columns per MMA.
 // accumulate_first = 0 makes the first MMA overwrite D (first stage of a tile).
+template <uint32_t BOX16>
 __device__ __forceinline__ void mma_stage8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc0, uint32_t idesc,
                                            uint32_t accumulate_first)
 {
-    static_assert(kBK / kMmaK == 8 && kBoxK / kMmaK == 4, "stage shape");
+    static_assert(kBK / kMmaK == 8 && kBoxK / kMmaK == 4 && kBoxK == 128 && kMmaK == 32, "stage shape");
     asm volatile(
         "{\n\t.reg .pred e, p, t;\n\t.reg .b32 r;\n\t"
         "mov.u32 r, %%laneid;\n\t"
@@ -154,7 +167,7 @@ __device__ __forceinline__ void mma_stage8(uint32_t d_tmem, uint32_t a_tmem, uin
         "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%17], %9, %11, t;\n\t"
         "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%18], %10, %11, t;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "r"(a_tmem + 8), "l"(b_desc0), "l"(b_desc0 + 2), "l"(b_desc0 + 4), "l"(b_desc0 + 6),
-        "l"(b_desc0 + 1024), "l"(b_desc0 + 1026), "l"(b_desc0 + 1028), "l"(b_desc0 + 1030), "r"(idesc),
+        "l"(b_desc0 + BOX16), "l"(b_desc0 + BOX16 + 2), "l"(b_desc0 + BOX16 + 4), "l"(b_desc0 + BOX16 + 6), "r"(idesc),
         "r"(accumulate_first), "r"(a_tmem + 16), "r"(a_tmem + 24), "r"(a_tmem + 32), "r"(a_tmem + 40),
         "r"(a_tmem + 48), "r"(a_tmem + 56), "r"(1u)
         : "memory");
@@ -227,20 +240,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr)
     return d;
 }
 
-// Instruction descriptor: D int32, A unsigned 8-bit (stored codes), B signed
-// 8-bit (activations), both K-major, M = 128, N = kBN.
-constexpr uint32_t kIdesc = (2u << 4) | (0u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) |
-                            (uint32_t(kBM >> 4) << 24);
-
 // ---------------------------------------------------------------- kernel
 
+template <int BN>
 struct Smem {
+    using C = TileCfg<BN>;
     // activation ring (1024-byte aligned for the 128-byte swizzle)
-    unsigned char q[kQStages][kBoxes][kQBox];
+    unsigned char q[kQStages][kBoxes][C::kQBox];
     unsigned char p[kQStages][kBoxes][kPBox];
     // per epilogue warp: d and row sums of the current tile's 128 tokens
-    float ep_d[4 * kEpiSplit][kEpiCols];
-    int32_t ep_r[4 * kEpiSplit][kEpiCols];
+    float ep_d[4 * C::kEpiSplit][C::kEpiCols];
+    int32_t ep_r[4 * C::kEpiSplit][C::kEpiCols];
     uint64_t full[kQStages];     // activation and packed boxes landed
     uint64_t empty[kQStages];    // the slot's bytes are no longer needed (MMAs completed)
     uint64_t afull[kAStages];    // A expanded into tensor memory (and its activations landed)
@@ -251,17 +261,24 @@ struct Smem {
     uint32_t tmem_base;
     int abort_flag;
 };
-constexpr uint32_t kSmemBytes = uint32_t(sizeof(Smem)) + 1024;  // + alignment slack
-static_assert(kSmemBytes > 116 * 1024, "one CTA per SM: its 512 tensor-memory columns are the whole SM's");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+// One CTA per SM: its 512 tensor-memory columns are the whole SM's, so the
+// dynamic shared memory asked for is kept above half of the SM's.
+template <int BN>
+constexpr uint32_t smem_bytes()
+{
+    constexpr uint32_t need = uint32_t(sizeof(Smem<BN>)) + 1024;  // + alignment slack
+    return need > 120 * 1024 ? need : 120 * 1024;
+}
+static_assert(smem_bytes<128>() <= 227 * 1024 && smem_bytes<32>() <= 227 * 1024, "shared memory per CTA");
 
 struct TileMap {
     int tiles_m;                 // token tiles
     int num_tiles;
+    int bn;                      // tokens per tile
     __device__ void coords(int t, int64_t &n0, int64_t &m0) const
     {
         n0 = int64_t(t / tiles_m) * kBM;
-        m0 = int64_t(t % tiles_m) * kBN;
+        m0 = int64_t(t % tiles_m) * bn;
     }
 };
 
@@ -305,13 +322,15 @@ __device__ __forceinline__ void epilogue_chunk_any(const uint32_t (&v)[32], cons
         epilogue_chunk<T, false, DBG>(v, sd, sr, n, m0, p, gamma);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN>
+__global__ void __launch_bounds__(TileCfg<BN>::kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap pmap,
             const GemmParams p, const TileMap tm)
 {
+    using C = TileCfg<BN>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
-    Smem &sm = *reinterpret_cast<Smem *>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
+    Smem<BN> &sm = *reinterpret_cast<Smem<BN> *>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
     volatile int *abort_flag = &sm.abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -328,7 +347,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&sm.tfull[b]), 1);
-            mbar_init(smem_u32(&sm.tempty[b]), 128 * kEpiSplit);
+            mbar_init(smem_u32(&sm.tempty[b]), 128 * C::kEpiSplit);
         }
         mbar_init(smem_u32(&sm.drain), 1);
         sm.abort_flag = 0;
@@ -342,7 +361,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t a_tmem0 = tmem + 2 * kBN;    // columns [256, 512): kAStages x 64
+    const uint32_t a_tmem0 = tmem + kDCols;     // columns [256, 512): kAStages x 64
 
     if (warp < kProducerWarps) {
         // ------------------------------------------------ TMA producers
@@ -367,7 +386,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
 #pragma unroll
                 for (int box = 0; box < kBoxes; ++box) {
                     const int k0 = kb * kBK + box * kBoxK;
-                    tma_load_2d_lane(box, smem_u32(sm.q[s][box]), &qmap, full, kQBox, k0, int32_t(m0));
+                    tma_load_2d_lane(box, smem_u32(sm.q[s][box]), &qmap, full, C::kQBox, k0, int32_t(m0));
                     tma_load_2d_lane(kBoxes + box, smem_u32(sm.p[s][box]), &pmap, full, kPBox, k0 * 2,
                                      int32_t(n0 / 8));
                 }
@@ -394,7 +413,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                 ok = false;
                 break;
             }
-            const uint32_t d_tmem = tmem + uint32_t(b * kBN);
+            const uint32_t d_tmem = tmem + uint32_t(b * BN);
             for (int kb = 0; kb < KB; ++kb, ++g) {
                 const int s = g % kQStages, a = g % kAStages;
                 // the tensor core reads the activation tile through the async
@@ -408,7 +427,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                     break;
                 }
                 tc_fence_after();
-                mma_stage8(d_tmem, a_tmem0 + a * kACols, q_desc0 + uint64_t(s) * (kBoxes * kQBox >> 4), kIdesc,
+                mma_stage8<(C::kQBox >> 4)>(d_tmem, a_tmem0 + a * kACols,
+                                            q_desc0 + uint64_t(s) * (kBoxes * C::kQBox >> 4), C::kIdesc,
                            kb > 0 ? 1u : 0u);
                 mma_commit(smem_u32(&sm.empty[s]));
                 mma_commit(smem_u32(&sm.aempty[a]));
@@ -477,7 +497,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
         // ------------------------------------------------ epilogue
         const int ew = warp - kEpiWarp0;              // this warp's staging slice
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
-        const int c0 = (ew / 4) * kEpiCols;           // first token column this warp drains
+        const int c0 = (ew / 4) * C::kEpiCols;        // first token column this warp drains
         const int rl = quarter * 32 + lane;
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
         const float gamma = p.w_scale[0];
@@ -490,7 +510,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
             tm.coords(t, n0, m0);
             __syncwarp();
 #pragma unroll
-            for (int c = 0; c < kEpiCols / 32; ++c) {
+            for (int c = 0; c < C::kEpiCols / 32; ++c) {
                 const int64_t m = m0 + c0 + c * 32 + lane;
                 sd[c * 32 + lane] = m < p.M ? __ldg(p.d + m) : 0.0f;
                 sr[c * 32 + lane] = m < p.M ? __ldg(p.rowsum + m) : 0;
@@ -502,9 +522,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
             tc_fence_after();
             const int64_t n = n0 + rl;
 #pragma unroll 1
-            for (int c = 0; c < kEpiCols / 32; ++c) {
+            for (int c = 0; c < C::kEpiCols / 32; ++c) {
                 uint32_t v[32];
-                tmem_ld32_wait(tmem + lane_addr + uint32_t(b * kBN + c0 + c * 32), v);
+                tmem_ld32_wait(tmem + lane_addr + uint32_t(b * BN + c0 + c * 32), v);
                 if (n < p.N) {
                     const int64_t mc = m0 + c0 + c * 32;
                     const float *d32 = sd + c * 32;
@@ -576,16 +596,15 @@ int make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t out
 
 size_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
 
-int launch_gemm(const GemvArgs &a, void *, size_t, cudaStream_t s)
+namespace {
+
+template <int BN>
+int launch_tiles(const GemvArgs &a, const DeviceInfo *di, cudaStream_t s)
 {
-    const DeviceInfo *di = device_info();
-    if (!di)
-        return BL_ERR_CUDA;
-    if (a.M > (int64_t(1) << 30) || a.N > (int64_t(1) << 30))
-        return BL_ERR_SHAPE;
+    using C = TileCfg<BN>;
     CUtensorMap qmap, pmap;
-    // activations: [M][K] int8, boxes of 128 k x 128 tokens, 128-byte swizzle
-    int st = make_map_2d(&qmap, a.q, uint64_t(a.K), uint64_t(a.M), uint64_t(a.K), kBoxK, kBN, true);
+    // activations: [M][K] int8, boxes of 128 k x BN tokens, 128-byte swizzle
+    int st = make_map_2d(&qmap, a.q, uint64_t(a.K), uint64_t(a.M), uint64_t(a.K), kBoxK, BN, true);
     if (st)
         return st;
     // packed weights as [row groups][K/64 * 128 B]: boxes of 16 groups x 256 B (128 k)
@@ -595,20 +614,34 @@ int launch_gemm(const GemvArgs &a, void *, size_t, cudaStream_t s)
     if (st)
         return st;
     int per_sm = 0;
-    if ((st = occupancy(reinterpret_cast<const void *>(gemm_kernel), kThreads, kSmemBytes, &per_sm)))
+    if ((st = occupancy(reinterpret_cast<const void *>(gemm_kernel<BN>), C::kThreads, smem_bytes<BN>(), &per_sm)))
         return st;
     if (per_sm < 1)
         return BL_ERR_UNSUPPORTED;
     GemmParams p{a.w_scale, a.d, a.rowsum, a.M, a.N, a.K, a.y, a.yt, a.ldy, a.acc_dbg, di->status};
     TileMap tm;
-    tm.tiles_m = int((a.M + kBN - 1) / kBN);
+    tm.tiles_m = int((a.M + BN - 1) / BN);
+    tm.bn = BN;
     const int64_t tiles = int64_t(tm.tiles_m) * ((a.N + kBM - 1) / kBM);
     if (tiles > (int64_t(1) << 30))
         return BL_ERR_SHAPE;
     tm.num_tiles = int(tiles);
     const int grid = int(std::min<int64_t>(tiles, di->sm_count));
-    gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(qmap, pmap, p, tm);
+    gemm_kernel<BN><<<grid, C::kThreads, smem_bytes<BN>(), s>>>(qmap, pmap, p, tm);
     return launch_status();
+}
+
+}  // namespace
+
+int launch_gemm(const GemvArgs &a, void *, size_t, cudaStream_t s)
+{
+    const DeviceInfo *di = device_info();
+    if (!di)
+        return BL_ERR_CUDA;
+    if (a.M > (int64_t(1) << 30) || a.N > (int64_t(1) << 30))
+        return BL_ERR_SHAPE;
+    // small batches: 32-token tiles (a 128-token tile would be mostly padding)
+    return a.M <= 32 ? launch_tiles<32>(a, di, s) : launch_tiles<128>(a, di, s);
 }
 
 }  // namespace bl

@@ -160,7 +160,9 @@ int bitlinear_quantize_act(const void *x, int xt, int64_t M, int64_t K,
  *   q, d, rowsum      from bitlinear_quantize_act (device), q is [M][K]
  *   y                 device, [M][ldy] of dtype yt (BL_F32 or BL_BF16), ldy >= N
  *   acc_dbg           NULL, or device [M][N] int32 receiving acc (before rescale)
- * M * K must not exceed 163840 (the activations are staged on chip).
+ * M * K must not exceed 163840 (the activations are staged on chip).  From
+ * M = 8 on the product runs on the tensor-core path of bitlinear_gemm (dp4a
+ * work grows with M); results are identical either way.
  */
 int bitlinear_gemv(const uint8_t *packed, const float *w_scale, int64_t N,
                    int64_t K, const int8_t *q, const float *d,

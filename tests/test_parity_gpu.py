@@ -167,6 +167,26 @@ def test_gemv_ragged_and_edge(bl, N, K, M, fused):
     _check_gemv(bl, W, x, torch.bfloat16, fused)
 
 
+@pytest.mark.parametrize("M", [8, 16])
+def test_small_batch_tensor_core_path(bl, M):
+    """From 8 tokens on, bitlinear_gemv and linear() run the tcgen05 path:
+    the four 2.4B shapes x 10 seeds, integers bit-exact, outputs equal."""
+    for K, N in si.DECODE_SHAPES_2B:
+        for seed in range(10):
+            W = si.weight(N, K, seed=2000 + seed)
+            g, codes, _ = oracle_weight(W)
+            w = _pack_gpu(bl, W)
+            x = si.activations(M, K, seed=seed * 17 + M)
+            y_o, acc_o = _oracle_gemv(g, codes, x)
+            xd = x.to(dev())
+            q, d, r = bl.quantize_act(xd)
+            acc = torch.empty(M, N, dtype=torch.int32, device=dev())
+            y = bl.gemv(w, q, d, r, acc_dbg=acc)
+            np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+            compare_outputs(y, y_o)
+            compare_outputs(bl.linear(w, xd), y_o)
+
+
 def test_gemv_fp32_input_and_strided_output(bl):
     N, K, M = 300, 256, 4
     W, x = seeded_problem(N, K, M, seed=11, xdtype=torch.float32)
