@@ -287,10 +287,12 @@ def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda"):
         q = torch.empty(M, K, dtype=torch.int8, device=device)
         d = torch.empty(M, dtype=torch.float32, device=device)
         r = torch.empty(M, dtype=torch.int32, device=device)
+        # split-K workspace: zero once, left zero by every call
+        gws = torch.zeros(max(bl.gemm_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=device)
 
         def call(wt):
             bl.quantize_act(x, out=(q, d, r))
-            bl.gemm(wt, q, d, r, out=y)
+            bl.gemm(wt, q, d, r, out=y, workspace=gws)
     for i in range(min(copies, 8)):
         call(ws[i])
     torch.cuda.synchronize()
@@ -309,7 +311,7 @@ def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda"):
     del g, ws
     return {"K": K, "N": N, "M": M, "us": t * 1e6, "GBps": nbytes / t / 1e9,
             "weight_copies": copies,
-            "path": "fused dp4a GEMV" if fused else "quantise + tcgen05 GEMM (32-token tiles)"}
+            "path": "fused dp4a GEMV" if fused else "quantise + tcgen05 GEMM (32-token tiles, split K)"}
 
 
 def isolated_binary(bl, K, N, iters=100, device="cuda"):

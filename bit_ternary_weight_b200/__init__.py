@@ -262,7 +262,8 @@ def gemm(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc
     out = _out(M, w.N, out_dtype, q.device, out)
     need = gemm_workspace_bytes(M, w.N, w.K)
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        # zero before its first use; every call leaves it zero again
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.bitlinear_gemm(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q), _ptr(d),
                                _ptr(rowsum), M, _ptr(out), _dt(out.dtype), out.stride(0),

@@ -110,6 +110,10 @@ struct GemmParams {
     int64_t ldy;
     int32_t *acc_dbg;
     int *status;
+    // split-K (tm.splits > 1): int32 partial sums and arrival counters, zero
+    // on entry and left zero
+    int32_t *ws;
+    int *counters;
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -271,14 +275,22 @@ constexpr uint32_t smem_bytes()
 }
 static_assert(smem_bytes<128>() <= 227 * 1024 && smem_bytes<32>() <= 227 * 1024, "shared memory per CTA");
 
+// Work units: output tile t = u / splits, k blocks [kb0, kb1) of split u % splits.
 struct TileMap {
     int tiles_m;                 // token tiles
     int num_tiles;
     int bn;                      // tokens per tile
-    __device__ void coords(int t, int64_t &n0, int64_t &m0) const
+    int splits;                  // k splits per tile (1: the whole K)
+    int kb_total;                // k blocks of the whole K
+    int num_units;               // num_tiles * splits
+    __device__ void unit(int u, int &t, int64_t &n0, int64_t &m0, int &kb0, int &kb1) const
     {
+        t = u / splits;
+        const int sp = u - t * splits;
         n0 = int64_t(t / tiles_m) * kBM;
         m0 = int64_t(t % tiles_m) * bn;
+        kb0 = int(int64_t(sp) * kb_total / splits);
+        kb1 = int(int64_t(sp + 1) * kb_total / splits);
     }
 };
 
@@ -334,7 +346,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
     volatile int *abort_flag = &sm.abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int KB = int((p.K + kBK - 1) / kBK);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kQStages; ++s) {
@@ -368,14 +379,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
         // lanes 0..kBoxes-1 copy the activation boxes of a stage, the next
         // kBoxes lanes its packed weight boxes; the warp waits as a whole
         int last = -1;   // global stage index of this warp's last issued stage
-        int base = 0;    // global stage index of the current tile's first k block
+        int base = 0;    // global stage index of the current unit's first k block
         bool ok = true;
-        for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, base += KB) {
+        for (int u = blockIdx.x; u < tm.num_units && ok; u += gridDim.x) {
+            int t, kb0, kb1;
             int64_t n0, m0;
-            tm.coords(t, n0, m0);
-            for (int kb = ((warp - base) % kProducerWarps + kProducerWarps) % kProducerWarps; kb < KB;
-                 kb += kProducerWarps) {
-                const int g = base + kb;
+            tm.unit(u, t, n0, m0, kb0, kb1);
+            const int nk = kb1 - kb0;
+            for (int i = ((warp - base) % kProducerWarps + kProducerWarps) % kProducerWarps; i < nk;
+                 i += kProducerWarps) {
+                const int g = base + i, kb = kb0 + i;
                 const int s = g % kQStages;
                 const uint32_t full = smem_u32(&sm.full[s]);
                 if (!__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.empty[s]), (uint32_t(g / kQStages) & 1u) ^ 1u,
@@ -392,6 +405,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                 }
                 last = g;
             }
+            base += nk;
         }
         if (last >= 0) {
             // the last stage's copies have landed before the CTA exits (at
@@ -402,10 +416,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer (whole warp, lane 0 issues)
-        const uint64_t q_desc0 = smem_desc_sw128(smem_u32(sm.q[0][0]));   // slot s adds s * 40 KB >> 4
+        const uint64_t q_desc0 = smem_desc_sw128(smem_u32(sm.q[0][0]));   // slot s adds its offset >> 4
         int g = 0, it = 0;
         bool ok = true, issued_any = false;
-        for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x, ++it) {
+        for (int u = blockIdx.x; u < tm.num_units && ok; u += gridDim.x, ++it) {
+            int t, kb0, kb1;
+            int64_t n0, m0;
+            tm.unit(u, t, n0, m0, kb0, kb1);
             const int b = it & 1;
             if (it >= 2 &&
                 !__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.tempty[b]), (uint32_t(it >> 1) & 1u) ^ 1u,
@@ -414,7 +431,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                 break;
             }
             const uint32_t d_tmem = tmem + uint32_t(b * BN);
-            for (int kb = 0; kb < KB; ++kb, ++g) {
+            for (int kb = kb0; kb < kb1; ++kb, ++g) {
                 const int s = g % kQStages, a = g % kAStages;
                 // the tensor core reads the activation tile through the async
                 // proxy: wait on the barrier its TMA completes, not only on the
@@ -429,7 +446,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                 tc_fence_after();
                 mma_stage8<(C::kQBox >> 4)>(d_tmem, a_tmem0 + a * kACols,
                                             q_desc0 + uint64_t(s) * (kBoxes * C::kQBox >> 4), C::kIdesc,
-                           kb > 0 ? 1u : 0u);
+                           kb > kb0 ? 1u : 0u);
                 mma_commit(smem_u32(&sm.empty[s]));
                 mma_commit(smem_u32(&sm.aempty[a]));
                 issued_any = true;
@@ -452,8 +469,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
         const uint32_t lane_addr = uint32_t(quarter * 32) << 16;
         int g = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < tm.num_tiles && ok; t += gridDim.x) {
-            for (int kb = 0; kb < KB; ++kb, ++g) {
+        for (int u = blockIdx.x; u < tm.num_units && ok; u += gridDim.x) {
+            int t, kb0, kb1;
+            int64_t n0, m0;
+            tm.unit(u, t, n0, m0, kb0, kb1);
+            for (int kb = kb0; kb < kb1; ++kb, ++g) {
                 if ((g & 1) != grp)
                     continue;
                 const int s = g % kQStages, a = g % kAStages;
@@ -504,10 +524,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
         float *sd = sm.ep_d[ew];
         int32_t *sr = sm.ep_r[ew];
         int it = 0;
-        for (int t = blockIdx.x; t < tm.num_tiles; t += gridDim.x, ++it) {
+        for (int u = blockIdx.x; u < tm.num_units; u += gridDim.x, ++it) {
             const int b = it & 1;
+            int t, kb0, kb1;
             int64_t n0, m0;
-            tm.coords(t, n0, m0);
+            tm.unit(u, t, n0, m0, kb0, kb1);
             __syncwarp();
 #pragma unroll
             for (int c = 0; c < C::kEpiCols / 32; ++c) {
@@ -521,10 +542,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                 break;
             tc_fence_after();
             const int64_t n = n0 + rl;
-#pragma unroll 1
-            for (int c = 0; c < C::kEpiCols / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32_wait(tmem + lane_addr + uint32_t(b * BN + c0 + c * 32), v);
+            auto finish = [&](const uint32_t (&v)[32], int c) {
                 if (n < p.N) {
                     const int64_t mc = m0 + c0 + c * 32;
                     const float *d32 = sd + c * 32;
@@ -541,9 +559,56 @@ gemm_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CU
                             epilogue_chunk_any<float, false>(v, d32, r32, n, mc, p, gamma);
                     }
                 }
+            };
+            if (tm.splits == 1) {
+#pragma unroll 1
+                for (int c = 0; c < C::kEpiCols / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32_wait(tmem + lane_addr + uint32_t(b * BN + c0 + c * 32), v);
+                    finish(v, c);
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&sm.tempty[b]));
+            } else {
+                // split-K: add this warp's partial sums (32 weight rows x its
+                // token columns) into the workspace, laid out [tile][token][row]
+                // so that a warp's adds for one token cover 128 contiguous bytes
+                int32_t *wsw = p.ws + (int64_t(t) * BN + c0) * kBM + rl;
+#pragma unroll 1
+                for (int c = 0; c < C::kEpiCols / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32_wait(tmem + lane_addr + uint32_t(b * BN + c0 + c * 32), v);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        atomicAdd(wsw + int64_t(c * 32 + j) * kBM, int(v[j]));
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&sm.tempty[b]));
+                // the warp of the last split to arrive finishes the tile's block
+                __threadfence();
+                __syncwarp();
+                int *cnt = p.counters + int64_t(t) * (4 * C::kEpiSplit) + ew;
+                int old = 0;
+                if (lane == 0)
+                    old = atomicAdd(cnt, 1);
+                old = __shfl_sync(0xffffffffu, old, 0);
+                if (old == tm.splits - 1) {
+                    __threadfence();
+#pragma unroll 1
+                    for (int c = 0; c < C::kEpiCols / 32; ++c) {
+                        uint32_t v[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            int32_t *w = wsw + int64_t(c * 32 + j) * kBM;
+                            v[j] = uint32_t(__ldcg(w));
+                            __stcg(w, 0);   // left zero for the next call
+                        }
+                        finish(v, c);
+                    }
+                    if (lane == 0)
+                        *cnt = 0;
+                }
             }
-            tc_fence_before();
-            mbar_arrive(smem_u32(&sm.tempty[b]));
         }
     }
 
@@ -594,12 +659,49 @@ int make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t out
 
 }  // namespace
 
-size_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+namespace {
+
+// Split-K plan: only small batches (32-token tiles) split K, and only while
+// their output tiles alone would leave SMs idle.  Workspace: int32 partial
+// sums [tile][32 tokens][128 rows], then one arrival counter per tile and
+// epilogue warp.
+struct SplitPlan {
+    int splits = 1;
+    size_t counters_offset = 0;
+    size_t bytes = 0;
+};
+
+SplitPlan split_plan(int64_t M, int64_t N, int64_t K, int sms)
+{
+    SplitPlan sp;
+    if (M > 32)
+        return sp;
+    const int64_t tiles = ((M + 31) / 32) * ((N + kBM - 1) / kBM);
+    const int64_t kb = (K + kBK - 1) / kBK;
+    if (tiles >= sms || kb < 2)
+        return sp;
+    // all units in one wave: a CTA that takes two units doubles the latency
+    const int64_t splits = std::min<int64_t>(sms / tiles, kb);
+    if (splits < 2)
+        return sp;
+    sp.splits = int(splits);
+    sp.counters_offset = size_t(tiles) * 32 * kBM * sizeof(int32_t);
+    sp.bytes = sp.counters_offset + size_t(tiles) * 4 * TileCfg<32>::kEpiSplit * sizeof(int);
+    return sp;
+}
+
+}  // namespace
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    const DeviceInfo *di = device_info();
+    return di ? split_plan(M, N, K, di->sm_count).bytes : 0;
+}
 
 namespace {
 
 template <int BN>
-int launch_tiles(const GemvArgs &a, const DeviceInfo *di, cudaStream_t s)
+int launch_tiles(const GemvArgs &a, const DeviceInfo *di, const SplitPlan &sp, void *ws, cudaStream_t s)
 {
     using C = TileCfg<BN>;
     CUtensorMap qmap, pmap;
@@ -618,30 +720,39 @@ int launch_tiles(const GemvArgs &a, const DeviceInfo *di, cudaStream_t s)
         return st;
     if (per_sm < 1)
         return BL_ERR_UNSUPPORTED;
-    GemmParams p{a.w_scale, a.d, a.rowsum, a.M, a.N, a.K, a.y, a.yt, a.ldy, a.acc_dbg, di->status};
+    GemmParams p{a.w_scale, a.d, a.rowsum, a.M, a.N, a.K, a.y, a.yt, a.ldy, a.acc_dbg, di->status,
+                 static_cast<int32_t *>(ws),
+                 ws ? reinterpret_cast<int *>(static_cast<char *>(ws) + sp.counters_offset) : nullptr};
     TileMap tm;
     tm.tiles_m = int((a.M + BN - 1) / BN);
     tm.bn = BN;
     const int64_t tiles = int64_t(tm.tiles_m) * ((a.N + kBM - 1) / kBM);
-    if (tiles > (int64_t(1) << 30))
+    if (tiles * sp.splits > (int64_t(1) << 30))
         return BL_ERR_SHAPE;
     tm.num_tiles = int(tiles);
-    const int grid = int(std::min<int64_t>(tiles, di->sm_count));
+    tm.splits = ws ? sp.splits : 1;
+    tm.kb_total = int((a.K + kBK - 1) / kBK);
+    tm.num_units = tm.num_tiles * tm.splits;
+    const int grid = int(std::min<int64_t>(tm.num_units, di->sm_count));
     gemm_kernel<BN><<<grid, C::kThreads, smem_bytes<BN>(), s>>>(qmap, pmap, p, tm);
     return launch_status();
 }
 
 }  // namespace
 
-int launch_gemm(const GemvArgs &a, void *, size_t, cudaStream_t s)
+int launch_gemm(const GemvArgs &a, void *ws, size_t ws_bytes, cudaStream_t s)
 {
     const DeviceInfo *di = device_info();
     if (!di)
         return BL_ERR_CUDA;
     if (a.M > (int64_t(1) << 30) || a.N > (int64_t(1) << 30))
         return BL_ERR_SHAPE;
+    // split K only with the workspace it needs (callers without one, such as
+    // bitlinear_gemv's small batches, run unsplit)
+    const SplitPlan sp = split_plan(a.M, a.N, a.K, di->sm_count);
+    void *w = sp.splits > 1 && ws && ws_bytes >= sp.bytes ? ws : nullptr;
     // small batches: 32-token tiles (a 128-token tile would be mostly padding)
-    return a.M <= 32 ? launch_tiles<32>(a, di, s) : launch_tiles<128>(a, di, s);
+    return a.M <= 32 ? launch_tiles<32>(a, di, sp, w, s) : launch_tiles<128>(a, di, sp, nullptr, s);
 }
 
 }  // namespace bl

@@ -215,7 +215,12 @@ int bitlinear_gemv_fused_multi(int count, const uint8_t *const *packed,
                                const int64_t *ldy, int32_t *const *acc_dbg,
                                unsigned flags, void *stream);
 
-/* Bytes of workspace bitlinear_gemm needs for this problem (0 if none). */
+/*
+ * Bytes of workspace bitlinear_gemm needs for this problem (0 if none).
+ * Nonzero for small batches (M <= 32) whose output tiles alone would leave
+ * SMs idle: K is then split across CTAs and the int32 partial sums meet in
+ * the workspace.
+ */
 size_t bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -225,7 +230,10 @@ size_t bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * "BitCompute", section "Future Roadmap" (tensor-core execution of the
  * ternary product).  Arguments as for bitlinear_gemv, plus
  *   ws, ws_bytes   device workspace, at least bitlinear_gemm_workspace_bytes
- *                  (may be NULL when that is 0).
+ *                  (may be NULL when that is 0).  It must be all zero before
+ *                  its first use, and every call leaves it zero; it may be
+ *                  reused by calls that are ordered on one stream, not shared
+ *                  by calls that can run at the same time.
  * q must be 16-byte aligned and K % 64 == 0.
  */
 int bitlinear_gemm(const uint8_t *packed, const float *w_scale, int64_t N,

@@ -289,6 +289,33 @@ def test_gemm_several_tiles_per_cta(bl, M, N, K):
     _check_gemm(bl, N, K, M, seed=M ^ N ^ K)
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 6912, 2560), (8, 6912, 2560), (16, 2560, 6912),
+                                   (32, 2560, 6912), (3, 300, 320), (17, 1000, 1280)])
+def test_gemm_split_k_small_batches(bl, M, N, K):
+    """Small batches split K across CTAs and meet in the int32 workspace:
+    bit-exact, the workspace is left zero, and a second call reusing it is
+    exact too."""
+    need = bl.gemm_workspace_bytes(M, N, K)
+    assert need > 0
+    W = si.weight(N, K, seed=M * 13 + N)
+    x = si.activations(M, K, seed=M + K)
+    g, codes, _ = oracle_weight(W)
+    w = _pack_gpu(bl, W)
+    q, d, r = bl.quantize_act(x.to(dev()))
+    q_o, d_o, r_o = oracle.quantize_act(x.float().numpy())
+    acc_o = oracle.ternary_acc(codes, q_o)
+    y_o = oracle.rescale(acc_o, d_o, g)
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev())
+    for _ in range(2):
+        acc = torch.full((M, N), 7, dtype=torch.int32, device=dev())
+        y = bl.gemm(w, q, d, r, acc_dbg=acc, workspace=ws)
+        torch.cuda.synchronize()
+        assert bl.last_device_status() == 0
+        np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+        compare_outputs(y, y_o)
+        assert int(torch.count_nonzero(ws)) == 0
+
+
 @pytest.mark.parametrize("K,N", si.PREFILL_SHAPES)
 @pytest.mark.parametrize("M", si.PREFILL_TOKENS)
 def test_gemm_prefill_full_size(bl, K, N, M):
