@@ -589,7 +589,7 @@ def run_case(args):
             fn = lambda: bl.gemv_fused(w, x)  # noqa: E731
         else:
             q, d, r = bl.quantize_act(x)
-            ws = torch.empty(max(bl.gemm_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
+            ws = torch.zeros(max(bl.gemm_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
             fn = lambda: bl.gemm(w, q, d, r, workspace=ws)  # noqa: E731
         nbytes, ops = bl.packed_bytes(N, K), 2 * M * N * K
     del W

@@ -622,8 +622,17 @@ int dispatch_m(const Params &p, unsigned flags, cudaStream_t s)
 
 }  // namespace
 
+int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s);
+bool gemv_stream_applies(const GemvBatch &b, int sm_count);
+
 int launch_gemv_batch(const GemvBatch &b, bool fused, cudaStream_t s)
 {
+    const DeviceInfo *di = device_info();
+    if (!di)
+        return BL_ERR_CUDA;
+    // one token on a large layer: the producer/consumer streaming kernel
+    if (gemv_stream_applies(b, di->sm_count))
+        return launch_gemv_stream(b, fused, s);
     Params p{};
     p.count = b.count;
     p.gstart[0] = 0;

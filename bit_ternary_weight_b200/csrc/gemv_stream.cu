@@ -1,0 +1,581 @@
+// gemv_stream.cu -- ternary decode GEMV for one token on large layers
+// (K a multiple of 4096, thousands of output rows).
+//
+// "How to Run BitNet Inference on GPU Using CUDA Kernels: A Complete Guide",
+// section "Understanding the Two-Phase Architecture": decode is a
+// memory-bound INT8-activation x INT2-weight product, so the weight stream
+// N*K/4 bytes is the whole cost and every instruction spent per weight byte
+// beyond the dot product itself lowers the bandwidth an SM can sustain.
+//
+// Design (B200, persistent CTAs):
+//   * A CTA is KC consumer warps plus one producer warp.  Up to K = 8192 it
+//     has KC = 8 and two CTAs share an SM, so that a CTA of the next launch
+//     (programmatic dependent launch) can start streaming beside one of this
+//     launch; for larger K it has KC = 16 and owns the SM, which halves the
+//     per-SM cost of quantising the activations.
+//   * Each CTA owns a contiguous range of 8-row groups (whose packed slabs,
+//     2*K bytes each, are contiguous in the tile layout).  It takes them in
+//     sets of at most R groups, sized evenly, with R (4..8) chosen per launch
+//     so that every CTA has the same number of sets; a set is streamed in
+//     K / (256 KC) stages, a stage holding the same 256*KC-k range of each of
+//     the set's groups (512*KC bytes per group).
+//   * The producer warp fills a four-stage ring with bulk asynchronous
+//     copies (one copy per group, each from a different lane, since the
+//     copies of one thread complete one after another), completion counted
+//     on the stage's mbarrier.
+//   * Consumer warp w always takes 512-byte piece w of each group in a stage
+//     (lane l: row l%8, 64 k), so the activations it needs, 64 bytes per
+//     lane, are loaded once per stage and used for all of the stage's groups
+//     (whose loads are issued together, by a body specialised on the group
+//     count).  Multiply with the stored codes s = code + 1: (word &
+//     0x03030303), (word & 0x0c0c0c0c), ... hold s, 4s, 16s, 64s per byte;
+//     one LOP3 and one dp4a per four weights into four accumulators per
+//     group, folded with shifts when the group's last stage is done;
+//     sum(code q) = sum(s q) - rowsum(q).
+//   * The ring is filled from the start; the consumers wait on the preceding
+//     launch only before they read the activations, which they quantise (or
+//     copy) into shared memory.
+//   * Every mbarrier wait is bounded; on expiry the CTA records
+//     BL_ERR_TIMEOUT, the consumers stop and the producer waits (bounded) for
+//     its copies in flight before the CTA exits.
+#include "bl_common.cuh"
+
+namespace bl {
+
+int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s);
+bool gemv_stream_applies(const GemvBatch &b, int sm_count);
+
+namespace {
+
+constexpr int kMaxConsumers = 16;
+constexpr int kStages = 4;                           // ring stages
+constexpr int kMaxSet = 8;                           // groups per set (stage), at most
+constexpr int kMaxGroupsPerCta = 64;
+constexpr int kSmallK = 8192;                        // up to here: KC = 8, two CTAs per SM
+
+// Geometry of a CTA with KC consumer warps.
+template <int KC>
+struct Geo {
+    static constexpr int kConsumerThreads = 32 * KC;
+    static constexpr int kThreads = kConsumerThreads + 32;   // + the producer warp
+    static constexpr int kStageK = 256 * KC;                 // k of one group per stage
+    static constexpr int kSlotBytes = 2 * kStageK;           // its packed bytes (8 rows x 2 bits)
+    static constexpr int kCtasPerSm = KC == 8 ? 2 : 1;
+};
+
+enum { SMODE_Q = 0, SMODE_X_BF16 = 1, SMODE_X_F32 = 2 };
+
+struct StreamParams {
+    const uint8_t *packed;
+    const float *w_scale;
+    int64_t N;
+    void *y;
+    int32_t *acc_dbg;
+    int64_t K;
+    const int8_t *q;
+    const float *d;
+    const int32_t *rowsum;
+    const void *x;
+    int yt;
+    // CTA b owns row groups [b*gpc_base + min(b, gpc_rem), ...), gpc_base (+1) of them
+    int64_t gpc_base;
+    int gpc_rem;
+    int set_cap;         // R: groups a stage holds at most (4 .. kMaxSet)
+    int *status;
+};
+
+struct StreamSmem {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    int abort_flag;
+    alignas(16) float bmax[kMaxConsumers];   // read back as float4
+    int bsum[kMaxConsumers];
+    float d;
+    int r;
+    int sacc[kMaxGroupsPerCta][8];
+    // followed by the ring (kStages x set_cap slots) and the int8 activations (K bytes)
+};
+
+constexpr size_t kHeader = (sizeof(StreamSmem) + 127) / 128 * 128;
+static_assert(offsetof(StreamSmem, bmax) % 16 == 0, "bmax is read as float4");
+
+// The CTA's ng groups in the fewest sets of at most R groups, sized evenly
+// (base or base + 1 groups; the first `extra` sets take one more).
+struct SetSplit {
+    int nsets, base, extra;
+    __device__ __forceinline__ SetSplit(int ng, int R)
+    {
+        nsets = (ng + R - 1) / R;
+        base = ng / nsets;
+        extra = ng - base * nsets;
+    }
+    __device__ __forceinline__ int size(int i) const { return base + (i < extra ? 1 : 0); }
+};
+
+__device__ __forceinline__ uint4 lds128(uint32_t saddr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(saddr));
+    return v;
+}
+
+template <int KC>
+__device__ __forceinline__ void consumers_sync() { named_barrier(1, Geo<KC>::kConsumerThreads); }
+
+// Four int32 values, each already within [-128, 127], as one little-endian
+// word of int8 (q0 in the low byte); the saturating pack equals the clamp.
+__device__ __forceinline__ uint32_t pack4_s8(int q0, int q1, int q2, int q3)
+{
+    uint32_t hi, d;
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(q3), "r"(q2));
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(q1), "r"(q0), "r"(hi));
+    return d;
+}
+
+// rint(x * s) for eight values (fp32 product, ties to even), packed as int8;
+// the sum of the eight added to *sum.
+__device__ __forceinline__ uint2 quant8(const float (&f)[8], float s, int &sum)
+{
+    int t[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        t[j] = __float2int_rn(__fmul_rn(f[j], s));
+    const uint32_t lo = pack4_s8(t[0], t[1], t[2], t[3]);
+    const uint32_t hi = pack4_s8(t[4], t[5], t[6], t[7]);
+    sum = dp4a_us(0x01010101u, lo, sum);
+    sum = dp4a_us(0x01010101u, hi, sum);
+    return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ void bf16x8_f32(const uint4 v, float (&f)[8])
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// Block-wide absmax of the consumer threads' maxima, then the scale
+// s = 127 / max(amax, eps); d = max(amax, eps) / 127 goes to sm.d.
+template <int KC>
+__device__ __forceinline__ float stream_scale(StreamSmem &sm, float amax)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // maxima are >= 0 and finite (fmaxf from 0 drops NaN): their bit
+    // patterns order like the values
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+    if (lane == 0)
+        sm.bmax[warp] = __uint_as_float(wmax);
+    consumers_sync<KC>();
+    float a = 0.0f;
+#pragma unroll
+    for (int w = 0; w < KC; w += 4) {
+        const float4 b4 = *reinterpret_cast<const float4 *>(&sm.bmax[w]);
+        a = fmaxf(fmaxf(a, b4.x), fmaxf(b4.y, fmaxf(b4.z, b4.w)));
+    }
+    const float a_eff = fmaxf(a, kEps);
+    if (tid == 0)
+        sm.d = __fdiv_rn(a_eff, kQb);
+    return __fdiv_rn(kQb, a_eff);
+}
+
+// Quantise the token x (K bf16 values) into qs: absmax, s = 127 / max(amax,
+// eps), q = clamp(rint(x * s)); each warp's partial row sum goes to bsum.
+// x stays in registers as raw bf16, CH 16-byte chunks per thread.
+template <int KC, int CH>
+__device__ __forceinline__ void stream_quantize_bf16(const StreamParams &p, StreamSmem &sm, int8_t *qs)
+{
+    constexpr int T = Geo<KC>::kConsumerThreads;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int chunks = int(p.K / 8);
+    uint4 raw[CH];
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+        const int c = tid + i * T;
+        raw[i] = c < chunks ? ld_ro_v4(static_cast<const __nv_bfloat16 *>(p.x) + int64_t(c) * 8)
+                            : make_uint4(0, 0, 0, 0);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+        float f[8];
+        bf16x8_f32(raw[i], f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            amax = fmaxf(amax, fabsf(f[j]));
+    }
+    const float s = stream_scale<KC>(sm, amax);
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+        const int c = tid + i * T;
+        if (c < chunks) {
+            float f[8];
+            bf16x8_f32(raw[i], f);
+            *reinterpret_cast<uint2 *>(qs + int64_t(c) * 8) = quant8(f, s, sum);
+        }
+    }
+    sum = __reduce_add_sync(0xffffffffu, sum);
+    if (lane == 0)
+        sm.bsum[warp] = sum;
+}
+
+// The same for any K and either input type: one pass for the absmax, a
+// second one that reads x again (from L2) to quantise.
+template <int KC, int XT>
+__device__ __forceinline__ void stream_quantize_2pass(const StreamParams &p, StreamSmem &sm, int8_t *qs)
+{
+    constexpr int T = Geo<KC>::kConsumerThreads;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int chunks = int(p.K / 8);
+    float amax = 0.0f;
+#pragma unroll 4
+    for (int c = tid; c < chunks; c += T) {
+        float f[8];
+        load8<XT>(p.x, int64_t(c) * 8, f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            amax = fmaxf(amax, fabsf(f[j]));
+    }
+    const float s = stream_scale<KC>(sm, amax);
+    int sum = 0;
+#pragma unroll 4
+    for (int c = tid; c < chunks; c += T) {
+        float f[8];
+        load8<XT>(p.x, int64_t(c) * 8, f);
+        *reinterpret_cast<uint2 *>(qs + int64_t(c) * 8) = quant8(f, s, sum);
+    }
+    sum = __reduce_add_sync(0xffffffffu, sum);
+    if (lane == 0)
+        sm.bsum[warp] = sum;
+}
+
+// Pre-quantised activations: copy q into shared memory, take d and the row sum.
+template <int KC>
+__device__ __forceinline__ void stream_copy_q(const StreamParams &p, StreamSmem &sm, int8_t *qs)
+{
+    const int tid = threadIdx.x;
+    const int vecs = int(p.K / 16);
+    for (int i = tid; i < vecs; i += Geo<KC>::kConsumerThreads)
+        reinterpret_cast<uint4 *>(qs)[i] = ld_ro_v4(p.q + int64_t(i) * 16);
+    if (tid == 0)
+        sm.d = p.d[0];
+    if (tid < KC)
+        sm.bsum[tid] = tid == 0 ? p.rowsum[0] : 0;
+}
+
+// One 16-byte piece of stored codes (64 k of one row) against the 64
+// activations q[0..3] into four accumulators (s, 4s, 16s, 64s weighted).
+__device__ __forceinline__ void mac4(const uint4 wv, const uint4 (&q)[4], int (&acc)[4])
+{
+    const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        acc[0] = dp4a_us(wd[w] & 0x03030303u, q[w].x, acc[0]);
+        acc[1] = dp4a_us(wd[w] & 0x0c0c0c0cu, q[w].y, acc[1]);
+        acc[2] = dp4a_us(wd[w] & 0x30303030u, q[w].z, acc[2]);
+        acc[3] = dp4a_us(wd[w] & 0xc0c0c0c0u, q[w].w, acc[3]);
+    }
+}
+
+// One stage of RG groups for this lane: the RG slots are consecutive, so the
+// loads take immediate offsets and are all issued before the arithmetic.
+template <int SLOT, int RG>
+__device__ __forceinline__ void stage_mac(uint32_t base, const uint4 (&q)[4], int (&acc)[kMaxSet][4])
+{
+    uint4 wv[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r)
+        wv[r] = lds128(base + r * SLOT);
+#pragma unroll
+    for (int r = 0; r < RG; ++r)
+        mac4(wv[r], q, acc[r]);
+}
+
+template <int SLOT>
+__device__ __forceinline__ void stage_mac_n(int rg, uint32_t base, const uint4 (&q)[4], int (&acc)[kMaxSet][4])
+{
+    switch (rg) {
+    case 1: stage_mac<SLOT, 1>(base, q, acc); break;
+    case 2: stage_mac<SLOT, 2>(base, q, acc); break;
+    case 3: stage_mac<SLOT, 3>(base, q, acc); break;
+    case 4: stage_mac<SLOT, 4>(base, q, acc); break;
+    case 5: stage_mac<SLOT, 5>(base, q, acc); break;
+    case 6: stage_mac<SLOT, 6>(base, q, acc); break;
+    case 7: stage_mac<SLOT, 7>(base, q, acc); break;
+    default: stage_mac<SLOT, 8>(base, q, acc); break;
+    }
+}
+static_assert(kMaxSet == 8, "stage_mac_n covers 1..8 groups");
+
+// Ring protocol.  Stage t (set i, k-range kb) occupies ring slot
+// t % kStages, room for R groups, of which it fills |set i|; full[slot]
+// counts its bytes, empty[slot] the KC consumer warps that have read it
+// (phase parity (t / kStages) & 1, kept as a running bit).
+template <int KC, int MODE, int CH>
+__global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
+    gemv_stream_kernel(const StreamParams p)
+{
+    using G = Geo<KC>;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    StreamSmem &sm = *reinterpret_cast<StreamSmem *>(smem_raw);
+    const uint32_t ring = smem_u32(smem_raw + kHeader);
+    const int R = p.set_cap;
+    const uint32_t stage_bytes = uint32_t(R) * G::kSlotBytes;
+    int8_t *qs = reinterpret_cast<int8_t *>(smem_raw + kHeader + size_t(kStages) * stage_bytes);
+    volatile int *abort_flag = &sm.abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bx = blockIdx.x;
+    const int64_t g_begin = bx * p.gpc_base + (bx < p.gpc_rem ? bx : p.gpc_rem);
+    const int ng = int(p.gpc_base) + (bx < p.gpc_rem ? 1 : 0);
+    const int subs = int(p.K / G::kStageK);    // stages per set
+    const int64_t slab = 2 * p.K;              // packed bytes of one row group
+    const SetSplit split(ng, R);
+
+    if (tid == 0) {
+        for (int b = 0; b < kStages; ++b) {
+            mbar_init(smem_u32(&sm.full[b]), 1);
+            mbar_init(smem_u32(&sm.empty[b]), KC);
+        }
+        sm.abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    for (int i = tid; i < ng * 8; i += G::kThreads)
+        (&sm.sacc[0][0])[i] = 0;
+    __syncthreads();
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    if (warp == KC) {
+        // ------------------------------------------------ producer warp
+        const uint8_t *src0 = p.packed + g_begin * slab;
+        int t = 0, sb = 0, g0 = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int i = 0; i < split.nsets && ok; ++i) {
+            const int rg = split.size(i);
+            for (int kb = 0; kb < subs; ++kb) {
+                if (!__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.empty[sb]), ph ^ 1u, abort_flag, p.status))) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t full = smem_u32(&sm.full[sb]);
+                if (lane == 0)
+                    mbar_arrive_tx(full, uint32_t(rg) * G::kSlotBytes);
+                __syncwarp();
+                // lanes (t*kMaxSet + r) mod 32 each copy one group's slot
+                const int r = (lane - t * kMaxSet) & 31;
+                if (r < rg)
+                    bulk_load(ring + uint32_t(sb) * stage_bytes + uint32_t(r) * G::kSlotBytes,
+                              src0 + int64_t(g0 + r) * slab + int64_t(kb) * G::kSlotBytes, G::kSlotBytes, full);
+                ++t;
+                if (++sb == kStages) {
+                    sb = 0;
+                    ph ^= 1u;
+                }
+            }
+            g0 += rg;
+        }
+        // the copies still in flight land before the CTA exits (at once,
+        // unless the consumers gave up before taking them)
+        volatile int no_abort = 0;
+        for (int u = t - kStages > 0 ? t - kStages : 0; u < t; ++u)
+            mbar_wait(smem_u32(&sm.full[u % kStages]), uint32_t(u / kStages) & 1u, &no_abort, p.status,
+                      100000000ull);
+        return;
+    }
+
+    // ---------------------------------------------------- consumer warps
+    // (nothing above waits on global memory, so the producer starts at once;
+    // the weight scale's latency hides under the prologue)
+    const float gamma = __ldg(p.w_scale);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if constexpr (MODE == SMODE_Q)
+        stream_copy_q<KC>(p, sm, qs);
+    else if constexpr (MODE == SMODE_X_BF16 && CH > 0)
+        stream_quantize_bf16<KC, CH>(p, sm, qs);
+    else
+        stream_quantize_2pass<KC, MODE == SMODE_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
+    consumers_sync<KC>();   // qs, d and bsum published
+
+    const uint32_t ring_lane = ring + uint32_t(warp) * 512 + uint32_t(lane) * 16;
+    const uint32_t q_lane = smem_u32(qs) + uint32_t(warp) * 256 + uint32_t(lane >> 3) * 64;
+    int acc[kMaxSet][4];
+#pragma unroll
+    for (int r = 0; r < kMaxSet; ++r)
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+            acc[r][a] = 0;
+    int sb = 0, g0 = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int i = 0; i < split.nsets && ok; ++i) {
+        const int rg = split.size(i);
+        for (int kb = 0; kb < subs; ++kb) {
+            if (!__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.full[sb]), ph, abort_flag, p.status))) {
+                ok = false;
+                break;
+            }
+            uint4 q[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                q[j] = lds128(q_lane + uint32_t(kb) * G::kStageK + 16 * j);
+            stage_mac_n<G::kSlotBytes>(rg, ring_lane + uint32_t(sb) * stage_bytes, q, acc);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&sm.empty[sb]));
+            if (++sb == kStages) {
+                sb = 0;
+                ph ^= 1u;
+            }
+        }
+        // the set's groups are complete: fold, sum the four lanes of a row
+        // (lanes l, l^8, l^16, l^24), add into the CTA's row sums
+#pragma unroll
+        for (int r = 0; r < kMaxSet; ++r) {
+            if (r < rg) {
+                int v = acc[r][0] + (acc[r][1] >> 2) + (acc[r][2] >> 4) + (acc[r][3] >> 6);
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+                    acc[r][a] = 0;
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                if (lane < 8)
+                    atomicAdd(&sm.sacc[g0 + r][lane], v);
+            }
+        }
+        g0 += rg;
+    }
+    if (tid == 0) {
+        int rs = 0;
+#pragma unroll
+        for (int w = 0; w < KC; ++w)
+            rs += sm.bsum[w];
+        sm.r = rs;
+    }
+    consumers_sync<KC>();
+    // rescale and write this CTA's rows
+    const float dd = sm.d;
+    const int rs = sm.r;
+    for (int idx = tid; idx < ng * 8; idx += G::kConsumerThreads) {
+        const int64_t row = g_begin * 8 + idx;
+        if (row < p.N) {
+            const int a = (&sm.sacc[0][0])[idx] - rs;
+            if (p.acc_dbg)
+                p.acc_dbg[row] = a;
+            store_y(p.y, p.yt, row, rescale1(a, dd, gamma));
+        }
+    }
+}
+
+template <int KC, int MODE, int CH>
+int launch_mode(const StreamParams &base, int64_t ng_total, cudaStream_t s, unsigned flags)
+{
+    using G = Geo<KC>;
+    const DeviceInfo *di = device_info();
+    if (!di)
+        return BL_ERR_CUDA;
+    auto kern = gemv_stream_kernel<KC, MODE, CH>;
+    auto smem_of = [&](int c) { return kHeader + size_t(kStages) * c * G::kSlotBytes + size_t(base.K); };
+    // R: the smallest stage capacity (>= 4 groups) that fits in shared memory
+    // and gives every CTA of a grid of `ctas` the same number of sets, so that
+    // no CTA streams an extra set of leftovers; 4 (which always fits: K <=
+    // 32768) otherwise
+    auto pick_r = [&](int64_t ctas) {
+        const int64_t lo = ng_total / ctas, hi = lo + (ng_total % ctas ? 1 : 0);
+        for (int c = 4; c <= kMaxSet; ++c)
+            if (smem_of(c) <= size_t(di->max_smem_optin) && (lo + c - 1) / c == (hi + c - 1) / c)
+                return c;
+        return 4;
+    };
+    // G::kCtasPerSm CTAs per SM; one per SM if they do not fit
+    int per_sm = 0, R = 4;
+    int64_t grid_n = 0;
+    for (int want = G::kCtasPerSm; want >= 1; --want) {
+        const int64_t cap = int64_t(want) * di->sm_count;
+        grid_n = ng_total < cap ? ng_total : cap;
+        R = pick_r(grid_n);
+        int st = occupancy(reinterpret_cast<const void *>(kern), G::kThreads, smem_of(R), &per_sm);
+        if (st)
+            return st;
+        if (per_sm >= want)
+            break;
+    }
+    if (per_sm < 1)
+        return BL_ERR_SHAPE;
+    const size_t smem = smem_of(R);
+    StreamParams pp = base;
+    pp.gpc_base = ng_total / grid_n;
+    pp.gpc_rem = int(ng_total % grid_n);
+    pp.set_cap = R;
+    pp.status = di->status;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid_n));
+    cfg.blockDim = dim3(G::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    if (flags & BL_FLAG_PDL) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, pp));
+}
+
+template <int KC>
+int launch_kc(const StreamParams &p, int64_t ng, bool fused, int xt, cudaStream_t s, unsigned flags)
+{
+    if (!fused)
+        return launch_mode<KC, SMODE_Q, 0>(p, ng, s, flags);
+    if (xt != BL_BF16)
+        return launch_mode<KC, SMODE_X_F32, 0>(p, ng, s, flags);
+    // raw bf16 held in registers: at most 8 chunks of 8 values per consumer
+    // thread (32 registers), else two passes over x
+    constexpr int kChunks = 8 * Geo<KC>::kConsumerThreads;
+    if (p.K <= int64_t(4) * kChunks)
+        return launch_mode<KC, SMODE_X_BF16, 4>(p, ng, s, flags);
+    if (p.K <= int64_t(8) * kChunks)
+        return launch_mode<KC, SMODE_X_BF16, 8>(p, ng, s, flags);
+    return launch_mode<KC, SMODE_X_BF16, 0>(p, ng, s, flags);
+}
+
+}  // namespace
+
+// One token, one problem, K a multiple of 4096 (at most 32768), at least four
+// row groups per SM and at most kMaxGroupsPerCta per CTA.
+bool gemv_stream_applies(const GemvBatch &b, int sm_count)
+{
+    if (b.count != 1 || b.M != 1 || b.K % 4096 != 0 || b.K > 32768 || sm_count <= 0)
+        return false;
+    const int64_t ng = (b.prob[0].N + 7) / 8;
+    return ng >= 4 * int64_t(sm_count) && ng <= int64_t(kMaxGroupsPerCta) * sm_count;
+}
+
+int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s)
+{
+    StreamParams p{};
+    p.packed = b.prob[0].packed;
+    p.w_scale = b.prob[0].w_scale;
+    p.N = b.prob[0].N;
+    p.y = b.prob[0].y;
+    p.acc_dbg = b.prob[0].acc_dbg;
+    p.K = b.K;
+    p.q = b.q;
+    p.d = b.d;
+    p.rowsum = b.rowsum;
+    p.x = b.x;
+    p.yt = b.yt;
+    const int64_t ng = (b.prob[0].N + 7) / 8;
+    if (b.K <= kSmallK)
+        return launch_kc<8>(p, ng, fused, b.xt, s, b.flags);
+    return launch_kc<16>(p, ng, fused, b.xt, s, b.flags);
+}
+
+}  // namespace bl

@@ -157,6 +157,25 @@ def test_decode_gemv_100b_shapes(bl, K, N):
     _check_gemv(bl, W, x, torch.bfloat16, True)
 
 
+# One token on a large layer (K a multiple of 4096, at least four row groups
+# per SM) runs the producer/consumer streaming kernel: both 100B shapes,
+# fp32 and bf16 activations, pre-quantised q, fp32 output, ragged N whose
+# last set of groups is short, K = 32768 (the largest register-resident
+# quantisation) and 64 row groups per CTA (its shared row-sum capacity).
+@pytest.mark.parametrize("N,K,fused,xdtype,out_dtype", [
+    (28672, 8192, True, torch.bfloat16, torch.bfloat16),
+    (8192, 28672, True, torch.float32, torch.bfloat16),
+    (8192, 28672, False, torch.bfloat16, torch.float32),
+    (4739, 4096, False, torch.bfloat16, torch.bfloat16),
+    (4739, 32768, True, torch.bfloat16, torch.bfloat16),
+    (4745, 8192, True, torch.float32, torch.float32),
+    (75776, 4096, True, torch.bfloat16, torch.bfloat16),
+])
+def test_gemv_stream_kernel(bl, N, K, fused, xdtype, out_dtype):
+    W, x = seeded_problem(N, K, 1, seed=N + K, xdtype=xdtype)
+    _check_gemv(bl, W, x, out_dtype, fused)
+
+
 @pytest.mark.parametrize("N,K,M", [(13, 64, 1), (1001, 192, 3), (8, 128, 16), (77, 320, 5),
                                    (1, 64, 2), (4096, 64, 7), (24, 10240, 16)])
 @pytest.mark.parametrize("fused", [True, False])
