@@ -263,8 +263,12 @@ def time_graph(graph, steps, world):
     return start.elapsed_time(end) / 1000.0
 
 
-def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda"):
-    """Per-launch time of one shape, rotating distinct weight copies (>= 4x L2)."""
+def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda", pdl=False):
+    """Per-launch time of one shape, rotating distinct weight copies (>= 4x L2).
+
+    pdl: consecutive launches (M = 1) overlap through programmatic dependent
+    launch, as consecutive GEMVs of a decode step do; each still reads x only
+    after the previous launch has finished."""
     nbytes = bl.packed_bytes(N, K)
     if copies is None:
         copies = max(2, int((4 * 126e6) // nbytes) + 1)
@@ -281,7 +285,9 @@ def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda"):
     # the path bl.linear takes: fused dp4a GEMV for few tokens, else quantise +
     # tensor-core GEMM (both launches timed)
     fused = M <= bl.GEMV_FUSED_MAX_M
-    if fused:
+    if fused and pdl:
+        call = lambda wt: bl.gemv_fused_multi([wt], x, outs=[y], pdl=True)  # noqa: E731
+    elif fused:
         call = lambda wt: bl.gemv_fused(wt, x, out=y)  # noqa: E731
     else:
         q = torch.empty(M, K, dtype=torch.int8, device=device)
@@ -310,8 +316,19 @@ def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda"):
     t = s.elapsed_time(e) / 1000.0 / iters
     del g, ws
     return {"K": K, "N": N, "M": M, "us": t * 1e6, "GBps": nbytes / t / 1e9,
-            "weight_copies": copies,
-            "path": "fused dp4a GEMV" if fused else "quantise + tcgen05 GEMM (32-token tiles, split K)"}
+            "weight_copies": copies, "pdl": pdl,
+            "path": gemv_path(K, N, M, fused)}
+
+
+def gemv_path(K, N, M, fused):
+    """Which kernel the library runs for this shape (mirrors its dispatch)."""
+    if not fused:
+        return "quantise + tcgen05 GEMM (32-token tiles, split K)"
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    ng = (N + 7) // 8
+    if M == 1 and K % 4096 == 0 and K <= 32768 and 4 * sms <= ng <= 64 * sms:
+        return "fused streaming GEMV (producer warp, bulk copies, mbarrier ring)"
+    return "fused dp4a GEMV (per-warp cp.async ring)"
 
 
 def isolated_binary(bl, K, N, iters=100, device="cuda"):
@@ -525,8 +542,10 @@ def run_ours(args, world, rank, local):
                 extra[key] = {"error": str(ex)[:300]}
         measure("isolated_2b", lambda: [isolated_gemv(bl, K, N, device=device)
                                         for (K, N) in si.DECODE_SHAPES_2B])
-        measure("isolated_100b", lambda: [isolated_gemv(bl, K, N, iters=50, device=device)
+        measure("isolated_100b", lambda: [isolated_gemv(bl, K, N, iters=200, device=device)
                                           for (K, N) in si.DECODE_SHAPES_100B])
+        measure("chained_100b_pdl", lambda: [isolated_gemv(bl, K, N, iters=200, device=device, pdl=True)
+                                             for (K, N) in si.DECODE_SHAPES_100B])
         measure("small_batch_2560x6912", lambda: [
             isolated_gemv(bl, 2560, 6912, M=m, iters=100, device=device) for m in si.SMALL_BATCH_M])
         measure("binary_100b", lambda: isolated_binary(bl, 8192, 28672, device=device))
