@@ -43,6 +43,28 @@ __device__ __forceinline__ uint4 ld_ro_v4(const void *p)
     return v;
 }
 
+// Data that the preceding launch may have written and that a kernel reads
+// only after griddepcontrol.wait (its activations under programmatic
+// dependent launch): an L2-coherent load, never the non-coherent read-only
+// path, which may serve a value fetched or scheduled before the wait.  The
+// memory clobber keeps the load after the wait in the compiler's order.
+__device__ __forceinline__ uint4 ld_dep_v4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ld_dep_u32(const void *p)
+{
+    uint32_t v;
+    asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // 4-way byte dot product, unsigned bytes of a times signed bytes of b.
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
 {
@@ -80,32 +102,38 @@ __device__ __forceinline__ float warp_max(float v)
     return v;
 }
 
-// Eight input elements (one 16-byte bf16 vector or two fp32 vectors) as fp32.
-template <int XT>
-__device__ __forceinline__ void load8(const void *base, int64_t idx, float f[8]);
-
-template <>
-__device__ __forceinline__ void load8<BL_BF16>(const void *base, int64_t idx, float f[8])
+template <bool DEP>
+__device__ __forceinline__ uint4 ld_in_v4(const void *p)
 {
-    uint4 v = ld_ro_v4(static_cast<const __nv_bfloat16 *>(base) + idx);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
+    if constexpr (DEP)
+        return ld_dep_v4(p);
+    else
+        return ld_ro_v4(p);
 }
 
-template <>
-__device__ __forceinline__ void load8<BL_F32>(const void *base, int64_t idx, float f[8])
+// Eight input elements (one 16-byte bf16 vector or two fp32 vectors) as fp32.
+// DEP: the elements may have been written by the preceding launch (read with
+// the coherent load, see ld_dep_v4).
+template <int XT, bool DEP = false>
+__device__ __forceinline__ void load8(const void *base, int64_t idx, float f[8])
 {
-    const float *p = static_cast<const float *>(base) + idx;
-    uint4 a = ld_ro_v4(p);
-    uint4 b = ld_ro_v4(p + 4);
-    f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y);
-    f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
-    f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y);
-    f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+    if constexpr (XT == BL_BF16) {
+        const uint4 v = ld_in_v4<DEP>(static_cast<const __nv_bfloat16 *>(base) + idx);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    } else {
+        const float *p = static_cast<const float *>(base) + idx;
+        const uint4 a = ld_in_v4<DEP>(p);
+        const uint4 b = ld_in_v4<DEP>(p + 4);
+        f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y);
+        f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+        f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y);
+        f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+    }
 }
 
 // int8 quantisation of one value with the per-token scale s: rint(x * s)

@@ -142,7 +142,7 @@ __device__ __forceinline__ void quantize_prologue_1(const Params &p, Smem<MT> &s
     for (int i = 0; i < 2; ++i) {
         const int c = tid + i * kThreads;
         if (c < chunks) {
-            load8<XT>(p.x, int64_t(c) * 8, f[i]);
+            load8<XT, true>(p.x, int64_t(c) * 8, f[i]);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 amax = fmaxf(amax, fabsf(f[i][j]));
@@ -199,7 +199,7 @@ __device__ __forceinline__ void quantize_prologue(const Params &p, Smem<MT> &sm,
         if (m < p.M)
             for (int64_t c = tid; c < chunks; c += kThreads) {
                 float f[8];
-                load8<XT>(p.x, m * p.ldx + c * 8, f);
+                load8<XT, true>(p.x, m * p.ldx + c * 8, f);
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     pmax[m] = fmaxf(pmax[m], fabsf(f[j]));
@@ -230,7 +230,7 @@ __device__ __forceinline__ void quantize_prologue(const Params &p, Smem<MT> &sm,
             const float s = sm.scale[m];
             for (int64_t c = tid; c < chunks; c += kThreads) {
                 float f[8];
-                load8<XT>(p.x, m * p.ldx + c * 8, f);
+                load8<XT, true>(p.x, m * p.ldx + c * 8, f);
                 uint32_t lo = 0, hi = 0;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -265,15 +265,15 @@ __device__ __forceinline__ void copy_prologue(const Params &p, Smem<MT> &sm, int
 {
     const int64_t vecs = int64_t(p.M) * p.K / 16;
     for (int64_t i = threadIdx.x; i < vecs; i += kThreads)
-        reinterpret_cast<uint4 *>(qs)[i] = ld_ro_v4(p.q + i * 16);
+        reinterpret_cast<uint4 *>(qs)[i] = ld_dep_v4(p.q + i * 16);
     if (threadIdx.x < p.M) {
-        sm.d[threadIdx.x] = p.d[threadIdx.x];
-        sm.r[threadIdx.x] = p.rowsum[threadIdx.x];
+        sm.d[threadIdx.x] = __uint_as_float(ld_dep_u32(p.d + threadIdx.x));
+        sm.r[threadIdx.x] = int(ld_dep_u32(p.rowsum + threadIdx.x));
     }
     // the epilogue reads row sums as the sum over warps of bsum
     for (int i = threadIdx.x; i < kWarps * MT; i += kThreads) {
         const int w = i / MT, m = i % MT;
-        sm.bsum[w][m] = (w == 0 && m < p.M) ? p.rowsum[m] : 0;
+        sm.bsum[w][m] = (w == 0 && m < p.M) ? int(ld_dep_u32(p.rowsum + m)) : 0;
     }
     __syncthreads();
 }

@@ -1,5 +1,5 @@
-// gemv_stream.cu -- ternary decode GEMV for one token on large layers
-// (K a multiple of 4096, thousands of output rows).
+// gemv_stream.cu -- ternary decode GEMV for one token (K a multiple of 256),
+// one or several products sharing the token (q/k/v, gate/up).
 //
 // "How to Run BitNet Inference on GPU Using CUDA Kernels: A Complete Guide",
 // section "Understanding the Two-Phase Architecture": decode is a
@@ -8,23 +8,28 @@
 // beyond the dot product itself lowers the bandwidth an SM can sustain.
 //
 // Design (B200, persistent CTAs):
-//   * A CTA is KC consumer warps plus one producer warp.  Up to K = 8192 it
-//     has KC = 8 and two CTAs share an SM, so that a CTA of the next launch
-//     (programmatic dependent launch) can start streaming beside one of this
-//     launch; for larger K it has KC = 16 and owns the SM, which halves the
-//     per-SM cost of quantising the activations.
-//   * Each CTA owns a contiguous range of 8-row groups (whose packed slabs,
-//     2*K bytes each, are contiguous in the tile layout).  It takes them in
-//     sets of at most R groups, sized evenly, with R (4..8) chosen per launch
-//     so that every CTA has the same number of sets; a set is streamed in
-//     K / (256 KC) stages, a stage holding the same 256*KC-k range of each of
-//     the set's groups (512*KC bytes per group).
+//   * A CTA is KC consumer warps plus one producer warp: KC = 8 up to
+//     K = 8192, else KC = 16.  Large launches (at least 16 row groups per
+//     SM) run two 8-warp CTAs per SM, so that a CTA of the next launch
+//     (programmatic dependent launch) can take the place of one that has
+//     finished, or one 16-warp CTA per SM, which halves the per-SM cost of
+//     quantising a long token.  Smaller launches run at most one CTA per SM,
+//     leaving room beside it for the next launch's CTA, which then fetches
+//     its weights while this launch computes.
+//   * The products' 8-row groups are concatenated into one list; each CTA
+//     owns a contiguous range of it (a group's packed slab, 2*K bytes, is
+//     contiguous in the tile layout).  It takes them in sets of at most R
+//     groups, sized evenly, with R (4..8) chosen per launch so that every CTA
+//     has the same number of sets; a set is streamed in ceil(K / (256 KC))
+//     stages, a stage holding the same k range (up to 256*KC k, 512 bytes per
+//     256 k) of each of the set's groups.
 //   * The producer warp fills a four-stage ring with bulk asynchronous
 //     copies (one copy per group, each from a different lane, since the
 //     copies of one thread complete one after another), completion counted
 //     on the stage's mbarrier.
 //   * Consumer warp w always takes 512-byte piece w of each group in a stage
-//     (lane l: row l%8, 64 k), so the activations it needs, 64 bytes per
+//     (lane l: row l%8, 64 k; in a stage that ends the k range short, only
+//     the warps with a piece compute), so the activations it needs, 64 bytes per
 //     lane, are loaded once per stage and used for all of the stage's groups
 //     (whose loads are issued together, by a body specialised on the group
 //     count).  Multiply with the stored codes s = code + 1: (word &
@@ -51,7 +56,8 @@ constexpr int kMaxConsumers = 16;
 constexpr int kStages = 4;                           // ring stages
 constexpr int kMaxSet = 8;                           // groups per set (stage), at most
 constexpr int kMaxGroupsPerCta = 64;
-constexpr int kSmallK = 8192;                        // up to here: KC = 8, two CTAs per SM
+constexpr int kSmallK = 8192;                        // up to here: KC = 8
+constexpr int kLargeGroupsPerSm = 16;                // from here on: two 8-warp CTAs per SM
 
 // Geometry of a CTA with KC consumer warps.
 template <int KC>
@@ -66,11 +72,9 @@ struct Geo {
 enum { SMODE_Q = 0, SMODE_X_BF16 = 1, SMODE_X_F32 = 2 };
 
 struct StreamParams {
-    const uint8_t *packed;
-    const float *w_scale;
-    int64_t N;
-    void *y;
-    int32_t *acc_dbg;
+    GemvProblem prob[kGemvMaxProblems];
+    int64_t gstart[kGemvMaxProblems + 1];  // prefix sums of the products' row groups
+    int count;
     int64_t K;
     const int8_t *q;
     const float *d;
@@ -92,6 +96,7 @@ struct StreamSmem {
     int bsum[kMaxConsumers];
     float d;
     int r;
+    float wscale[kGemvMaxProblems];   // each product's gamma_eff
     int sacc[kMaxGroupsPerCta][8];
     // followed by the ring (kStages x set_cap slots) and the int8 activations (K bytes)
 };
@@ -111,6 +116,17 @@ struct SetSplit {
     }
     __device__ __forceinline__ int size(int i) const { return base + (i < extra ? 1 : 0); }
 };
+
+// Product of concatenated row group G.
+__device__ __forceinline__ int locate(const StreamParams &p, int64_t G)
+{
+    int pi = 0;
+#pragma unroll
+    for (int i = 1; i < kGemvMaxProblems; ++i)
+        if (i < p.count && G >= p.gstart[i])
+            pi = i;
+    return pi;
+}
 
 __device__ __forceinline__ uint4 lds128(uint32_t saddr)
 {
@@ -196,7 +212,7 @@ __device__ __forceinline__ void stream_quantize_bf16(const StreamParams &p, Stre
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
         const int c = tid + i * T;
-        raw[i] = c < chunks ? ld_ro_v4(static_cast<const __nv_bfloat16 *>(p.x) + int64_t(c) * 8)
+        raw[i] = c < chunks ? ld_dep_v4(static_cast<const __nv_bfloat16 *>(p.x) + int64_t(c) * 8)
                             : make_uint4(0, 0, 0, 0);
     }
     float amax = 0.0f;
@@ -236,7 +252,7 @@ __device__ __forceinline__ void stream_quantize_2pass(const StreamParams &p, Str
 #pragma unroll 4
     for (int c = tid; c < chunks; c += T) {
         float f[8];
-        load8<XT>(p.x, int64_t(c) * 8, f);
+        load8<XT, true>(p.x, int64_t(c) * 8, f);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
             amax = fmaxf(amax, fabsf(f[j]));
@@ -246,7 +262,7 @@ __device__ __forceinline__ void stream_quantize_2pass(const StreamParams &p, Str
 #pragma unroll 4
     for (int c = tid; c < chunks; c += T) {
         float f[8];
-        load8<XT>(p.x, int64_t(c) * 8, f);
+        load8<XT, true>(p.x, int64_t(c) * 8, f);
         *reinterpret_cast<uint2 *>(qs + int64_t(c) * 8) = quant8(f, s, sum);
     }
     sum = __reduce_add_sync(0xffffffffu, sum);
@@ -261,11 +277,11 @@ __device__ __forceinline__ void stream_copy_q(const StreamParams &p, StreamSmem 
     const int tid = threadIdx.x;
     const int vecs = int(p.K / 16);
     for (int i = tid; i < vecs; i += Geo<KC>::kConsumerThreads)
-        reinterpret_cast<uint4 *>(qs)[i] = ld_ro_v4(p.q + int64_t(i) * 16);
+        reinterpret_cast<uint4 *>(qs)[i] = ld_dep_v4(p.q + int64_t(i) * 16);
     if (tid == 0)
-        sm.d = p.d[0];
+        sm.d = __uint_as_float(ld_dep_u32(p.d));
     if (tid < KC)
-        sm.bsum[tid] = tid == 0 ? p.rowsum[0] : 0;
+        sm.bsum[tid] = tid == 0 ? int(ld_dep_u32(p.rowsum)) : 0;
 }
 
 // One 16-byte piece of stored codes (64 k of one row) against the 64
@@ -333,7 +349,8 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
     const int bx = blockIdx.x;
     const int64_t g_begin = bx * p.gpc_base + (bx < p.gpc_rem ? bx : p.gpc_rem);
     const int ng = int(p.gpc_base) + (bx < p.gpc_rem ? 1 : 0);
-    const int subs = int(p.K / G::kStageK);    // stages per set
+    const int P = int(p.K / 256);              // 512-byte pieces per group
+    const int subs = (P + KC - 1) / KC;        // stages per set
     const int64_t slab = 2 * p.K;              // packed bytes of one row group
     const SetSplit split(ng, R);
 
@@ -352,26 +369,36 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
 
     if (warp == KC) {
         // ------------------------------------------------ producer warp
-        const uint8_t *src0 = p.packed + g_begin * slab;
         int t = 0, sb = 0, g0 = 0;
         uint32_t ph = 0;
         bool ok = true;
         for (int i = 0; i < split.nsets && ok; ++i) {
             const int rg = split.size(i);
+            // lane r < rg: the packed slab of the set's group r
+            const uint8_t *src = nullptr;
+            if (lane < rg) {
+                const int64_t G = g_begin + g0 + lane;
+                const int pi = locate(p, G);
+                src = p.prob[pi].packed + (G - p.gstart[pi]) * slab;
+            }
             for (int kb = 0; kb < subs; ++kb) {
+                const int np = min(KC, P - kb * KC);          // pieces of each group in this stage
+                const uint32_t bytes = uint32_t(np) * 512;
                 if (!__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.empty[sb]), ph ^ 1u, abort_flag, p.status))) {
                     ok = false;
                     break;
                 }
                 const uint32_t full = smem_u32(&sm.full[sb]);
                 if (lane == 0)
-                    mbar_arrive_tx(full, uint32_t(rg) * G::kSlotBytes);
+                    mbar_arrive_tx(full, uint32_t(rg) * bytes);
                 __syncwarp();
-                // lanes (t*kMaxSet + r) mod 32 each copy one group's slot
+                // lanes (t*kMaxSet + r) mod 32 each copy one group's part
                 const int r = (lane - t * kMaxSet) & 31;
+                const uint8_t *src_r = reinterpret_cast<const uint8_t *>(
+                    __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src), r & 31));
                 if (r < rg)
                     bulk_load(ring + uint32_t(sb) * stage_bytes + uint32_t(r) * G::kSlotBytes,
-                              src0 + int64_t(g0 + r) * slab + int64_t(kb) * G::kSlotBytes, G::kSlotBytes, full);
+                              src_r + int64_t(kb) * G::kSlotBytes, bytes, full);
                 ++t;
                 if (++sb == kStages) {
                     sb = 0;
@@ -392,7 +419,8 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
     // ---------------------------------------------------- consumer warps
     // (nothing above waits on global memory, so the producer starts at once;
     // the weight scale's latency hides under the prologue)
-    const float gamma = __ldg(p.w_scale);
+    if (tid < p.count)
+        sm.wscale[tid] = __ldg(p.prob[tid].w_scale);
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if constexpr (MODE == SMODE_Q)
         stream_copy_q<KC>(p, sm, qs);
@@ -420,11 +448,13 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
                 ok = false;
                 break;
             }
-            uint4 q[4];
+            if (kb * KC + warp < P) {   // this warp's piece exists in the stage
+                uint4 q[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                q[j] = lds128(q_lane + uint32_t(kb) * G::kStageK + 16 * j);
-            stage_mac_n<G::kSlotBytes>(rg, ring_lane + uint32_t(sb) * stage_bytes, q, acc);
+                for (int j = 0; j < 4; ++j)
+                    q[j] = lds128(q_lane + uint32_t(kb) * G::kStageK + 16 * j);
+                stage_mac_n<G::kSlotBytes>(rg, ring_lane + uint32_t(sb) * stage_bytes, q, acc);
+            }
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(smem_u32(&sm.empty[sb]));
@@ -462,19 +492,23 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
     const float dd = sm.d;
     const int rs = sm.r;
     for (int idx = tid; idx < ng * 8; idx += G::kConsumerThreads) {
-        const int64_t row = g_begin * 8 + idx;
-        if (row < p.N) {
+        const int64_t Gr = g_begin + (idx >> 3);
+        const int pi = locate(p, Gr);
+        const GemvProblem &pr = p.prob[pi];
+        const int64_t row = (Gr - p.gstart[pi]) * 8 + (idx & 7);
+        if (row < pr.N) {
             const int a = (&sm.sacc[0][0])[idx] - rs;
-            if (p.acc_dbg)
-                p.acc_dbg[row] = a;
-            store_y(p.y, p.yt, row, rescale1(a, dd, gamma));
+            if (pr.acc_dbg)
+                pr.acc_dbg[row] = a;
+            store_y(pr.y, p.yt, row, rescale1(a, dd, sm.wscale[pi]));
         }
     }
 }
 
 template <int KC, int MODE, int CH>
-int launch_mode(const StreamParams &base, int64_t ng_total, cudaStream_t s, unsigned flags)
+int launch_mode(const StreamParams &base, cudaStream_t s, unsigned flags)
 {
+    const int64_t ng_total = base.gstart[base.count];
     using G = Geo<KC>;
     const DeviceInfo *di = device_info();
     if (!di)
@@ -492,10 +526,13 @@ int launch_mode(const StreamParams &base, int64_t ng_total, cudaStream_t s, unsi
                 return c;
         return 4;
     };
-    // G::kCtasPerSm CTAs per SM; one per SM if they do not fit
+    // large launches (>= kLargeGroupsPerSm row groups per SM): G::kCtasPerSm
+    // CTAs per SM (one if they do not fit); the others at most one per SM,
+    // which leaves room beside each CTA for one of the next launch
+    const int top = ng_total >= kLargeGroupsPerSm * int64_t(di->sm_count) ? G::kCtasPerSm : 1;
     int per_sm = 0, R = 4;
     int64_t grid_n = 0;
-    for (int want = G::kCtasPerSm; want >= 1; --want) {
+    for (int want = top; want >= 1; --want) {
         const int64_t cap = int64_t(want) * di->sm_count;
         grid_n = ng_total < cap ? ng_total : cap;
         R = pick_r(grid_n);
@@ -530,52 +567,56 @@ int launch_mode(const StreamParams &base, int64_t ng_total, cudaStream_t s, unsi
 }
 
 template <int KC>
-int launch_kc(const StreamParams &p, int64_t ng, bool fused, int xt, cudaStream_t s, unsigned flags)
+int launch_kc(const StreamParams &p, bool fused, int xt, cudaStream_t s, unsigned flags)
 {
     if (!fused)
-        return launch_mode<KC, SMODE_Q, 0>(p, ng, s, flags);
+        return launch_mode<KC, SMODE_Q, 0>(p, s, flags);
     if (xt != BL_BF16)
-        return launch_mode<KC, SMODE_X_F32, 0>(p, ng, s, flags);
+        return launch_mode<KC, SMODE_X_F32, 0>(p, s, flags);
     // raw bf16 held in registers: at most 8 chunks of 8 values per consumer
     // thread (32 registers), else two passes over x
     constexpr int kChunks = 8 * Geo<KC>::kConsumerThreads;
     if (p.K <= int64_t(4) * kChunks)
-        return launch_mode<KC, SMODE_X_BF16, 4>(p, ng, s, flags);
+        return launch_mode<KC, SMODE_X_BF16, 4>(p, s, flags);
     if (p.K <= int64_t(8) * kChunks)
-        return launch_mode<KC, SMODE_X_BF16, 8>(p, ng, s, flags);
-    return launch_mode<KC, SMODE_X_BF16, 0>(p, ng, s, flags);
+        return launch_mode<KC, SMODE_X_BF16, 8>(p, s, flags);
+    return launch_mode<KC, SMODE_X_BF16, 0>(p, s, flags);
 }
 
 }  // namespace
 
-// One token, one problem, K a multiple of 4096 (at most 32768), at least four
-// row groups per SM and at most kMaxGroupsPerCta per CTA.
+// One token, K a multiple of 256 (at most 32768), at most kMaxGroupsPerCta
+// row groups per CTA (one CTA per SM).
 bool gemv_stream_applies(const GemvBatch &b, int sm_count)
 {
-    if (b.count != 1 || b.M != 1 || b.K % 4096 != 0 || b.K > 32768 || sm_count <= 0)
+    if (b.M != 1 || b.K % 256 != 0 || b.K > 32768 || b.count < 1 || sm_count <= 0)
         return false;
-    const int64_t ng = (b.prob[0].N + 7) / 8;
-    return ng >= 4 * int64_t(sm_count) && ng <= int64_t(kMaxGroupsPerCta) * sm_count;
+    int64_t ng = 0;
+    for (int i = 0; i < b.count; ++i)
+        ng += (b.prob[i].N + 7) / 8;
+    return ng <= int64_t(kMaxGroupsPerCta) * sm_count;
 }
 
 int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s)
 {
     StreamParams p{};
-    p.packed = b.prob[0].packed;
-    p.w_scale = b.prob[0].w_scale;
-    p.N = b.prob[0].N;
-    p.y = b.prob[0].y;
-    p.acc_dbg = b.prob[0].acc_dbg;
+    p.count = b.count;
+    p.gstart[0] = 0;
+    for (int i = 0; i < b.count; ++i) {
+        p.prob[i] = b.prob[i];
+        p.gstart[i + 1] = p.gstart[i] + (b.prob[i].N + 7) / 8;
+    }
+    for (int i = b.count; i < kGemvMaxProblems; ++i)
+        p.gstart[i + 1] = p.gstart[b.count];
     p.K = b.K;
     p.q = b.q;
     p.d = b.d;
     p.rowsum = b.rowsum;
     p.x = b.x;
     p.yt = b.yt;
-    const int64_t ng = (b.prob[0].N + 7) / 8;
     if (b.K <= kSmallK)
-        return launch_kc<8>(p, ng, fused, b.xt, s, b.flags);
-    return launch_kc<16>(p, ng, fused, b.xt, s, b.flags);
+        return launch_kc<8>(p, fused, b.xt, s, b.flags);
+    return launch_kc<16>(p, fused, b.xt, s, b.flags);
 }
 
 }  // namespace bl

@@ -176,6 +176,42 @@ def test_gemv_stream_kernel(bl, N, K, fused, xdtype, out_dtype):
     _check_gemv(bl, W, x, out_dtype, fused)
 
 
+# One token with K a multiple of 256 always runs the streaming kernel: ragged
+# last stages (K = 2304: 9 pieces of 256 k; 768: 3; 256: 1), products of
+# mixed sizes whose concatenated row groups straddle product boundaries inside
+# a CTA's sets, eight products at once, small and large launches.
+@pytest.mark.parametrize("Ns,K,fused,xdtype", [
+    ([1001], 2304, True, torch.bfloat16),
+    ([8], 256, False, torch.bfloat16),
+    ([1], 768, True, torch.float32),
+    ([4739], 2304, False, torch.bfloat16),
+    ([2000, 3001, 17, 4500], 1280, True, torch.bfloat16),
+    ([640, 13, 2560, 999, 64, 7, 1500, 3], 6912, True, torch.float32),
+    ([6912, 6912], 2560, True, torch.bfloat16),
+])
+def test_gemv_stream_products_and_ragged_k(bl, Ns, K, fused, xdtype):
+    x = si.activations(1, K, seed=K + len(Ns), dtype=xdtype)
+    ws, refs = [], []
+    for i, N in enumerate(Ns):
+        W = si.weight(N, K, seed=900 + 7 * i + N)
+        g, codes, _ = oracle_weight(W)
+        refs.append(_oracle_gemv(g, codes, x))
+        ws.append(_pack_gpu(bl, W))
+    accs = [torch.empty(1, N, dtype=torch.int32, device=dev()) for N in Ns]
+    xd = x.to(dev())
+    if fused:
+        outs = bl.gemv_fused_multi(ws, xd, acc_dbgs=accs)
+    else:
+        assert len(ws) == 1
+        q, d, r = bl.quantize_act(xd)
+        outs = [bl.gemv(ws[0], q, d, r, acc_dbg=accs[0])]
+    torch.cuda.synchronize()
+    for (y_o, acc_o), y, acc in zip(refs, outs, accs):
+        np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+        compare_outputs(y, y_o)
+    assert bl.last_device_status() == 0
+
+
 @pytest.mark.parametrize("N,K,M", [(13, 64, 1), (1001, 192, 3), (8, 128, 16), (77, 320, 5),
                                    (1, 64, 2), (4096, 64, 7), (24, 10240, 16)])
 @pytest.mark.parametrize("fused", [True, False])
@@ -365,15 +401,18 @@ def test_multi_gemv_qkv_shapes(bl, M):
         compare_outputs(y, y_o)
 
 
-def test_pdl_dependent_chain(bl):
+@pytest.mark.parametrize("K,M", [(2560, 1), (2560, 3), (8192, 1)])
+def test_pdl_dependent_chain(bl, K, M):
     """A chain where each launch reads the previous launch's output, all with
-    BL_FLAG_PDL, inside a CUDA graph: the result must equal the oracle chain."""
-    K = 2560
+    BL_FLAG_PDL, inside a CUDA graph (so that consecutive launches really
+    overlap): the result must equal the oracle chain.  One token at K = 2560
+    runs small streaming launches, three tokens the per-warp-ring kernel, one
+    token at K = 8192 large streaming launches (two CTAs per SM)."""
     Ws = [si.weight(K, K, seed=70 + i) for i in range(6)]
     oracles = [oracle_weight(W) for W in Ws]
     ws = [_pack_gpu(bl, W) for W in Ws]
-    x0 = si.activations(1, K, seed=77)
-    xs = [x0.to(dev())] + [torch.empty(1, K, dtype=torch.bfloat16, device=dev()) for _ in Ws]
+    x0 = si.activations(M, K, seed=77)
+    xs = [x0.to(dev())] + [torch.empty(M, K, dtype=torch.bfloat16, device=dev()) for _ in Ws]
     for _ in range(2):  # warm-up, eager
         for i, w in enumerate(ws):
             bl.gemv_fused_multi([w], xs[i], outs=[xs[i + 1]], pdl=True)
