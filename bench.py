@@ -74,7 +74,7 @@ def profiled_traffic():
     import hashlib
     import re
     prof = os.path.join(ROOT, "profiles", "decode_stream_2b_gemv_launches.md")
-    src = os.path.join(ROOT, "bit_ternary_weight_b200", "csrc", "gemv.cu")
+    src = os.path.join(ROOT, "bit_ternary_weight_b200", "csrc", "gemv_stream.cu")
     try:
         text = open(prof).read()
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
@@ -571,7 +571,7 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": value / world, "peak": hbm, "unit": "GB/s",
                      "frac": value / world / hbm, "traffic": profiled_traffic(),
                      "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                     "kernel": "gemv_kernel<1, bf16 fused> (4 launches per layer)",
+                     "kernel": "gemv_stream_kernel<KC=8, bf16 fused> (4 launches per layer)",
                      "note": "algorithmic bytes = packed weight bytes per launch; duration = "
                              "step time / launches (CUDA events over the timed region)"},
         "cpu_baseline": cpu,

@@ -199,21 +199,23 @@ __device__ __forceinline__ float stream_scale(StreamSmem &sm, float amax)
     return __fdiv_rn(kQb, a_eff);
 }
 
-// Quantise the token x (K bf16 values) into qs: absmax, s = 127 / max(amax,
-// eps), q = clamp(rint(x * s)); each warp's partial row sum goes to bsum.
-// x stays in registers as raw bf16, CH 16-byte chunks per thread.
+// Quantise the token x into qs.  Consumer warp w only ever reads the
+// activations of its own pieces (256 k each: pieces w, w + KC, w + 2 KC, ...),
+// so it quantises exactly those and needs no block barrier afterwards; only
+// the absmax is block-wide.  s = 127 / max(amax, eps), q = clamp(rint(x *
+// s)); each warp's partial row sum goes to bsum.  Lane l takes elements
+// 8l .. 8l + 7 of each piece; x stays in registers as raw bf16, CH pieces.
 template <int KC, int CH>
 __device__ __forceinline__ void stream_quantize_bf16(const StreamParams &p, StreamSmem &sm, int8_t *qs)
 {
-    constexpr int T = Geo<KC>::kConsumerThreads;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int chunks = int(p.K / 8);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int P = int(p.K / 256);
     uint4 raw[CH];
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
-        const int c = tid + i * T;
-        raw[i] = c < chunks ? ld_dep_v4(static_cast<const __nv_bfloat16 *>(p.x) + int64_t(c) * 8)
-                            : make_uint4(0, 0, 0, 0);
+        const int j = i * KC + warp;
+        raw[i] = j < P ? ld_dep_v4(static_cast<const __nv_bfloat16 *>(p.x) + (int64_t(j) * 32 + lane) * 8)
+                       : make_uint4(0, 0, 0, 0);
     }
     float amax = 0.0f;
 #pragma unroll
@@ -221,67 +223,72 @@ __device__ __forceinline__ void stream_quantize_bf16(const StreamParams &p, Stre
         float f[8];
         bf16x8_f32(raw[i], f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            amax = fmaxf(amax, fabsf(f[j]));
+        for (int e = 0; e < 8; ++e)
+            amax = fmaxf(amax, fabsf(f[e]));
     }
     const float s = stream_scale<KC>(sm, amax);
     int sum = 0;
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
-        const int c = tid + i * T;
-        if (c < chunks) {
+        const int j = i * KC + warp;
+        if (j < P) {
             float f[8];
             bf16x8_f32(raw[i], f);
-            *reinterpret_cast<uint2 *>(qs + int64_t(c) * 8) = quant8(f, s, sum);
+            *reinterpret_cast<uint2 *>(qs + (j * 32 + lane) * 8) = quant8(f, s, sum);
         }
     }
     sum = __reduce_add_sync(0xffffffffu, sum);
     if (lane == 0)
         sm.bsum[warp] = sum;
+    __syncwarp();
 }
 
-// The same for any K and either input type: one pass for the absmax, a
-// second one that reads x again (from L2) to quantise.
+// The same for any K and either input type: one pass over the warp's pieces
+// for the absmax, a second one that reads them again (from L2) to quantise.
 template <int KC, int XT>
 __device__ __forceinline__ void stream_quantize_2pass(const StreamParams &p, StreamSmem &sm, int8_t *qs)
 {
-    constexpr int T = Geo<KC>::kConsumerThreads;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int chunks = int(p.K / 8);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int P = int(p.K / 256);
     float amax = 0.0f;
 #pragma unroll 4
-    for (int c = tid; c < chunks; c += T) {
+    for (int j = warp; j < P; j += KC) {
         float f[8];
-        load8<XT, true>(p.x, int64_t(c) * 8, f);
+        load8<XT, true>(p.x, (int64_t(j) * 32 + lane) * 8, f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            amax = fmaxf(amax, fabsf(f[j]));
+        for (int e = 0; e < 8; ++e)
+            amax = fmaxf(amax, fabsf(f[e]));
     }
     const float s = stream_scale<KC>(sm, amax);
     int sum = 0;
 #pragma unroll 4
-    for (int c = tid; c < chunks; c += T) {
+    for (int j = warp; j < P; j += KC) {
         float f[8];
-        load8<XT, true>(p.x, int64_t(c) * 8, f);
-        *reinterpret_cast<uint2 *>(qs + int64_t(c) * 8) = quant8(f, s, sum);
+        load8<XT, true>(p.x, (int64_t(j) * 32 + lane) * 8, f);
+        *reinterpret_cast<uint2 *>(qs + (j * 32 + lane) * 8) = quant8(f, s, sum);
     }
     sum = __reduce_add_sync(0xffffffffu, sum);
     if (lane == 0)
         sm.bsum[warp] = sum;
+    __syncwarp();
 }
 
-// Pre-quantised activations: copy q into shared memory, take d and the row sum.
+// Pre-quantised activations: each warp copies the q of its own pieces (no
+// block barrier); warp 0 takes d and the row sum.
 template <int KC>
 __device__ __forceinline__ void stream_copy_q(const StreamParams &p, StreamSmem &sm, int8_t *qs)
 {
-    const int tid = threadIdx.x;
-    const int vecs = int(p.K / 16);
-    for (int i = tid; i < vecs; i += Geo<KC>::kConsumerThreads)
-        reinterpret_cast<uint4 *>(qs)[i] = ld_dep_v4(p.q + int64_t(i) * 16);
-    if (tid == 0)
-        sm.d = __uint_as_float(ld_dep_u32(p.d));
-    if (tid < KC)
-        sm.bsum[tid] = tid == 0 ? int(ld_dep_u32(p.rowsum)) : 0;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int P = int(p.K / 256);
+    for (int j = warp; j < P; j += KC)
+        if (lane < 16)
+            *reinterpret_cast<uint4 *>(qs + j * 256 + lane * 16) = ld_dep_v4(p.q + int64_t(j) * 256 + lane * 16);
+    if (lane == 0) {
+        sm.bsum[warp] = warp == 0 ? int(ld_dep_u32(p.rowsum)) : 0;
+        if (warp == 0)
+            sm.d = __uint_as_float(ld_dep_u32(p.d));
+    }
+    __syncwarp();
 }
 
 // One 16-byte piece of stored codes (64 k of one row) against the 64
@@ -428,7 +435,7 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
         stream_quantize_bf16<KC, CH>(p, sm, qs);
     else
         stream_quantize_2pass<KC, MODE == SMODE_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
-    consumers_sync<KC>();   // qs, d and bsum published
+    // (each warp reads only the activations it wrote itself: no barrier)
 
     const uint32_t ring_lane = ring + uint32_t(warp) * 512 + uint32_t(lane) * 16;
     const uint32_t q_lane = smem_u32(qs) + uint32_t(warp) * 256 + uint32_t(lane >> 3) * 64;
