@@ -95,7 +95,6 @@ struct StreamSmem {
     alignas(16) float bmax[kMaxConsumers];   // read back as float4
     int bsum[kMaxConsumers];
     float d;
-    int r;
     float wscale[kGemvMaxProblems];   // each product's gamma_eff
     int sacc[kMaxGroupsPerCta][8];
     // followed by the ring (kStages x set_cap slots) and the int8 activations (K bytes)
@@ -335,6 +334,48 @@ __device__ __forceinline__ void stage_mac_n(int rg, uint32_t base, const uint4 (
 }
 static_assert(kMaxSet == 8, "stage_mac_n covers 1..8 groups");
 
+// End of a set of RG groups for this warp: fold each group's four
+// accumulators, sum the four lanes of a row (lanes l, l^8, l^16, l^24) and
+// add the row's partial into the CTA's row sums; the groups' shuffle chains
+// are independent and interleave.
+template <int RG>
+__device__ __forceinline__ void set_flush(int (&acc)[kMaxSet][4], int (*sacc)[8], int lane)
+{
+    int v[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+        v[r] = acc[r][0] + (acc[r][1] >> 2) + (acc[r][2] >> 4) + (acc[r][3] >> 6);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+            acc[r][a] = 0;
+    }
+#pragma unroll
+    for (int r = 0; r < RG; ++r)
+        v[r] += __shfl_xor_sync(0xffffffffu, v[r], 8);
+#pragma unroll
+    for (int r = 0; r < RG; ++r)
+        v[r] += __shfl_xor_sync(0xffffffffu, v[r], 16);
+    if (lane < 8) {
+#pragma unroll
+        for (int r = 0; r < RG; ++r)
+            atomicAdd(&sacc[r][lane], v[r]);
+    }
+}
+
+__device__ __forceinline__ void set_flush_n(int rg, int (&acc)[kMaxSet][4], int (*sacc)[8], int lane)
+{
+    switch (rg) {
+    case 1: set_flush<1>(acc, sacc, lane); break;
+    case 2: set_flush<2>(acc, sacc, lane); break;
+    case 3: set_flush<3>(acc, sacc, lane); break;
+    case 4: set_flush<4>(acc, sacc, lane); break;
+    case 5: set_flush<5>(acc, sacc, lane); break;
+    case 6: set_flush<6>(acc, sacc, lane); break;
+    case 7: set_flush<7>(acc, sacc, lane); break;
+    default: set_flush<8>(acc, sacc, lane); break;
+    }
+}
+
 // Ring protocol.  Stage t (set i, k-range kb) occupies ring slot
 // t % kStages, room for R groups, of which it fills |set i|; full[slot]
 // counts its bytes, empty[slot] the KC consumer warps that have read it
@@ -470,34 +511,17 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
                 ph ^= 1u;
             }
         }
-        // the set's groups are complete: fold, sum the four lanes of a row
-        // (lanes l, l^8, l^16, l^24), add into the CTA's row sums
-#pragma unroll
-        for (int r = 0; r < kMaxSet; ++r) {
-            if (r < rg) {
-                int v = acc[r][0] + (acc[r][1] >> 2) + (acc[r][2] >> 4) + (acc[r][3] >> 6);
-#pragma unroll
-                for (int a = 0; a < 4; ++a)
-                    acc[r][a] = 0;
-                v += __shfl_xor_sync(0xffffffffu, v, 8);
-                v += __shfl_xor_sync(0xffffffffu, v, 16);
-                if (lane < 8)
-                    atomicAdd(&sm.sacc[g0 + r][lane], v);
-            }
-        }
+        // the set's groups are complete: add their partial row sums
+        set_flush_n(rg, acc, &sm.sacc[g0], lane);
         g0 += rg;
-    }
-    if (tid == 0) {
-        int rs = 0;
-#pragma unroll
-        for (int w = 0; w < KC; ++w)
-            rs += sm.bsum[w];
-        sm.r = rs;
     }
     consumers_sync<KC>();
     // rescale and write this CTA's rows
     const float dd = sm.d;
-    const int rs = sm.r;
+    int rs = 0;
+#pragma unroll
+    for (int w = 0; w < KC; ++w)
+        rs += sm.bsum[w];
     for (int idx = tid; idx < ng * 8; idx += G::kConsumerThreads) {
         const int64_t Gr = g_begin + (idx >> 3);
         const int pi = locate(p, Gr);
