@@ -20,16 +20,17 @@
 //     owns a contiguous range of it (a group's packed slab, 2*K bytes, is
 //     contiguous in the tile layout).  It takes them in sets of at most R
 //     groups, sized evenly, with R (4..8) chosen per launch so that every CTA
-//     has the same number of sets; a set is streamed in ceil(K / (256 KC))
-//     stages, a stage holding the same k range (up to 256*KC k, 512 bytes per
-//     256 k) of each of the set's groups.
+//     has the same number of sets; a set is streamed in stages, a stage
+//     holding the same k range of each of the set's groups (512 bytes per
+//     256 k): the whole range when it is at most 512*KC k, else 256*KC k.
 //   * The producer warp fills a four-stage ring with bulk asynchronous
 //     copies (one copy per group, each from a different lane, since the
 //     copies of one thread complete one after another), completion counted
 //     on the stage's mbarrier.
-//   * Consumer warp w always takes 512-byte piece w of each group in a stage
-//     (lane l: row l%8, 64 k; in a stage that ends the k range short, only
-//     the warps with a piece compute), so the activations it needs, 64 bytes per
+//   * Consumer warp w always takes 512-byte pieces w (and w + KC) of each
+//     group in a stage (lane l: row l%8, 64 k; in a stage that ends the k
+//     range short, only the warps with a piece compute), so the activations
+//     it needs, 64 bytes per
 //     lane, are loaded once per stage and used for all of the stage's groups
 //     (whose loads are issued together, by a body specialised on the group
 //     count).  Multiply with the stored codes s = code + 1: (word &
@@ -64,12 +65,15 @@ template <int KC>
 struct Geo {
     static constexpr int kConsumerThreads = 32 * KC;
     static constexpr int kThreads = kConsumerThreads + 32;   // + the producer warp
-    static constexpr int kStageK = 256 * KC;                 // k of one group per stage
-    static constexpr int kSlotBytes = 2 * kStageK;           // its packed bytes (8 rows x 2 bits)
     static constexpr int kCtasPerSm = KC == 8 ? 2 : 1;
 };
 
 enum { SMODE_Q = 0, SMODE_X_BF16 = 1, SMODE_X_F32 = 2 };
+
+// 512-byte pieces (256 k) of one group per stage: the whole k range when it
+// is at most two pieces per consumer warp (one stage per set), else one per
+// warp.  Either way warp w only ever takes pieces w, w + KC, w + 2 KC, ...
+__host__ __device__ __forceinline__ int stage_pieces(int P, int KC) { return P <= 2 * KC ? P : KC; }
 
 struct StreamParams {
     GemvProblem prob[kGemvMaxProblems];
@@ -304,32 +308,36 @@ __device__ __forceinline__ void mac4(const uint4 wv, const uint4 (&q)[4], int (&
     }
 }
 
-// One stage of RG groups for this lane: the RG slots are consecutive, so the
-// loads take immediate offsets and are all issued before the arithmetic.
+// One stage of RG groups for this lane: the RG slots lie SLOT bytes apart
+// (a compile-time stride when SLOT > 0, so the loads take immediate offsets;
+// else slot_rt), and all loads are issued before the arithmetic.
 template <int SLOT, int RG>
-__device__ __forceinline__ void stage_mac(uint32_t base, const uint4 (&q)[4], int (&acc)[kMaxSet][4])
+__device__ __forceinline__ void stage_mac(uint32_t base, uint32_t slot_rt, const uint4 (&q)[4],
+                                          int (&acc)[kMaxSet][4])
 {
+    const uint32_t slot = SLOT > 0 ? uint32_t(SLOT) : slot_rt;
     uint4 wv[RG];
 #pragma unroll
     for (int r = 0; r < RG; ++r)
-        wv[r] = lds128(base + r * SLOT);
+        wv[r] = lds128(base + r * slot);
 #pragma unroll
     for (int r = 0; r < RG; ++r)
         mac4(wv[r], q, acc[r]);
 }
 
 template <int SLOT>
-__device__ __forceinline__ void stage_mac_n(int rg, uint32_t base, const uint4 (&q)[4], int (&acc)[kMaxSet][4])
+__device__ __forceinline__ void stage_mac_n(int rg, uint32_t base, uint32_t slot, const uint4 (&q)[4],
+                                            int (&acc)[kMaxSet][4])
 {
     switch (rg) {
-    case 1: stage_mac<SLOT, 1>(base, q, acc); break;
-    case 2: stage_mac<SLOT, 2>(base, q, acc); break;
-    case 3: stage_mac<SLOT, 3>(base, q, acc); break;
-    case 4: stage_mac<SLOT, 4>(base, q, acc); break;
-    case 5: stage_mac<SLOT, 5>(base, q, acc); break;
-    case 6: stage_mac<SLOT, 6>(base, q, acc); break;
-    case 7: stage_mac<SLOT, 7>(base, q, acc); break;
-    default: stage_mac<SLOT, 8>(base, q, acc); break;
+    case 1: stage_mac<SLOT, 1>(base, slot, q, acc); break;
+    case 2: stage_mac<SLOT, 2>(base, slot, q, acc); break;
+    case 3: stage_mac<SLOT, 3>(base, slot, q, acc); break;
+    case 4: stage_mac<SLOT, 4>(base, slot, q, acc); break;
+    case 5: stage_mac<SLOT, 5>(base, slot, q, acc); break;
+    case 6: stage_mac<SLOT, 6>(base, slot, q, acc); break;
+    case 7: stage_mac<SLOT, 7>(base, slot, q, acc); break;
+    default: stage_mac<SLOT, 8>(base, slot, q, acc); break;
     }
 }
 static_assert(kMaxSet == 8, "stage_mac_n covers 1..8 groups");
@@ -389,7 +397,10 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
     StreamSmem &sm = *reinterpret_cast<StreamSmem *>(smem_raw);
     const uint32_t ring = smem_u32(smem_raw + kHeader);
     const int R = p.set_cap;
-    const uint32_t stage_bytes = uint32_t(R) * G::kSlotBytes;
+    const int P = int(p.K / 256);              // 512-byte pieces per group
+    const int PS = stage_pieces(P, KC);        // pieces of each group per stage
+    const uint32_t slot = uint32_t(PS) * 512;  // ring bytes of one group per stage
+    const uint32_t stage_bytes = uint32_t(R) * slot;
     int8_t *qs = reinterpret_cast<int8_t *>(smem_raw + kHeader + size_t(kStages) * stage_bytes);
     volatile int *abort_flag = &sm.abort_flag;
 
@@ -397,8 +408,7 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
     const int bx = blockIdx.x;
     const int64_t g_begin = bx * p.gpc_base + (bx < p.gpc_rem ? bx : p.gpc_rem);
     const int ng = int(p.gpc_base) + (bx < p.gpc_rem ? 1 : 0);
-    const int P = int(p.K / 256);              // 512-byte pieces per group
-    const int subs = (P + KC - 1) / KC;        // stages per set
+    const int subs = (P + PS - 1) / PS;        // stages per set
     const int64_t slab = 2 * p.K;              // packed bytes of one row group
     const SetSplit split(ng, R);
 
@@ -430,7 +440,7 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
                 src = p.prob[pi].packed + (G - p.gstart[pi]) * slab;
             }
             for (int kb = 0; kb < subs; ++kb) {
-                const int np = min(KC, P - kb * KC);          // pieces of each group in this stage
+                const int np = min(PS, P - kb * PS);          // pieces of each group in this stage
                 const uint32_t bytes = uint32_t(np) * 512;
                 if (!__all_sync(0xffffffffu, mbar_wait_fast(smem_u32(&sm.empty[sb]), ph ^ 1u, abort_flag, p.status))) {
                     ok = false;
@@ -445,8 +455,8 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
                 const uint8_t *src_r = reinterpret_cast<const uint8_t *>(
                     __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src), r & 31));
                 if (r < rg)
-                    bulk_load(ring + uint32_t(sb) * stage_bytes + uint32_t(r) * G::kSlotBytes,
-                              src_r + int64_t(kb) * G::kSlotBytes, bytes, full);
+                    bulk_load(ring + uint32_t(sb) * stage_bytes + uint32_t(r) * slot,
+                              src_r + int64_t(kb) * slot, bytes, full);
                 ++t;
                 if (++sb == kStages) {
                     sb = 0;
@@ -496,12 +506,28 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
                 ok = false;
                 break;
             }
-            if (kb * KC + warp < P) {   // this warp's piece exists in the stage
-                uint4 q[4];
+            // this warp's pieces of the stage: w and (one stage per set) w + KC
+            const int np = min(PS, P - kb * PS);
+            if (PS == KC) {
+                if (warp < np) {
+                    uint4 q[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    q[j] = lds128(q_lane + uint32_t(kb) * G::kStageK + 16 * j);
-                stage_mac_n<G::kSlotBytes>(rg, ring_lane + uint32_t(sb) * stage_bytes, q, acc);
+                    for (int j = 0; j < 4; ++j)
+                        q[j] = lds128(q_lane + uint32_t(kb * KC) * 256 + 16 * j);
+                    stage_mac_n<KC * 512>(rg, ring_lane + uint32_t(sb) * stage_bytes, slot, q, acc);
+                }
+            } else {
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    if (warp + m * KC < np) {
+                        uint4 q[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            q[j] = lds128(q_lane + uint32_t(m * KC) * 256 + 16 * j);
+                        stage_mac_n<0>(rg, ring_lane + uint32_t(sb) * stage_bytes + uint32_t(m * KC) * 512, slot, q,
+                                       acc);
+                    }
+                }
             }
             __syncwarp();
             if (lane == 0)
@@ -545,7 +571,8 @@ int launch_mode(const StreamParams &base, cudaStream_t s, unsigned flags)
     if (!di)
         return BL_ERR_CUDA;
     auto kern = gemv_stream_kernel<KC, MODE, CH>;
-    auto smem_of = [&](int c) { return kHeader + size_t(kStages) * c * G::kSlotBytes + size_t(base.K); };
+    const int ps = stage_pieces(int(base.K / 256), KC);
+    auto smem_of = [&](int c) { return kHeader + size_t(kStages) * c * ps * 512 + size_t(base.K); };
     // R: the smallest stage capacity (>= 4 groups) that fits in shared memory
     // and gives every CTA of a grid of `ctas` the same number of sets, so that
     // no CTA streams an extra set of leftovers; 4 (which always fits: K <=
