@@ -326,7 +326,7 @@ def gemv_path(K, N, M, fused):
         return "quantise + tcgen05 GEMM (32-token tiles, split K)"
     sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     ng = (N + 7) // 8
-    if M == 1 and K % 4096 == 0 and K <= 32768 and 4 * sms <= ng <= 64 * sms:
+    if M == 1 and K % 256 == 0 and K <= 32768 and ng <= 64 * sms:
         return "fused streaming GEMV (producer warp, bulk copies, mbarrier ring)"
     return "fused dp4a GEMV (per-warp cp.async ring)"
 

@@ -1,4 +1,8 @@
-// gemv.cu -- ternary decode GEMV for 1 <= M <= 16 tokens (M = 1 is decode).
+// gemv.cu -- ternary decode GEMV for 1 <= M <= 16 tokens with a per-warp
+// weight ring.  One token with K a multiple of 256 runs the streaming kernel
+// of gemv_stream.cu instead (launch_gemv_batch routes it there); this kernel
+// takes the fused entry points' small batches (2..16 tokens) and single
+// tokens whose K is not a multiple of 256.
 //
 // "How to Run BitNet Inference on GPU Using CUDA Kernels: A Complete Guide",
 // sections "Understanding the Two-Phase Architecture" and "Key Components and
@@ -26,7 +30,9 @@
 //     fetch of one BitLinear overlaps the tail of the previous one.
 //   * The activations (int8, M*K bytes) sit in shared memory.  The fused
 //     entry points quantise x in the prologue (absmax, scale, rint, row sum;
-//     one register-resident pass for a single token).
+//     one register-resident pass for a single token).  Everything the
+//     preceding launch may have written (x, or q, d and the row sums) is read
+//     after the dependency wait with L2-coherent loads.
 //   * Inner loop, stored codes s = code + 1 in {0,1,2}: for four consecutive
 //     k, (word & 0x03030303), (word & 0x0c0c0c0c), (word & 0x30303030) and
 //     (word & 0xc0c0c0c0) hold s, 4s, 16s, 64s per byte; dp4a (unsigned x
