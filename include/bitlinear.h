@@ -174,6 +174,12 @@ int bitlinear_gemv(const uint8_t *packed, const float *w_scale, int64_t N,
  * whole decode BitLinear (quantise, product, rescale) in one launch.
  *   x    device, [M][ldx] of dtype xt (BL_F32 or BL_BF16)
  *   other arguments as for bitlinear_gemv.
+ * One token with K a multiple of 256 (at most 32768) runs a streaming kernel
+ * (a producer warp fills a shared-memory ring with bulk copies of the packed
+ * weights); a chain of such launches on one stream reaches the highest weight
+ * bandwidth with bitlinear_gemv_fused_multi and BL_FLAG_PDL inside a CUDA
+ * graph.  Other shapes run a kernel with a per-warp weight ring.  Results are
+ * identical either way.
  */
 int bitlinear_gemv_fused(const uint8_t *packed, const float *w_scale,
                          int64_t N, int64_t K, const void *x, int xt,
