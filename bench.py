@@ -23,7 +23,11 @@ Metric: effective weight bandwidth, packed weight bytes / device time, GB/s,
 against the measured HBM copy bandwidth.  Inputs are synthetic and seeded
 (weights N(0, 0.02^2) absmean-packed; x ~ N(0, 1) with 0.1% x20 outliers,
 bf16).  With N GPUs every rank runs its own independent decode stream (no
-collective), so the scaling is weak and the value is the sum over ranks.
+collective), so the scaling is weak and the value is the sum over ranks.  With
+--split the ranks share one model instead: every product is split by output
+rows (whole 8-row groups of the packed weight per rank), each launch is
+followed by an all-gather of its outputs, and the value is the one model's
+weight bytes per step over the slowest rank's time (strong scaling).
 
 The reference arm (--impl reference) times the CPU oracle on the host cores on
 a bounded sample of the same workload.  Extra measurements (the isolated layer
@@ -247,6 +251,53 @@ def build_stream(bl, layers: int, seed: int, device):
 def run_step(bl, launches, pdl=True):
     for (ws, x, ys) in launches:
         bl.gemv_fused_multi(ws, x, outs=ys, pdl=pdl)
+
+
+def build_split_stream(bl, layers: int, seed: int, device):
+    """The decode stream split by output rows over the ranks (column-parallel):
+    every rank packs the same model (same seeds), keeps the shard of whole
+    8-row groups it owns of every weight, runs its shards of each launch and
+    all-gathers the outputs, so each launch's full output is on every rank
+    before the next one reads it.  Returns the per-launch ColumnParallelDecode
+    objects with their inputs, the token input, the final output, the host
+    token and the packed bytes per step that this rank streams and that the
+    whole job streams."""
+    from bit_ternary_weight_b200.sharding import ColumnParallelDecode
+    shapes = {name: (K, N) for (name, K, N) in si.LAYER_SHAPES_2B}
+    gen = torch.Generator(device=device)
+    x0 = torch.empty(1, si.HIDDEN_2B, dtype=torch.bfloat16, device=device)
+    chain = []
+    h = x0
+    rank_bytes = total_bytes = 0
+    for layer in range(layers):
+        cpds = []
+        for li, (lname, names) in enumerate(LAYER_LAUNCHES_2B):
+            ws = []
+            for j, name in enumerate(names):
+                K, N = shapes[name]
+                gen.manual_seed(seed * 100003 + layer * 31 + li * 7 + j)
+                W = torch.randn(N, K, generator=gen, device=device, dtype=torch.float32) * 0.02
+                ws.append(bl.pack(W))
+                del W
+                total_bytes += ws[-1].packed.numel()
+            cpd = ColumnParallelDecode(ws, device=device)
+            rank_bytes += sum(sw.packed.numel() for (_, _, sw) in cpd.shards if sw is not None)
+            cpds.append(cpd)
+        qkv, o_proj, gate_up, down = cpds
+        chain.append((qkv, h))
+        chain.append((o_proj, qkv.outputs()[0]))
+        chain.append((gate_up, o_proj.outputs()[0]))
+        chain.append((down, gate_up.outputs()[0]))
+        h = down.outputs()[0]
+    host_x0 = si.activations(1, si.HIDDEN_2B, seed=seed)
+    x0.copy_(host_x0)
+    torch.cuda.synchronize()
+    return chain, x0, h, host_x0, rank_bytes, total_bytes
+
+
+def run_split_step(chain, pdl=True):
+    for cpd, x in chain:
+        cpd(x, pdl=pdl)
 
 
 def time_graph(graph, steps, world):
@@ -477,16 +528,24 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", torch.cuda.current_device())
     hbm, bf16, bf16_sus, peak_kind = peaks()
 
-    launches, xs, ys, host_x, step_bytes = build_stream(bl, args.layers, seed=rank, device=device)
+    if args.split:
+        # one model split over the ranks: every rank builds it from the same seed
+        launches, xs, ys, host_x, rank_bytes, step_bytes = build_split_stream(
+            bl, args.layers, seed=0, device=device)
+        step = lambda: run_split_step(launches)  # noqa: E731
+    else:
+        launches, xs, ys, host_x, step_bytes = build_stream(bl, args.layers, seed=rank, device=device)
+        rank_bytes = step_bytes
+        step = lambda: run_step(bl, launches)  # noqa: E731
     # xs: the token's input (copied in every e2e step); ys: its final output
     launches_per_step = len(launches)
     # eager warm-up through the public API, then capture the step
     for _ in range(2):
-        run_step(bl, launches)
+        step()
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        run_step(bl, launches)
+        step()
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
@@ -495,7 +554,10 @@ def run_ours(args, world, rank, local):
         t = time_graph(graph, args.steps, world)
     clocks = clk.summary()
     t = max_over_ranks(t, world)
-    value = job_throughput(step_bytes, args.steps, world, t)
+    # replicas: every rank streams a whole model per step (weak scaling);
+    # split: the ranks stream one model between them (strong scaling)
+    job_ranks = 1 if args.split else world
+    value = job_throughput(step_bytes, args.steps, job_ranks, t)
     ms_per_step = t / args.steps * 1000
 
     # e2e: host activations in, host outputs back, every step, through the same
@@ -517,7 +579,7 @@ def run_ours(args, world, rank, local):
     e.record()
     torch.cuda.synchronize()
     t_e2e = max_over_ranks(s.elapsed_time(e) / 1000.0, world)
-    e2e_value = job_throughput(step_bytes, args.steps, world, t_e2e)
+    e2e_value = job_throughput(step_bytes, args.steps, job_ranks, t_e2e)
 
     # eager (no graph) public-API loop, for context
     torch.cuda.synchronize()
@@ -526,7 +588,7 @@ def run_ours(args, world, rank, local):
     s.record()
     for _ in range(eager_steps):
         xs.copy_(pin_x, non_blocking=True)
-        run_step(bl, launches)
+        step()
         pin_y.copy_(ys, non_blocking=True)
     e.record()
     torch.cuda.synchronize()
@@ -534,7 +596,7 @@ def run_ours(args, world, rank, local):
     del graph
 
     extra = {}
-    if rank == 0 and not args.no_extra:
+    if rank == 0 and not args.no_extra and not args.split:
         def measure(key, fn):
             try:
                 extra[key] = fn()
@@ -561,15 +623,21 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong" if args.split else "weak",
+        "vs_baseline": None,
         "dtype": "int8", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) bf16 x with 0.1% x20 outliers)",
         "config": {"workload": WORKLOAD, "layers": args.layers,
                    "launches_per_step": launches_per_step,
                    "weight_bytes_per_step": step_bytes,
+                   "weight_bytes_per_step_per_rank": rank_bytes,
                    "l2": "inputs larger than L2: 521 MB of distinct packed weights per step",
-                   "parallelism": f"{world} independent replicas (weak scaling)"},
-        "roofline": {"bound": "hbm", "achieved": value / world, "peak": hbm, "unit": "GB/s",
-                     "frac": value / world / hbm, "traffic": profiled_traffic(),
+                   "parallelism": (f"N-split over {world} ranks (each launch's output rows "
+                                   "split in whole 8-row groups, all-gather of y after every "
+                                   "launch)") if args.split else
+                                  f"{world} independent replicas (weak scaling)"},
+        "roofline": {"bound": "hbm", "achieved": rank_bytes * args.steps / t / 1e9, "peak": hbm,
+                     "unit": "GB/s", "frac": rank_bytes * args.steps / t / 1e9 / hbm,
+                     "traffic": profiled_traffic(),
                      "peak_kind": f"{peak_kind} HBM copy bandwidth",
                      "kernel": "gemv_stream_kernel<KC=8, bf16 fused> (4 launches per layer)",
                      "note": "algorithmic bytes = packed weight bytes per launch; duration = "
@@ -644,6 +712,10 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=2.0)
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split", action="store_true",
+                    help="split one model's products by output rows over the ranks "
+                         "(column-parallel, all-gather of y per launch) instead of "
+                         "running independent replicas")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

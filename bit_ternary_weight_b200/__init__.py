@@ -22,6 +22,7 @@ Pages the operations follow (title, section):
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from dataclasses import dataclass
@@ -118,6 +119,14 @@ def _stream(device: torch.device):
     return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
 
 
+def _on(device: torch.device):
+    """Make the tensors' GPU current for the call: the library launches on the
+    current device and rejects memory of any other GPU."""
+    if device.type == "cuda":
+        return torch.cuda.device(device)
+    return contextlib.nullcontext()
+
+
 @dataclass
 class TernaryWeight:
     """A packed ternary weight: TL bytes, the fp32 gamma_eff and the shape."""
@@ -150,8 +159,9 @@ def pack(W: torch.Tensor) -> TernaryWeight:
     w_scale = torch.empty(1, dtype=torch.float32, device=W.device)
     ws_bytes = int(_lib.bitlinear_pack_workspace_bytes(N, K))
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=W.device)
-    _check(_lib.bitlinear_pack(_ptr(W), _dt(W.dtype), N, K, _ptr(packed), _ptr(w_scale),
-                               _ptr(ws), ws.numel(), _stream(W.device)), "bitlinear_pack")
+    with _on(W.device):
+        _check(_lib.bitlinear_pack(_ptr(W), _dt(W.dtype), N, K, _ptr(packed), _ptr(w_scale),
+                                   _ptr(ws), ws.numel(), _stream(W.device)), "bitlinear_pack")
     return TernaryWeight(packed, w_scale, N, K)
 
 
@@ -164,9 +174,10 @@ def pack_noalloc(W: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor) -
     not exceed PACK_NOALLOC_MAX_ROWS).  For callers that cannot allocate
     device memory when they pack; this function allocates nothing either."""
     N, K = W.shape
-    _check(_lib.bitlinear_pack_noalloc(_ptr(W), _dt(W.dtype), N, K, _ptr(packed),
-                                       _ptr(w_scale), _stream(W.device)),
-           "bitlinear_pack_noalloc")
+    with _on(W.device):
+        _check(_lib.bitlinear_pack_noalloc(_ptr(W), _dt(W.dtype), N, K, _ptr(packed),
+                                           _ptr(w_scale), _stream(W.device)),
+               "bitlinear_pack_noalloc")
     return TernaryWeight(packed, w_scale, N, K)
 
 
@@ -182,9 +193,10 @@ def quantize_act(x: torch.Tensor, out=None):
         r = torch.empty(M, dtype=torch.int32, device=x.device)
     else:
         q, d, r = out
-    _check(_lib.bitlinear_quantize_act(_ptr(x), _dt(x.dtype), M, K, x.stride(0), _ptr(q),
-                                       _ptr(d), _ptr(r), _stream(x.device)),
-           "bitlinear_quantize_act")
+    with _on(x.device):
+        _check(_lib.bitlinear_quantize_act(_ptr(x), _dt(x.dtype), M, K, x.stride(0), _ptr(q),
+                                           _ptr(d), _ptr(r), _stream(x.device)),
+               "bitlinear_quantize_act")
     return q, d, r
 
 
@@ -198,9 +210,10 @@ def gemv(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc
     """Decode GEMV (1 <= M <= 16) on pre-quantised activations."""
     M = q.shape[0]
     out = _out(M, w.N, out_dtype, q.device, out)
-    _check(_lib.bitlinear_gemv(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q), _ptr(d),
-                               _ptr(rowsum), M, _ptr(out), _dt(out.dtype), out.stride(0),
-                               _ptr(acc_dbg), _stream(q.device)), "bitlinear_gemv")
+    with _on(q.device):
+        _check(_lib.bitlinear_gemv(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q), _ptr(d),
+                                   _ptr(rowsum), M, _ptr(out), _dt(out.dtype), out.stride(0),
+                                   _ptr(acc_dbg), _stream(q.device)), "bitlinear_gemv")
     return out
 
 
@@ -211,10 +224,11 @@ def gemv_fused(w: TernaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16, out=
         x = x.unsqueeze(0)
     M = x.shape[0]
     out = _out(M, w.N, out_dtype, x.device, out)
-    _check(_lib.bitlinear_gemv_fused(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(x),
-                                     _dt(x.dtype), x.stride(0), M, _ptr(out), _dt(out.dtype),
-                                     out.stride(0), _ptr(acc_dbg), _stream(x.device)),
-           "bitlinear_gemv_fused")
+    with _on(x.device):
+        _check(_lib.bitlinear_gemv_fused(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(x),
+                                         _dt(x.dtype), x.stride(0), M, _ptr(out), _dt(out.dtype),
+                                         out.stride(0), _ptr(acc_dbg), _stream(x.device)),
+               "bitlinear_gemv_fused")
     return out
 
 
@@ -244,10 +258,11 @@ def gemv_fused_multi(weights, x: torch.Tensor, out_dtype=torch.bfloat16, outs=No
     ys = P(*[o.data_ptr() for o in outs])
     ldys = I64(*[o.stride(0) for o in outs])
     accs = None if acc_dbgs is None else P(*[0 if a is None else a.data_ptr() for a in acc_dbgs])
-    _check(_lib.bitlinear_gemv_fused_multi(n, packed, scales, Ns, weights[0].K, _ptr(x),
-                                           _dt(x.dtype), x.stride(0), M, ys, _dt(outs[0].dtype),
-                                           ldys, accs, BL_FLAG_PDL if pdl else 0,
-                                           _stream(x.device)), "bitlinear_gemv_fused_multi")
+    with _on(x.device):
+        _check(_lib.bitlinear_gemv_fused_multi(n, packed, scales, Ns, weights[0].K, _ptr(x),
+                                               _dt(x.dtype), x.stride(0), M, ys, _dt(outs[0].dtype),
+                                               ldys, accs, BL_FLAG_PDL if pdl else 0,
+                                               _stream(x.device)), "bitlinear_gemv_fused_multi")
     return outs
 
 
@@ -265,10 +280,11 @@ def gemm(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc
         # zero before its first use; every call leaves it zero again
         workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(_lib.bitlinear_gemm(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q), _ptr(d),
-                               _ptr(rowsum), M, _ptr(out), _dt(out.dtype), out.stride(0),
-                               _ptr(acc_dbg), _ptr(workspace), ws_bytes, _stream(q.device)),
-           "bitlinear_gemm")
+    with _on(q.device):
+        _check(_lib.bitlinear_gemm(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q), _ptr(d),
+                                   _ptr(rowsum), M, _ptr(out), _dt(out.dtype), out.stride(0),
+                                   _ptr(acc_dbg), _ptr(workspace), ws_bytes, _stream(q.device)),
+               "bitlinear_gemm")
     return out
 
 
@@ -295,8 +311,9 @@ def binary_pack(W: torch.Tensor) -> BinaryWeight:
         raise BitLinearError(BL_ERR_SHAPE, "binary_pack")
     bits = torch.empty(N, K // 64, dtype=torch.int64, device=W.device)
     s_w = torch.empty(1, dtype=torch.float32, device=W.device)
-    _check(_lib.bitlinear_binary_pack(_ptr(W), _dt(W.dtype), N, K, _ptr(bits), _ptr(s_w),
-                                      _stream(W.device)), "bitlinear_binary_pack")
+    with _on(W.device):
+        _check(_lib.bitlinear_binary_pack(_ptr(W), _dt(W.dtype), N, K, _ptr(bits), _ptr(s_w),
+                                          _stream(W.device)), "bitlinear_binary_pack")
     return BinaryWeight(bits, s_w, N, K)
 
 
@@ -305,9 +322,10 @@ def binary_gemv(w: BinaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16, out=
     x = x.reshape(-1)
     if out is None:
         out = torch.empty(w.N, dtype=out_dtype, device=x.device)
-    _check(_lib.bitlinear_binary_gemv(_ptr(w.bits), _ptr(w.s_w), w.N, w.K, _ptr(x),
-                                      _dt(x.dtype), _ptr(out), _dt(out.dtype), _ptr(acc_dbg),
-                                      _stream(x.device)), "bitlinear_binary_gemv")
+    with _on(x.device):
+        _check(_lib.bitlinear_binary_gemv(_ptr(w.bits), _ptr(w.s_w), w.N, w.K, _ptr(x),
+                                          _dt(x.dtype), _ptr(out), _dt(out.dtype), _ptr(acc_dbg),
+                                          _stream(x.device)), "bitlinear_binary_gemv")
     return out
 
 

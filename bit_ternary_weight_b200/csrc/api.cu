@@ -27,6 +27,14 @@ thread_local char g_cuda_err[256] = "";
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+bool valid_dtype(int t) { return t == BL_F32 || t == BL_BF16; }
+int elem_bytes(int t) { return t == BL_BF16 ? 2 : 4; }
+
+}  // namespace
+
+// Device (or managed) memory that belongs to the current device.  Memory of
+// another GPU is rejected too: the kernels launch on the current device, and a
+// pointer into a peer's memory would be dereferenced there.
 bool is_device_ptr(const void *p)
 {
     cudaPointerAttributes attr;
@@ -35,11 +43,17 @@ bool is_device_ptr(const void *p)
         cudaGetLastError();
         return false;
     }
-    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+    if (attr.type == cudaMemoryTypeManaged)
+        return true;
+    if (attr.type != cudaMemoryTypeDevice)
+        return false;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return attr.device == dev;
 }
-
-bool valid_dtype(int t) { return t == BL_F32 || t == BL_BF16; }
-int elem_bytes(int t) { return t == BL_BF16 ? 2 : 4; }
 
 // Common shape rule: N >= 1, K >= 64, K % 64 == 0, and sizes that keep every
 // index inside int32 tiles and int64 byte offsets comfortably.
@@ -50,12 +64,14 @@ bool valid_nk(int64_t N, int64_t K)
 }
 
 // Device presence and architecture; returns BL_OK and the info, or an error.
+// The library is built for sm_100a only, whose code runs on compute
+// capability 10.0 alone.
 int need_device(const DeviceInfo **out)
 {
     const DeviceInfo *di = device_info();
     if (!di)
         return BL_ERR_CUDA;
-    if (di->cc_major != 10)
+    if (di->cc_major != 10 || di->cc_minor != 0)
         return BL_ERR_UNSUPPORTED;
     *out = di;
     return BL_OK;
@@ -68,8 +84,6 @@ int check_dev_ptrs(std::initializer_list<const void *> ptrs)
             return BL_ERR_NOT_DEVICE_PTR;
     return BL_OK;
 }
-
-}  // namespace
 
 const DeviceInfo *device_info()
 {
@@ -166,11 +180,11 @@ const char *bitlinear_status_string(int status)
     case BL_ERR_DTYPE: return "BL_ERR_DTYPE: unsupported element type";
     case BL_ERR_SHAPE: return "BL_ERR_SHAPE: shape or stride out of range";
     case BL_ERR_ALIGN: return "BL_ERR_ALIGN: pointer or stride not 16-byte aligned";
-    case BL_ERR_NOT_DEVICE_PTR: return "BL_ERR_NOT_DEVICE_PTR: host pointer where device memory is required";
+    case BL_ERR_NOT_DEVICE_PTR: return "BL_ERR_NOT_DEVICE_PTR: host memory or another GPU's memory where memory of the current device is required";
     case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE: workspace missing or too small";
     case BL_ERR_CUDA: return "BL_ERR_CUDA: CUDA runtime error";
     case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT: a device-side bounded wait ran out";
-    case BL_ERR_UNSUPPORTED: return "BL_ERR_UNSUPPORTED: needs an sm_100 (B200) device";
+    case BL_ERR_UNSUPPORTED: return "BL_ERR_UNSUPPORTED: needs a compute capability 10.0 (B200, sm_100a) device";
     default: return "unknown status";
     }
 }

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <initializer_list>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -20,6 +21,22 @@ struct DeviceInfo {
 
 // Properties of the current device (cached per device).  nullptr on error.
 const DeviceInfo *device_info();
+
+// --- argument checks shared by every entry point -------------------------
+
+// Device (or managed) memory of the current device.
+bool is_device_ptr(const void *p);
+
+// N >= 1, K >= 64, K % 64 == 0, within the index ranges the kernels use.
+bool valid_nk(int64_t N, int64_t K);
+
+// A compute capability 10.0 device is current: BL_OK and its info, else
+// BL_ERR_CUDA / BL_ERR_UNSUPPORTED.
+int need_device(const DeviceInfo **out);
+
+// BL_ERR_NOT_DEVICE_PTR if any non-NULL pointer is not device memory of the
+// current device, else BL_OK.
+int check_dev_ptrs(std::initializer_list<const void *> ptrs);
 
 // Records `e` as the last CUDA error of this thread and returns BL_ERR_CUDA,
 // or BL_OK when e == cudaSuccess.

@@ -169,16 +169,6 @@ int scratch_address(double **out)
     return BL_OK;
 }
 
-bool device_pointer(const void *p)
-{
-    cudaPointerAttributes attr;
-    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
-        cudaGetLastError();
-        return false;
-    }
-    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
-}
-
 }  // namespace
 
 }  // namespace bl
@@ -191,20 +181,19 @@ extern "C" int bitlinear_pack_noalloc(const void *W, int wt, int64_t N, int64_t 
         return BL_ERR_NULL;
     if (wt != BL_F32 && wt != BL_BF16)
         return BL_ERR_DTYPE;
-    if (N < 1 || K < 64 || K % 64 != 0 || K > (int64_t(1) << 22) || N > kNoAllocMaxRows)
+    if (!valid_nk(N, K) || N > kNoAllocMaxRows)
         return BL_ERR_SHAPE;
     if ((reinterpret_cast<uintptr_t>(W) & 15u) || (reinterpret_cast<uintptr_t>(packed) & 15u) ||
         (reinterpret_cast<uintptr_t>(w_scale) & 3u))
         return BL_ERR_ALIGN;
-    const DeviceInfo *di = device_info();
-    if (!di)
-        return BL_ERR_CUDA;
-    if (di->cc_major != 10)
-        return BL_ERR_UNSUPPORTED;
-    if (!device_pointer(W) || !device_pointer(packed) || !device_pointer(w_scale))
-        return BL_ERR_NOT_DEVICE_PTR;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({W, packed, w_scale})))
+        return st;
     double *scratch = nullptr;
-    int st = scratch_address(&scratch);
+    st = scratch_address(&scratch);
     if (st)
         return st;
     return launch_pack(W, wt, N, K, packed, w_scale, scratch, static_cast<cudaStream_t>(stream));

@@ -43,8 +43,12 @@
  *
  * Conventions for every entry point:
  *   - Pointers named as device pointers must be device (or managed) memory of
- *     the current device; a host pointer gives BL_ERR_NOT_DEVICE_PTR.  There
- *     is no CPU fallback.
+ *     the current device; a host pointer, or memory that belongs to another
+ *     GPU, gives BL_ERR_NOT_DEVICE_PTR.  Kernels launch on the current device,
+ *     so a caller with tensors on another GPU makes that GPU current first.
+ *     There is no CPU fallback.
+ *   - The library runs on compute capability 10.0 (B200, sm_100a) only; any
+ *     other current device gives BL_ERR_UNSUPPORTED.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Every call is asynchronous on it; the caller owns all memory
  *     and keeps it alive until the stream has passed the call.
@@ -75,11 +79,11 @@ typedef enum {
     BL_ERR_DTYPE = 2,           /* unsupported element type */
     BL_ERR_SHAPE = 3,           /* N, K, M, strides out of range */
     BL_ERR_ALIGN = 4,           /* pointer or stride misaligned */
-    BL_ERR_NOT_DEVICE_PTR = 5,  /* a device pointer is host memory */
+    BL_ERR_NOT_DEVICE_PTR = 5,  /* a device pointer is host or another GPU's memory */
     BL_ERR_WORKSPACE = 6,       /* workspace missing or too small */
     BL_ERR_CUDA = 7,            /* CUDA runtime error */
     BL_ERR_TIMEOUT = 8,         /* a device-side bounded wait ran out */
-    BL_ERR_UNSUPPORTED = 9      /* no sm_100 device */
+    BL_ERR_UNSUPPORTED = 9      /* the current device is not compute capability 10.0 */
 } bl_status;
 
 typedef enum { BL_F32 = 0, BL_BF16 = 1 } bl_dtype;
@@ -237,9 +241,13 @@ size_t bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * ternary product).  Arguments as for bitlinear_gemv, plus
  *   ws, ws_bytes   device workspace, at least bitlinear_gemm_workspace_bytes
  *                  (may be NULL when that is 0).  It must be all zero before
- *                  its first use, and every call leaves it zero; it may be
- *                  reused by calls that are ordered on one stream, not shared
- *                  by calls that can run at the same time.
+ *                  its first use, and every call that completes leaves it
+ *                  zero; it may be reused by calls that are ordered on one
+ *                  stream, not shared by calls that can run at the same time.
+ *                  A call whose bounded wait ran out (the next
+ *                  bitlinear_last_device_status() returns BL_ERR_TIMEOUT) may
+ *                  leave partial sums and arrival counts in it: zero it again
+ *                  before the next call that uses it.
  * q must be 16-byte aligned and K % 64 == 0.
  */
 int bitlinear_gemm(const uint8_t *packed, const float *w_scale, int64_t N,

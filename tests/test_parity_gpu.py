@@ -371,12 +371,49 @@ def test_gemm_split_k_small_batches(bl, M, N, K):
         assert int(torch.count_nonzero(ws)) == 0
 
 
+def _tile_sample(M: int, seed: int, per_tile: int = 2) -> np.ndarray:
+    """Token rows to check at full size: both edges of every 128-token tile
+    boundary plus `per_tile` random tokens inside every tile, so that every
+    (weight-row tile, token tile) pair of the persistent walk -- each CTA's
+    first and last tile, and both accumulator buffers -- has checked outputs."""
+    rng = np.random.default_rng(seed)
+    rows = [0, M - 1]
+    for t0 in range(0, M, 128):
+        t1 = min(M, t0 + 128)
+        rows += [t0, t1 - 1]
+        rows += list(rng.integers(t0, t1, per_tile))
+    return np.unique(np.asarray(rows, dtype=np.int64))
+
+
 @pytest.mark.parametrize("K,N", si.PREFILL_SHAPES)
 @pytest.mark.parametrize("M", si.PREFILL_TOKENS)
 def test_gemm_prefill_full_size(bl, K, N, M):
-    rng = np.random.default_rng(M + K)
-    sample = np.unique(np.concatenate([[0, M - 1, 127, 128], rng.integers(0, M, 60)]))
-    _check_gemm(bl, N, K, M, seed=3, sample=sample)
+    """Every output column of tokens drawn from every 128-token tile."""
+    _check_gemm(bl, N, K, M, seed=3, sample=_tile_sample(M, M + K))
+
+
+def test_gemm_prefill_every_output_m2048(bl):
+    """Prefill 2048 tokens x (2560 -> 6912): every one of the 14.2 M outputs
+    and int32 accumulators against the oracle (several tiles per CTA, both
+    accumulator buffers, every ring wrap)."""
+    _check_gemm(bl, 6912, 2560, 2048, seed=5)
+
+
+def test_other_gpus_memory_rejected(bl):
+    """A tensor on another GPU while cuda:0 is current: rejected before any
+    launch (the raw C ABI, which does not switch devices)."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two GPUs")
+    import ctypes
+    w = _pack_gpu(bl, si.weight(16, 64))
+    x1 = torch.zeros(1, 64, dtype=torch.bfloat16, device="cuda:1")
+    y0 = torch.empty(1, 16, dtype=torch.bfloat16, device=dev())
+    with torch.cuda.device(0):
+        st = bl.lib.bitlinear_gemv_fused(
+            ctypes.c_void_p(w.packed.data_ptr()), ctypes.c_void_p(w.w_scale.data_ptr()), 16, 64,
+            ctypes.c_void_p(x1.data_ptr()), bl.BL_BF16, 64, 1, ctypes.c_void_p(y0.data_ptr()),
+            bl.BL_BF16, 16, None, None)
+    assert st == bl.BL_ERR_NOT_DEVICE_PTR
 
 
 # ------------------------------------------------------------------ shared-input multi GEMV, PDL chains
@@ -431,3 +468,44 @@ def test_pdl_dependent_chain(bl, K, M):
         compare_outputs(xs[i + 1], y_o)
         x = torch.from_numpy(oracle.to_bf16_bits(y_o).view(np.int16)).view(torch.bfloat16)
     assert bl.last_device_status() == 0
+
+
+# ------------------------------------------------------------------ N-split (column-parallel) shards
+
+@pytest.mark.parametrize("world,M", [(2, 1), (3, 1), (4, 1), (3, 3)])
+def test_row_split_shards_equal_unsplit(bl, world, M):
+    """Each rank's shard (a view of whole 8-row groups of the packed weight,
+    the whole tensor's gamma) run through the fused multi-product GEMV into
+    its slot of a gather buffer: the slots, laid end to end, are the unsplit
+    outputs bit for bit.  All ranks are emulated on this one GPU, one after
+    another; no rank waits on another."""
+    from bit_ternary_weight_b200.sharding import row_partition, shard_weight
+    K = si.HIDDEN_2B
+    Ns = [si.HIDDEN_2B, si.KV_2B, 1001]
+    x = si.activations(M, K, seed=600 + world)
+    xd = x.to(dev())
+    ws, refs = [], []
+    for i, N in enumerate(Ns):
+        W = si.weight(N, K, seed=610 + i)
+        g, codes, _ = oracle_weight(W)
+        refs.append(_oracle_gemv(g, codes, x)[0])
+        ws.append(_pack_gpu(bl, W))
+    parts = [row_partition(N, world) for N in Ns]
+    bufs = [torch.full((world * M * p[0].rows_per_rank,), float("nan"), dtype=torch.bfloat16,
+                       device=dev()) for p in parts]
+    for r in range(world):
+        live = []
+        for w, p, buf in zip(ws, parts, bufs):
+            sh = p[r]
+            sw = shard_weight(w, sh)
+            if sw is None:
+                continue
+            slot = buf[r * M * sh.rows_per_rank:(r + 1) * M * sh.rows_per_rank]
+            live.append((sw, slot.view(M, sh.rows_per_rank)[:, :sh.rows]))
+        if live:
+            bl.gemv_fused_multi([a for a, _ in live], xd, outs=[b for _, b in live])
+    torch.cuda.synchronize()
+    for N, p, buf, y_o in zip(Ns, parts, bufs, refs):
+        R = p[0].rows_per_rank
+        full = buf.view(world, M, R).permute(1, 0, 2).reshape(M, world * R)[:, :N]
+        compare_outputs(full, y_o)
