@@ -61,6 +61,7 @@ def _load():
             "oracle_pack": (None, [vp, i64, i64, vp]),
             "oracle_unpack": (None, [vp, i64, i64, vp]),
             "oracle_quantize_act": (None, [vp, i64, i64, vp, vp, vp]),
+            "oracle_rmsnorm": (None, [vp, i64, i64, vp, f32, vp]),
             "oracle_ternary_acc": (None, [vp, vp, i64, i64, i64, vp]),
             "oracle_rescale": (None, [vp, vp, f32, i64, i64, vp]),
             "oracle_to_bf16": (None, [vp, i64, vp]),
@@ -142,6 +143,29 @@ def quantize_act(x: np.ndarray):
     r = np.empty(M, np.int32)
     _load().oracle_quantize_act(_p(x), M, K, _p(q), _p(d), _p(r))
     return q, d, r
+
+
+RMS_EPS = 1e-5  # the reading's default epsilon
+
+
+def rmsnorm(x: np.ndarray, gain=None, eps: float = RMS_EPS) -> np.ndarray:
+    """h = (x * r) * gain with r = 1 / sqrt(mean(x^2) + eps): the mean square
+    summed in fp64 and rounded once to fp32, everything after it in fp32
+    (correctly rounded square root and division).  fp32 [M, K]."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    h = np.empty((M, K), np.float32)
+    g = None if gain is None else _c(np.asarray(gain).reshape(-1), np.float32)
+    if g is not None and g.size != K:
+        raise ValueError("gain must have K elements")
+    _load().oracle_rmsnorm(_p(x), M, K, None if g is None else _p(g),
+                           float(np.float32(eps)), _p(h))
+    return h
+
+
+def rmsnorm_quantize_act(x: np.ndarray, gain=None, eps: float = RMS_EPS):
+    """RMSNorm, then per-token absmax int8: (q, d, rowsum) of the normalised rows."""
+    return quantize_act(rmsnorm(x, gain, eps))
 
 
 def ternary_acc(codes: np.ndarray, q: np.ndarray) -> np.ndarray:

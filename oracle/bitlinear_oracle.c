@@ -175,6 +175,38 @@ void oracle_quantize_act(const float *x, int64_t M, int64_t K, int8_t *q,
 }
 
 /* ---------------------------------------------------------------------------
+ * RMSNorm in front of the activation quantiser.  [FLOOR] "What's inside"
+ * (rmsnorm.cu: a mean-square reduction over the row, an rsqrt scale applied
+ * element by element) and [GUIDE] "Understanding the Two-Phase Architecture"
+ * (the Attention and FeedForward layers feed their inputs to BitLinear).
+ * The pages give no formula; the reading here, per token m:
+ *   S     = sum_k (double)x[k] * (double)x[k]     fp64, k ascending
+ *   ms    = (float)(S / (double)K)                rounded once to fp32
+ *   r     = 1.0f / sqrtf(ms + eps)                fp32 add, correctly rounded
+ *                                                 square root and division
+ *   h[k]  = (x[k] * r) * g[k]                     two fp32 products, in that
+ *                                                 order (g = 1 without a gain)
+ * h stays fp32 and goes straight to oracle_quantize_act.
+ * ------------------------------------------------------------------------- */
+void oracle_rmsnorm(const float *x, int64_t M, int64_t K, const float *gain,
+                    float eps, float *h)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        const float *xm = x + m * K;
+        double S = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+            S += (double)xm[k] * (double)xm[k];
+        float ms = (float)(S / (double)K);
+        float den = sqrtf(ms + eps);
+        float r = 1.0f / den;
+        for (int64_t k = 0; k < K; ++k) {
+            float t = xm[k] * r;
+            h[m * K + k] = gain ? t * gain[k] : t;
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------
  * Ternary product with exact integer accumulation.  [BITC] "Features": a
  * product with -1 / 0 / +1 is subtract / skip / add.  [GUIDE] FAQ: an
  * INT8 x INT2 GEMM.  Accumulated in int64 and narrowed (|acc| <= 128 * K).

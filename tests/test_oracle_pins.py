@@ -288,3 +288,70 @@ def test_binary_bit_order():
     b = oracle.binary_signs(v)
     assert b.shape == (1, 2)
     assert int(b[0, 0]) == 1 << 3 and int(b[0, 1]) == 1 << 60
+
+
+# ---------------------------------------------------------------- RMSNorm
+
+def test_rmsnorm_hand_worked(golden):
+    g = golden("rmsnorm_hand.json")
+    x = _f32(g["x"])
+    h = oracle.rmsnorm(x, eps=g["eps"])
+    np.testing.assert_array_equal(h, _f32(g["h_no_gain"]))
+    h = oracle.rmsnorm(x, gain=_f32(g["gain"]), eps=g["eps"])
+    np.testing.assert_array_equal(h, _f32(g["h_gain"]))
+
+
+@pytest.mark.parametrize("c", [1.0, -2.0, 0.25, 64.0, -1024.0])
+def test_rmsnorm_constant_row_gives_the_gain(c):
+    # x = c everywhere: mean square c^2, root |c| (exact for powers of two),
+    # r = 1/|c| exact, so h = sign(c) * gain exactly when eps = 0
+    K = 64
+    gain = np.linspace(-3.0, 3.0, K, dtype=np.float32)
+    h = oracle.rmsnorm(np.full((1, K), c, np.float32), gain=gain, eps=0.0)
+    np.testing.assert_array_equal(h[0], np.sign(c) * gain)
+
+
+def test_rmsnorm_power_of_two_scale_invariance():
+    x = si.activations(3, 512, seed=4, dtype=torch.float32).numpy()
+    gain = 1.0 + 0.1 * si.activations(1, 512, seed=5, outliers=False, dtype=torch.float32).numpy()
+    h = oracle.rmsnorm(x, gain=gain, eps=0.0)
+    for a in (2.0, 0.125, -8.0):
+        np.testing.assert_array_equal(oracle.rmsnorm(x * np.float32(a), gain=gain, eps=0.0),
+                                      np.sign(a) * h)
+
+
+@pytest.mark.parametrize("eps", [0.0, 1e-5, 1e-2])
+@pytest.mark.parametrize("scale", [1.0, 1e-3])
+def test_rmsnorm_against_fp64_definition(eps, scale):
+    # textbook RMSNorm in fp64 (numpy); the fp32 chain (mean rounded to fp32,
+    # eps added in fp32, sqrt, divide, two products) stays within a few ulp
+    M, K = 4, 2560
+    x = (si.activations(M, K, seed=7, dtype=torch.float32).numpy() * np.float32(scale))
+    gain = 1.0 + 0.2 * si.activations(1, K, seed=8, outliers=False, dtype=torch.float32).numpy()[0]
+    h = oracle.rmsnorm(x, gain=gain, eps=eps).astype(np.float64)
+    x64 = x.astype(np.float64)
+    ms = (x64 * x64).mean(axis=1, keepdims=True)
+    want = x64 / np.sqrt(ms + eps) * gain.astype(np.float64)
+    ulp = np.spacing(np.abs(want).astype(np.float32)).astype(np.float64)
+    assert np.all(np.abs(h - want) <= 4 * ulp + 1e-30)
+
+
+def test_rmsnorm_eps_dominates_a_tiny_row():
+    # mean square 1e-8 << eps = 1e-5: h = x / sqrt(1.001e-5), about 0.0316,
+    # not 1 (as it would be without eps)
+    x = np.full((1, 256), 1e-4, np.float32)
+    h = oracle.rmsnorm(x, eps=1e-5)
+    assert h[0, 0] == pytest.approx(1e-4 / math.sqrt(1e-8 + 1e-5), rel=1e-6)
+
+
+def test_rmsnorm_zero_row_and_quantiser():
+    x = np.zeros((2, 128), np.float32)
+    x[1, 5] = 3.0
+    h = oracle.rmsnorm(x)
+    assert not h[0].any()
+    q, d, r = oracle.rmsnorm_quantize_act(x)
+    assert not q[0].any() and r[0] == 0
+    # a one-hot row normalises to 3 / sqrt(9/K + eps) (sqrt(K) without eps) at
+    # its position, which quantises to 127
+    assert h[1, 5] == pytest.approx(3.0 / math.sqrt(9.0 / 128 + 1e-5), rel=1e-6)
+    assert q[1, 5] == 127 and r[1] == 127
