@@ -69,6 +69,8 @@ def _load():
             "oracle_binary_signs": (None, [vp, i64, i64, ctypes.c_int, vp]),
             "oracle_binary_acc": (None, [vp, vp, i64, i64, vp]),
             "oracle_binary_rescale": (None, [vp, f32, f32, i64, vp]),
+            "oracle_bitplanes": (None, [vp, i64, i64, vp, vp]),
+            "oracle_bitplane_acc": (None, [vp, vp, vp, i64, i64, vp]),
             "oracle_num_threads": (ctypes.c_int, []),
         }
         for name, (res, args) in sig.items():
@@ -262,3 +264,43 @@ def binary_gemv(W: np.ndarray, x: np.ndarray):
     acc = binary_acc(Wb, xb, K)
     return {"Wb": Wb, "xb": xb, "s_w": s_w, "s_x": s_x, "acc": acc,
             "y": binary_rescale(acc, s_w, s_x)}
+
+
+# --------------------------------------------------------------------------
+# ternary weights x 1-bit activations (two bit-planes)
+# --------------------------------------------------------------------------
+
+def bitplanes(codes: np.ndarray):
+    """Signed codes [N, K] -> (mag, sign) uint64 [N, ceil(K/64)]: mag bit set
+    for a non-zero weight, sign bit set for a negative one."""
+    codes = _c(codes, np.int8)
+    N, K = codes.shape
+    words = (K + 63) // 64
+    mag = np.empty((N, words), np.uint64)
+    sign = np.empty((N, words), np.uint64)
+    _load().oracle_bitplanes(_p(codes), N, K, _p(mag), _p(sign))
+    return mag, sign
+
+
+def bitplane_acc(mag: np.ndarray, sign: np.ndarray, xb: np.ndarray, K: int) -> np.ndarray:
+    """dot[n] = popc(mag & XNOR(sign, x)) - popc(mag & XOR(sign, x)) over the row."""
+    mag = _c(mag, np.uint64)
+    sign = _c(sign, np.uint64)
+    xb = _c(xb, np.uint64).reshape(-1)
+    N = mag.shape[0]
+    acc = np.empty(N, np.int32)
+    _load().oracle_bitplane_acc(_p(mag), _p(sign), _p(xb), N, K, _p(acc))
+    return acc
+
+
+def bitplane_gemv(codes: np.ndarray, gamma_eff, x: np.ndarray):
+    """Ternary codes [N, K] against the sign bits of one token x [K]:
+    y = (float)dot * (gamma_eff * max|x|)."""
+    x = _c(x, np.float32).reshape(1, -1)
+    K = codes.shape[1]
+    mag, sign = bitplanes(codes)
+    xb = binary_signs(x, pad_bit=0)
+    s_x = absmax(x)
+    acc = bitplane_acc(mag, sign, xb, K)
+    return {"mag": mag, "sign": sign, "xb": xb, "s_x": s_x, "acc": acc,
+            "y": binary_rescale(acc, gamma_eff, s_x)}

@@ -329,6 +329,57 @@ void oracle_binary_rescale(const int32_t *acc, float s_w, float s_x, int64_t N,
         y[n] = (float)acc[n] * s;
 }
 
+/* ---------------------------------------------------------------------------
+ * Ternary weights x 1-bit activations on two bit-planes.  [FLOOR] "The core
+ * math": a ternary row is two bit-planes, mag (bit set: the weight is
+ * non-zero) and sign (bit set: the weight is negative), and
+ *   dot = POPCNT(mag & XNOR(sign, x)) - POPCNT(mag & XOR(sign, x)),
+ * with x the activation's sign bits; [FLOOR] "What's inside": ternary
+ * weights as two bit-plane u64 word arrays.  Readings: the planes come from
+ * the same absmean codes as the 2-bit path; bit j of word w holds k = 64 w + j;
+ * the activation bit is set for negative values (as in the binary variant, so
+ * XNOR marks a positive product); y = (float)dot * (gamma_eff * s_x) with
+ * s_x = max |x| (the binary variant's activation scale).  Pad bits (K not a
+ * multiple of 64) are 0 in mag, so they never count.
+ * ------------------------------------------------------------------------- */
+void oracle_bitplanes(const int8_t *codes, int64_t N, int64_t K, uint64_t *mag,
+                      uint64_t *sign)
+{
+    int64_t words = (K + 63) / 64;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t w = 0; w < words; ++w) {
+            uint64_t m = 0, s = 0;
+            for (int64_t j = 0; j < 64; ++j) {
+                int64_t k = 64 * w + j;
+                if (k >= K)
+                    continue;
+                int c = codes[n * K + k];
+                if (c != 0)
+                    m |= (uint64_t)1 << j;
+                if (c < 0)
+                    s |= (uint64_t)1 << j;
+            }
+            mag[n * words + w] = m;
+            sign[n * words + w] = s;
+        }
+}
+
+void oracle_bitplane_acc(const uint64_t *mag, const uint64_t *sign,
+                         const uint64_t *xb, int64_t N, int64_t K, int32_t *acc)
+{
+    int64_t words = (K + 63) / 64;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        int64_t dot = 0;
+        for (int64_t w = 0; w < words; ++w) {
+            uint64_t m = mag[n * words + w], s = sign[n * words + w];
+            dot += popcount64_plain(m & ~(s ^ xb[w]));
+            dot -= popcount64_plain(m & (s ^ xb[w]));
+        }
+        acc[n] = (int32_t)dot;
+    }
+}
+
 /* Threads the OpenMP loops above use (1 when built without OpenMP). */
 #ifdef _OPENMP
 #include <omp.h>

@@ -355,3 +355,51 @@ def test_rmsnorm_zero_row_and_quantiser():
     # its position, which quantises to 127
     assert h[1, 5] == pytest.approx(3.0 / math.sqrt(9.0 / 128 + 1e-5), rel=1e-6)
     assert q[1, 5] == 127 and r[1] == 127
+
+
+# ---------------------------------------------------------------- ternary x 1-bit bit-planes
+
+def test_bitplane_hand_worked():
+    # codes [1, 0, -1, 1], x = [2, -3, -1, 0]: mag bits k0, k2, k3 = 0b1101,
+    # sign bit k2 = 0b0100, x sign bits k1, k2 = 0b0110.  By hand:
+    # sum code * sign(x) = (+1)(+1) + 0 + (-1)(-1) + (+1)(+1) = 3 (x = 0 counts +1)
+    codes = np.array([[1, 0, -1, 1]], np.int8)
+    mag, sign = oracle.bitplanes(codes)
+    assert int(mag[0, 0]) == 0b1101 and int(sign[0, 0]) == 0b0100
+    out = oracle.bitplane_gemv(codes, np.float32(0.5), _f32([2.0, -3.0, -1.0, 0.0]))
+    assert int(out["xb"][0, 0]) == 0b0110
+    assert out["acc"][0] == 3
+    assert out["s_x"] == np.float32(3.0)
+    assert out["y"][0] == np.float32(3 * 0.5 * 3.0)
+
+
+@pytest.mark.parametrize("N,K", [(7, 64), (5, 200), (3, 1), (9, 4096)])
+def test_bitplane_dot_is_the_signed_product(N, K):
+    # brute force: sum_k code[n][k] * (x[k] < 0 ? -1 : +1), zeros and -0.0 included
+    rng = np.random.default_rng(N * 1000 + K)
+    codes = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    x = rng.standard_normal(K).astype(np.float32)
+    x[rng.integers(0, K, max(1, K // 10))] = 0.0
+    x[rng.integers(0, K, max(1, K // 10))] = -0.0
+    out = oracle.bitplane_gemv(codes, np.float32(1.0), x)
+    sx = np.where(x < 0, -1, 1).astype(np.int64)
+    want = (codes.astype(np.int64) * sx[None, :]).sum(axis=1)
+    np.testing.assert_array_equal(out["acc"], want)
+
+
+def test_bitplane_invariants():
+    W = si.weight(64, 640, seed=3).numpy()
+    g = oracle.weight_scale(W)
+    codes = oracle.ternary_codes(W, g)
+    mag, sign = oracle.bitplanes(codes)
+    # sign bits only where the weight is non-zero; popcount(mag) = non-zeros
+    assert not np.any(sign & ~mag)
+    nz = np.array([sum(bin(int(v)).count("1") for v in row) for row in mag])
+    np.testing.assert_array_equal(nz, (codes != 0).sum(axis=1))
+    x = si.activations(1, 640, seed=4, dtype=torch.float32).numpy()[0]
+    acc = oracle.bitplane_gemv(codes, g, x)["acc"]
+    # |dot| <= non-zeros and dot has their parity
+    assert np.all(np.abs(acc) <= nz) and np.all((acc - nz) % 2 == 0)
+    # flipping every activation's sign negates every dot product (no x is 0)
+    assert np.all(x != 0)
+    np.testing.assert_array_equal(oracle.bitplane_gemv(codes, g, -x)["acc"], -acc)
