@@ -79,12 +79,21 @@ _SIGNATURES = {
                                     _i64, _vp, _vp]),
     "bitlinear_gemv_fused_multi": (_int, [_int, _vp, _vp, _vp, _i64, _vp, _int, _i64, _i64,
                                           _vp, _int, _vp, _vp, ctypes.c_uint, _vp]),
+    "bitlinear_rmsnorm_quantize_act": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int,
+                                              ctypes.c_float, _vp, _vp, _vp, _vp]),
+    "bitlinear_rmsnorm_gemv_fused_multi": (_int, [_int, _vp, _vp, _vp, _i64, _vp, _int, _vp,
+                                                  _int, ctypes.c_float, _vp, _int, _vp, _vp,
+                                                  ctypes.c_uint, _vp]),
     "bitlinear_gemm_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bitlinear_gemm": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _int, _i64,
                               _vp, _vp, _sz, _vp]),
     "bitlinear_binary_packed_bytes": (_sz, [_i64, _i64]),
     "bitlinear_binary_pack": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _vp]),
     "bitlinear_binary_gemv": (_int, [_vp, _vp, _i64, _i64, _vp, _int, _vp, _int, _vp, _vp]),
+    "bitlinear_lut_gemv": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _int, _vp, _vp]),
+    "bitlinear_bitplane_bytes": (_sz, [_i64, _i64]),
+    "bitlinear_bitplane_pack": (_int, [_vp, _i64, _i64, _vp, _vp]),
+    "bitlinear_bitplane_gemv": (_int, [_vp, _vp, _i64, _i64, _vp, _int, _vp, _int, _vp, _vp]),
     "bitlinear_last_device_status": (_int, [_vp]),
     "bitlinear_device_sm_count": (_int, []),
 }
@@ -266,6 +275,56 @@ def gemv_fused_multi(weights, x: torch.Tensor, out_dtype=torch.bfloat16, outs=No
     return outs
 
 
+RMS_EPS = 1e-5  # default RMSNorm epsilon (the library's reading; the pages give none)
+
+
+def rmsnorm_quantize_act(x: torch.Tensor, gain=None, eps: float = RMS_EPS, out=None):
+    """RMSNorm each token (gain [K] fp32/bf16 or None), then per-token absmax
+    int8: returns (q int8 [M,K], d fp32 [M], rowsum int32 [M])."""
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    M, K = x.shape
+    if out is None:
+        q = torch.empty(M, K, dtype=torch.int8, device=x.device)
+        d = torch.empty(M, dtype=torch.float32, device=x.device)
+        r = torch.empty(M, dtype=torch.int32, device=x.device)
+    else:
+        q, d, r = out
+    gt = BL_F32 if gain is None else _dt(gain.dtype)
+    with _on(x.device):
+        _check(_lib.bitlinear_rmsnorm_quantize_act(_ptr(x), _dt(x.dtype), M, K, x.stride(0),
+                                                   _ptr(gain), gt, float(eps), _ptr(q), _ptr(d),
+                                                   _ptr(r), _stream(x.device)),
+               "bitlinear_rmsnorm_quantize_act")
+    return q, d, r
+
+
+def rmsnorm_gemv_fused_multi(weights, x: torch.Tensor, gain=None, eps: float = RMS_EPS,
+                             out_dtype=torch.bfloat16, outs=None, acc_dbgs=None,
+                             pdl: bool = False):
+    """One token through RMSNorm, quantisation and several decode BitLinears
+    sharing it (gate/up, q/k/v), in one launch.  x: [K] or [1, K]."""
+    x = x.reshape(-1)
+    n = len(weights)
+    if outs is None:
+        outs = [torch.empty(1, w.N, dtype=out_dtype, device=x.device) for w in weights]
+    P = ctypes.c_void_p * n
+    I64 = ctypes.c_int64 * n
+    packed = P(*[w.packed.data_ptr() for w in weights])
+    scales = P(*[w.w_scale.data_ptr() for w in weights])
+    Ns = I64(*[w.N for w in weights])
+    ys = P(*[o.data_ptr() for o in outs])
+    ldys = I64(*[o.stride(0) if o.dim() > 1 else o.numel() for o in outs])
+    accs = None if acc_dbgs is None else P(*[0 if a is None else a.data_ptr() for a in acc_dbgs])
+    gt = BL_F32 if gain is None else _dt(gain.dtype)
+    with _on(x.device):
+        _check(_lib.bitlinear_rmsnorm_gemv_fused_multi(
+            n, packed, scales, Ns, weights[0].K, _ptr(x), _dt(x.dtype), _ptr(gain), gt,
+            float(eps), ys, _dt(outs[0].dtype), ldys, accs, BL_FLAG_PDL if pdl else 0,
+            _stream(x.device)), "bitlinear_rmsnorm_gemv_fused_multi")
+    return outs
+
+
 def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(_lib.bitlinear_gemm_workspace_bytes(M, N, K))
 
@@ -326,6 +385,51 @@ def binary_gemv(w: BinaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16, out=
         _check(_lib.bitlinear_binary_gemv(_ptr(w.bits), _ptr(w.s_w), w.N, w.K, _ptr(x),
                                           _dt(x.dtype), _ptr(out), _dt(out.dtype), _ptr(acc_dbg),
                                           _stream(x.device)), "bitlinear_binary_gemv")
+    return out
+
+
+def lut_gemv(w: TernaryWeight, q, d, out_dtype=torch.bfloat16, out=None, acc_dbg=None):
+    """One token's ternary GEMV by table lookup (K <= 12288), on pre-quantised
+    activations (q [1, K] or [K], d [1]); same results as gemv()."""
+    q = q.reshape(-1)
+    if out is None:
+        out = torch.empty(1, w.N, dtype=out_dtype, device=q.device)
+    with _on(q.device):
+        _check(_lib.bitlinear_lut_gemv(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q),
+                                       _ptr(d), _ptr(out), _dt(out.dtype), _ptr(acc_dbg),
+                                       _stream(q.device)), "bitlinear_lut_gemv")
+    return out
+
+
+@dataclass
+class BitPlaneWeight:
+    """Ternary weight as (mag, sign) bit-planes, with the packed weight's gamma."""
+    planes: torch.Tensor   # int64 [N, K/64, 2] (uint64 words)
+    w_scale: torch.Tensor  # float32 [1]
+    N: int
+    K: int
+
+
+def bitplane_pack(w: TernaryWeight) -> BitPlaneWeight:
+    """Bit-planes of a packed ternary weight (same codes, same gamma)."""
+    planes = torch.empty(w.N, w.K // 64, 2, dtype=torch.int64, device=w.packed.device)
+    with _on(w.packed.device):
+        _check(_lib.bitlinear_bitplane_pack(_ptr(w.packed), w.N, w.K, _ptr(planes),
+                                            _stream(w.packed.device)), "bitlinear_bitplane_pack")
+    return BitPlaneWeight(planes, w.w_scale, w.N, w.K)
+
+
+def bitplane_gemv(w: BitPlaneWeight, x: torch.Tensor, out_dtype=torch.bfloat16, out=None,
+                  acc_dbg=None):
+    """Ternary weights x the sign bits of one token: y = dot * (gamma * max|x|)."""
+    x = x.reshape(-1)
+    if out is None:
+        out = torch.empty(w.N, dtype=out_dtype, device=x.device)
+    with _on(x.device):
+        _check(_lib.bitlinear_bitplane_gemv(_ptr(w.planes), _ptr(w.w_scale), w.N, w.K, _ptr(x),
+                                            _dt(x.dtype), _ptr(out), _dt(out.dtype),
+                                            _ptr(acc_dbg), _stream(x.device)),
+               "bitlinear_bitplane_gemv")
     return out
 
 

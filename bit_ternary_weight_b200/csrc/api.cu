@@ -250,6 +250,30 @@ int bitlinear_quantize_act(const void *x, int xt, int64_t M, int64_t K, int64_t 
                                static_cast<cudaStream_t>(stream));
 }
 
+int bitlinear_rmsnorm_quantize_act(const void *x, int xt, int64_t M, int64_t K, int64_t ldx,
+                                   const void *gain, int gt, float eps, int8_t *q, float *d,
+                                   int32_t *rowsum, void *stream)
+{
+    if (!x || !q || !d || !rowsum)
+        return BL_ERR_NULL;
+    if (!valid_dtype(xt) || (gain && !valid_dtype(gt)))
+        return BL_ERR_DTYPE;
+    if (!valid_nk(1, K) || M < 1 || M > (int64_t(1) << 31) || ldx < K || !(eps >= 0.0f) ||
+        !(eps <= 3.0e38f) || !rmsnorm_quantize_fits(xt, K, gain != nullptr))
+        return BL_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(gain) || (ldx * elem_bytes(xt)) % 16 ||
+        (reinterpret_cast<uintptr_t>(d) & 3u) || (reinterpret_cast<uintptr_t>(rowsum) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({x, gain, q, d, rowsum})))
+        return st;
+    return launch_rmsnorm_quantize_act(x, xt, M, K, ldx, gain, gt, eps, q, d, rowsum,
+                                       static_cast<cudaStream_t>(stream));
+}
+
 namespace {
 
 int check_gemv_common(const uint8_t *packed, const float *w_scale, int64_t N,
@@ -375,6 +399,57 @@ int bitlinear_gemv_fused_multi(int count, const uint8_t *const *packed,
     return launch_gemv_batch(b, true, static_cast<cudaStream_t>(stream));
 }
 
+int bitlinear_rmsnorm_gemv_fused_multi(int count, const uint8_t *const *packed,
+                                       const float *const *w_scale, const int64_t *N, int64_t K,
+                                       const void *x, int xt, const void *gain, int gt, float eps,
+                                       void *const *y, int yt, const int64_t *ldy,
+                                       int32_t *const *acc_dbg, unsigned flags, void *stream)
+{
+    if (!packed || !w_scale || !N || !y || !ldy || !x)
+        return BL_ERR_NULL;
+    if (count < 1 || count > kGemvMaxProblems)
+        return BL_ERR_SHAPE;
+    if (flags & ~BL_FLAG_PDL)
+        return BL_ERR_SHAPE;
+    if (!valid_dtype(xt) || !valid_dtype(yt) || (gain && !valid_dtype(gt)))
+        return BL_ERR_DTYPE;
+    if (!(eps >= 0.0f) || !(eps <= 3.0e38f))
+        return BL_ERR_SHAPE;
+    int st;
+    for (int i = 0; i < count; ++i) {
+        if ((st = check_gemv_common(packed[i], w_scale[i], N[i], K, 1, y[i], yt, ldy[i], 1)))
+            return st;
+        if (acc_dbg && (reinterpret_cast<uintptr_t>(acc_dbg[i]) & 3u))
+            return BL_ERR_ALIGN;
+    }
+    if (!aligned16(x) || !aligned16(gain))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    if ((st = need_device(&di)))
+        return st;
+    GemvBatch b{};
+    b.count = count;
+    for (int i = 0; i < count; ++i)
+        b.prob[i] = GemvProblem{packed[i], w_scale[i], N[i], y[i], ldy[i],
+                                acc_dbg ? acc_dbg[i] : nullptr};
+    b.K = K;
+    b.M = 1;
+    b.x = x;
+    b.xt = xt;
+    b.ldx = K;
+    b.yt = yt;
+    b.flags = flags;
+    // the streaming one-token kernel only: K a multiple of 256 up to 32768
+    if (!gemv_stream_applies(b, di->sm_count))
+        return BL_ERR_SHAPE;
+    if ((st = check_dev_ptrs({x, gain})))
+        return st;
+    for (int i = 0; i < count; ++i)
+        if ((st = check_dev_ptrs({packed[i], w_scale[i], y[i], acc_dbg ? acc_dbg[i] : nullptr})))
+            return st;
+    return launch_gemv_stream(b, true, static_cast<cudaStream_t>(stream), gain, gt, eps, true);
+}
+
 size_t bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
     if (!valid_nk(N, K) || M < 1)
@@ -455,8 +530,82 @@ int bitlinear_binary_gemv(const uint64_t *Wb, const float *s_w, int64_t N, int64
         return st;
     if ((st = check_dev_ptrs({Wb, s_w, x, y, acc_dbg})))
         return st;
+    if (popc_stream_applies_binary(K))
+        return launch_binary_gemv_stream(Wb, s_w, N, K, x, xt, y, yt, acc_dbg,
+                                         static_cast<cudaStream_t>(stream));
     return launch_binary_gemv(Wb, s_w, N, K, x, xt, y, yt, acc_dbg,
                               static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_lut_gemv(const uint8_t *packed, const float *w_scale, int64_t N, int64_t K,
+                       const int8_t *q, const float *d, void *y, int yt, int32_t *acc_dbg,
+                       void *stream)
+{
+    if (!q || !d)
+        return BL_ERR_NULL;
+    int st = check_gemv_common(packed, w_scale, N, K, 1, y, yt, N, 1);
+    if (st)
+        return st;
+    if (!lut_gemv_applies(K))
+        return BL_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(d) & 3u) || (reinterpret_cast<uintptr_t>(acc_dbg) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    if ((st = need_device(&di)))
+        return st;
+    if ((st = check_dev_ptrs({packed, w_scale, q, d, y, acc_dbg})))
+        return st;
+    return launch_lut_gemv(packed, w_scale, N, K, q, d, y, yt, acc_dbg,
+                           static_cast<cudaStream_t>(stream));
+}
+
+size_t bitlinear_bitplane_bytes(int64_t N, int64_t K)
+{
+    if (!valid_nk(N, K))
+        return 0;
+    return static_cast<size_t>(N) * static_cast<size_t>(K / 64) * 16;
+}
+
+int bitlinear_bitplane_pack(const uint8_t *packed, int64_t N, int64_t K, uint64_t *planes,
+                            void *stream)
+{
+    if (!packed || !planes)
+        return BL_ERR_NULL;
+    if (!valid_nk(N, K) || K > 65536)
+        return BL_ERR_SHAPE;
+    if (!aligned16(packed) || !aligned16(planes))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({packed, planes})))
+        return st;
+    return launch_bitplane_pack(packed, N, K, planes, static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_bitplane_gemv(const uint64_t *planes, const float *w_scale, int64_t N, int64_t K,
+                            const void *x, int xt, void *y, int yt, int32_t *acc_dbg,
+                            void *stream)
+{
+    if (!planes || !w_scale || !x || !y)
+        return BL_ERR_NULL;
+    if (!valid_dtype(xt) || !valid_dtype(yt))
+        return BL_ERR_DTYPE;
+    if (!valid_nk(N, K) || K > 65536)
+        return BL_ERR_SHAPE;
+    if (!aligned16(planes) || !aligned16(x) || (reinterpret_cast<uintptr_t>(w_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(y) & (yt == BL_BF16 ? 1u : 3u)) ||
+        (reinterpret_cast<uintptr_t>(acc_dbg) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({planes, w_scale, x, y, acc_dbg})))
+        return st;
+    return launch_bitplane_gemv(planes, w_scale, N, K, x, xt, y, yt, acc_dbg,
+                                static_cast<cudaStream_t>(stream));
 }
 
 int bitlinear_last_device_status(void *stream)

@@ -56,6 +56,14 @@ int launch_quantize_act(const void *x, int xt, int64_t M, int64_t K,
                         int64_t ldx, int8_t *q, float *d, int32_t *rowsum,
                         cudaStream_t s);
 
+// RMSNorm, then per-token absmax quantisation of the normalised rows.
+int launch_rmsnorm_quantize_act(const void *x, int xt, int64_t M, int64_t K, int64_t ldx,
+                                const void *gain, int gt, float eps, int8_t *q, float *d,
+                                int32_t *rowsum, cudaStream_t s);
+// Whether a row of K elements (and the gain) fits the RMSNorm kernel's
+// shared-memory staging.
+bool rmsnorm_quantize_fits(int xt, int64_t K, bool has_gain);
+
 int launch_pack(const void *W, int wt, int64_t N, int64_t K, uint8_t *packed,
                 float *w_scale, double *row_sums, cudaStream_t s);
 
@@ -106,6 +114,13 @@ struct GemvBatch {
 
 int launch_gemv_batch(const GemvBatch &b, bool fused, cudaStream_t s);
 
+// The streaming one-token kernel (gemv_stream.cu): whether it takes the batch,
+// and its launch with the token normalised (RMSNorm with gain / eps) before
+// quantisation when `norm` is set.
+bool gemv_stream_applies(const GemvBatch &b, int sm_count);
+int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s, const void *gain, int gt,
+                       float eps, bool norm);
+
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int launch_gemm(const GemvArgs &a, void *ws, size_t ws_bytes, cudaStream_t s);
 
@@ -114,5 +129,23 @@ int launch_binary_pack(const void *W, int wt, int64_t N, int64_t K,
 int launch_binary_gemv(const uint64_t *Wb, const float *s_w, int64_t N,
                        int64_t K, const void *x, int xt, void *y, int yt,
                        int32_t *acc_dbg, cudaStream_t s);
+
+// Streaming popcount GEMVs (popc_stream.cu): binary weights (rows of K/8
+// bytes, which must be a multiple of 16) and ternary bit-planes (rows of K/4
+// bytes), K <= 65536.
+bool popc_stream_applies_binary(int64_t K);
+int launch_binary_gemv_stream(const uint64_t *Wb, const float *s_w, int64_t N, int64_t K,
+                              const void *x, int xt, void *y, int yt, int32_t *acc_dbg,
+                              cudaStream_t s);
+int launch_bitplane_pack(const uint8_t *packed, int64_t N, int64_t K, uint64_t *planes,
+                         cudaStream_t s);
+int launch_bitplane_gemv(const uint64_t *planes, const float *w_scale, int64_t N, int64_t K,
+                         const void *x, int xt, void *y, int yt, int32_t *acc_dbg, cudaStream_t s);
+
+// Lookup-table ternary GEMV of one token (lut_gemv.cu), K <= 12288.
+bool lut_gemv_applies(int64_t K);
+int launch_lut_gemv(const uint8_t *packed, const float *w_scale, int64_t N, int64_t K,
+                    const int8_t *q, const float *d, void *y, int yt, int32_t *acc_dbg,
+                    cudaStream_t s);
 
 }  // namespace bl

@@ -68,7 +68,9 @@ struct Geo {
     static constexpr int kCtasPerSm = KC == 8 ? 2 : 1;
 };
 
-enum { SMODE_Q = 0, SMODE_X_BF16 = 1, SMODE_X_F32 = 2 };
+// Activations: pre-quantised q; raw bf16 / fp32 x quantised in the prologue;
+// or x normalised (RMSNorm) and then quantised in the prologue.
+enum { SMODE_Q = 0, SMODE_X_BF16 = 1, SMODE_X_F32 = 2, SMODE_NORM_BF16 = 3, SMODE_NORM_F32 = 4 };
 
 // 512-byte pieces (256 k) of one group per stage: the whole k range when it
 // is at most two pieces per consumer warp (one stage per set), else one per
@@ -84,6 +86,9 @@ struct StreamParams {
     const float *d;
     const int32_t *rowsum;
     const void *x;
+    const void *gain;    // RMSNorm gain [K] (SMODE_NORM_*), NULL for none
+    int gt;              // its dtype
+    float eps;           // RMSNorm epsilon
     int yt;
     // CTA b owns row groups [b*gpc_base + min(b, gpc_rem), ...), gpc_base (+1) of them
     int64_t gpc_base;
@@ -98,6 +103,7 @@ struct StreamSmem {
     int abort_flag;
     alignas(16) float bmax[kMaxConsumers];   // read back as float4
     int bsum[kMaxConsumers];
+    double bss[kMaxConsumers];               // RMSNorm: per-warp sums of squares
     float d;
     float wscale[kGemvMaxProblems];   // each product's gamma_eff
     int sacc[kMaxGroupsPerCta][8];
@@ -294,6 +300,126 @@ __device__ __forceinline__ void stream_copy_q(const StreamParams &p, StreamSmem 
     __syncwarp();
 }
 
+// Eight gain values (k .. k + 7) as fp32; 1.0 without a gain (an exact
+// identity for the product that applies it).
+__device__ __forceinline__ void stream_gain8(const StreamParams &p, int64_t k, float (&g)[8])
+{
+    if (!p.gain) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            g[j] = 1.0f;
+    } else if (p.gt == BL_BF16) {
+        bf16x8_f32(ld_ro_v4(static_cast<const __nv_bfloat16 *>(p.gain) + k), g);
+    } else {
+        const float *gp = static_cast<const float *>(p.gain) + k;
+        const uint4 a = ld_ro_v4(gp), b = ld_ro_v4(gp + 4);
+        g[0] = __uint_as_float(a.x); g[1] = __uint_as_float(a.y);
+        g[2] = __uint_as_float(a.z); g[3] = __uint_as_float(a.w);
+        g[4] = __uint_as_float(b.x); g[5] = __uint_as_float(b.y);
+        g[6] = __uint_as_float(b.z); g[7] = __uint_as_float(b.w);
+    }
+}
+
+// Block-wide sum of the consumer threads' fp64 partial sums of squares, then
+// the RMSNorm factor r = 1 / sqrt((float)(S / K) + eps) (fp32, correctly
+// rounded square root and division).
+template <int KC>
+__device__ __forceinline__ float stream_rms_factor(const StreamParams &p, StreamSmem &sm, double ss)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+    if (lane == 0)
+        sm.bss[warp] = ss;
+    consumers_sync<KC>();
+    double S = 0.0;
+#pragma unroll
+    for (int w = 0; w < KC; ++w)
+        S = __dadd_rn(S, sm.bss[w]);
+    const float ms = __double2float_rn(__ddiv_rn(S, double(p.K)));
+    return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.eps)));
+}
+
+// RMSNorm, then quantisation, of the token x: h = (x * r) * gain, each warp
+// for the activations of its own pieces (as in stream_quantize_bf16); two
+// block-wide reductions (the sum of squares, then the absmax of h).  CH > 0
+// (bf16 x only): the warp's raw x stays in registers, CH pieces; CH = 0: x
+// is read again from L2 for each pass.
+template <int KC, int XT, int CH>
+__device__ __forceinline__ void stream_rmsnorm_quantize(const StreamParams &p, StreamSmem &sm, int8_t *qs)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int P = int(p.K / 256);
+    constexpr int RC = CH > 0 ? CH : 1;
+    uint4 raw[RC];
+    if constexpr (CH == 0)
+        raw[0] = make_uint4(0, 0, 0, 0);   // unused: x is re-read from L2
+    auto load_x = [&](int i, int j, float (&f)[8]) {
+        if constexpr (CH > 0)
+            bf16x8_f32(raw[i], f);
+        else
+            load8<XT, true>(p.x, (int64_t(j) * 32 + lane) * 8, f);
+    };
+    if constexpr (CH > 0) {
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int j = i * KC + warp;
+            raw[i] = j < P ? ld_dep_v4(static_cast<const __nv_bfloat16 *>(p.x) + (int64_t(j) * 32 + lane) * 8)
+                           : make_uint4(0, 0, 0, 0);
+        }
+    }
+    constexpr int kUnroll = CH > 0 ? CH : 4;
+    double ss = 0.0;
+#pragma unroll kUnroll
+    for (int i = 0; i < (CH > 0 ? CH : (P + KC - 1) / KC); ++i) {
+        const int j = i * KC + warp;
+        if (j < P) {
+            float f[8];
+            load_x(i, j, f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                ss = __dadd_rn(ss, __dmul_rn(double(f[e]), double(f[e])));
+        }
+    }
+    const float r = stream_rms_factor<KC>(p, sm, ss);
+    auto h8 = [&](int i, int j, float (&h)[8]) {
+        float g[8];
+        load_x(i, j, h);
+        stream_gain8(p, (int64_t(j) * 32 + lane) * 8, g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            h[e] = __fmul_rn(__fmul_rn(h[e], r), g[e]);
+    };
+    float amax = 0.0f;
+#pragma unroll kUnroll
+    for (int i = 0; i < (CH > 0 ? CH : (P + KC - 1) / KC); ++i) {
+        const int j = i * KC + warp;
+        if (j < P) {
+            float h[8];
+            h8(i, j, h);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                amax = fmaxf(amax, fabsf(h[e]));
+        }
+    }
+    const float s = stream_scale<KC>(sm, amax);
+    int sum = 0;
+#pragma unroll kUnroll
+    for (int i = 0; i < (CH > 0 ? CH : (P + KC - 1) / KC); ++i) {
+        const int j = i * KC + warp;
+        if (j < P) {
+            float h[8];
+            h8(i, j, h);
+            *reinterpret_cast<uint2 *>(qs + (j * 32 + lane) * 8) = quant8(h, s, sum);
+        }
+    }
+    sum = __reduce_add_sync(0xffffffffu, sum);
+    if (lane == 0)
+        sm.bsum[warp] = sum;
+    __syncwarp();
+}
+
 // One 16-byte piece of stored codes (64 k of one row) against the 64
 // activations q[0..3] into four accumulators (s, 4s, 16s, 64s weighted).
 __device__ __forceinline__ void mac4(const uint4 wv, const uint4 (&q)[4], int (&acc)[4])
@@ -482,6 +608,10 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if constexpr (MODE == SMODE_Q)
         stream_copy_q<KC>(p, sm, qs);
+    else if constexpr (MODE == SMODE_NORM_BF16)
+        stream_rmsnorm_quantize<KC, BL_BF16, CH>(p, sm, qs);
+    else if constexpr (MODE == SMODE_NORM_F32)
+        stream_rmsnorm_quantize<KC, BL_F32, 0>(p, sm, qs);
     else if constexpr (MODE == SMODE_X_BF16 && CH > 0)
         stream_quantize_bf16<KC, CH>(p, sm, qs);
     else
@@ -625,8 +755,16 @@ int launch_mode(const StreamParams &base, cudaStream_t s, unsigned flags)
 }
 
 template <int KC>
-int launch_kc(const StreamParams &p, bool fused, int xt, cudaStream_t s, unsigned flags)
+int launch_kc(const StreamParams &p, bool fused, int xt, cudaStream_t s, unsigned flags, bool norm)
 {
+    if (norm) {
+        if (xt != BL_BF16)
+            return launch_mode<KC, SMODE_NORM_F32, 0>(p, s, flags);
+        constexpr int kNormChunks = 8 * Geo<KC>::kConsumerThreads;
+        if (p.K <= int64_t(4) * kNormChunks)
+            return launch_mode<KC, SMODE_NORM_BF16, 4>(p, s, flags);
+        return launch_mode<KC, SMODE_NORM_BF16, 0>(p, s, flags);
+    }
     if (!fused)
         return launch_mode<KC, SMODE_Q, 0>(p, s, flags);
     if (xt != BL_BF16)
@@ -655,7 +793,8 @@ bool gemv_stream_applies(const GemvBatch &b, int sm_count)
     return ng <= int64_t(kMaxGroupsPerCta) * sm_count;
 }
 
-int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s)
+int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s, const void *gain, int gt,
+                       float eps, bool norm)
 {
     StreamParams p{};
     p.count = b.count;
@@ -671,10 +810,18 @@ int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s)
     p.d = b.d;
     p.rowsum = b.rowsum;
     p.x = b.x;
+    p.gain = gain;
+    p.gt = gt;
+    p.eps = eps;
     p.yt = b.yt;
     if (b.K <= kSmallK)
-        return launch_kc<8>(p, fused, b.xt, s, b.flags);
-    return launch_kc<16>(p, fused, b.xt, s, b.flags);
+        return launch_kc<8>(p, fused, b.xt, s, b.flags, norm);
+    return launch_kc<16>(p, fused, b.xt, s, b.flags, norm);
+}
+
+int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s)
+{
+    return launch_gemv_stream(b, fused, s, nullptr, BL_F32, 0.0f, false);
 }
 
 }  // namespace bl

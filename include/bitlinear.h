@@ -226,6 +226,58 @@ int bitlinear_gemv_fused_multi(int count, const uint8_t *const *packed,
                                unsigned flags, void *stream);
 
 /*
+ * RMSNorm, then per-token absmax int8 quantisation of the normalised rows:
+ * the step in front of a BitLinear in a decoder layer, in one launch.
+ * Source: "bit-floor" README, section "What's inside" (rmsnorm.cu: a
+ * mean-square reduction over the row, an rsqrt scale applied per element);
+ * "How to Run BitNet Inference on GPU Using CUDA Kernels", section
+ * "Understanding the Two-Phase Architecture" (Attention and FeedForward feed
+ * their inputs to BitLinear).  Per token m (identical on the CPU oracle):
+ *   S    = sum_k x[m][k]^2 in fp64;  ms = (float)(S / K)
+ *   r    = 1 / sqrt(ms + eps)        fp32, correctly rounded sqrt and divide
+ *   h[k] = (x[m][k] * r) * gain[k]   two fp32 products (gain NULL: x * r)
+ *   q, d, rowsum of h as bitlinear_quantize_act defines them.
+ * The fp64 sum runs in a different order than the oracle's; the two can
+ * differ only when S / K lies within about 1e-15 (relative) of an fp32
+ * rounding boundary.
+ *   x, xt, M, K, ldx, q, d, rowsum   as for bitlinear_quantize_act
+ *   gain    device [K] of dtype gt (BL_F32 or BL_BF16), 16-byte aligned, or
+ *           NULL for no gain
+ *   eps     >= 0, finite (1e-5 is this library's default reading)
+ * A token's row (and the gain as fp32) is staged in shared memory: K * 2
+ * (bf16) or K * 4 (fp32) bytes, plus K * 4 with a gain, must fit in 200 KiB,
+ * else BL_ERR_SHAPE.
+ */
+int bitlinear_rmsnorm_quantize_act(const void *x, int xt, int64_t M, int64_t K,
+                                   int64_t ldx, const void *gain, int gt,
+                                   float eps, int8_t *q, float *d,
+                                   int32_t *rowsum, void *stream);
+
+/*
+ * Decode BitLinears of one token with RMSNorm in front, in one launch: the
+ * token x is normalised (as bitlinear_rmsnorm_quantize_act defines it),
+ * quantised, multiplied by `count` packed weights that share it (for
+ * instance gate and up, or q, k and v) and rescaled.  Sources as for
+ * bitlinear_rmsnorm_quantize_act and bitlinear_gemv_fused_multi.
+ *   x, xt        device [K] (one token), BL_F32 or BL_BF16
+ *   gain, gt, eps  as for bitlinear_rmsnorm_quantize_act
+ *   other arguments as for bitlinear_gemv_fused_multi (with M = 1)
+ * Runs the streaming one-token kernel only: K a multiple of 256 up to 32768
+ * and at most 64 row groups of 8 per SM, else BL_ERR_SHAPE (other shapes:
+ * bitlinear_rmsnorm_quantize_act, then bitlinear_gemv).  Under BL_FLAG_PDL
+ * the gain, like the packed weights and scales, must not have been written
+ * by the kernel immediately before this call.
+ */
+int bitlinear_rmsnorm_gemv_fused_multi(int count, const uint8_t *const *packed,
+                                       const float *const *w_scale,
+                                       const int64_t *N, int64_t K,
+                                       const void *x, int xt, const void *gain,
+                                       int gt, float eps, void *const *y, int yt,
+                                       const int64_t *ldy,
+                                       int32_t *const *acc_dbg, unsigned flags,
+                                       void *stream);
+
+/*
  * Bytes of workspace bitlinear_gemm needs for this problem (0 if none).
  * Nonzero for small batches (M <= 32) whose output tiles alone would leave
  * SMs idle: K is then split across CTAs and the int32 partial sums meet in
@@ -280,6 +332,62 @@ int bitlinear_binary_pack(const void *W, int wt, int64_t N, int64_t K,
 int bitlinear_binary_gemv(const uint64_t *Wb, const float *s_w, int64_t N,
                           int64_t K, const void *x, int xt, void *y, int yt,
                           int32_t *acc_dbg, void *stream);
+
+/*
+ * Ternary GEMV of one token by table lookup (the lookup-table method of the
+ * TL1 / TL2 CPU kernels: "Run 100B Models on Your Laptop CPU: Microsoft
+ * BitNet Exposed", section "Key Features That Make BitNet Insane", T-MAC's
+ * lookup tables), on the TL packed weights.  For each pair of activations
+ * (k, k + 4) that one 4-bit field of a TL byte covers, a 16-entry table of
+ * (s_a - 1) q[k] + (s_b - 1) q[k + 4] is built in shared memory and indexed
+ * by the field; acc is the same exact integer as bitlinear_gemv's, and
+ * y = ((float)acc * d) * gamma_eff.  Offered for comparison with the dp4a
+ * GEMV (same inputs, same results).
+ *   packed, w_scale   from bitlinear_pack (device)
+ *   q, d              device, one token from bitlinear_quantize_act (q [K])
+ *   y                 device [N] of dtype yt;  acc_dbg NULL or device [N]
+ * K <= 12288 (the tables take 16.5 bytes of shared memory per k).
+ */
+int bitlinear_lut_gemv(const uint8_t *packed, const float *w_scale, int64_t N,
+                       int64_t K, const int8_t *q, const float *d, void *y,
+                       int yt, int32_t *acc_dbg, void *stream);
+
+/* Bytes of the bit-plane array: N * (K/64) * 16 (a mag and a sign word per
+ * 64 k of each row). */
+size_t bitlinear_bitplane_bytes(int64_t N, int64_t K);
+
+/*
+ * Ternary weights as two bit-planes, from the TL packed array: for every row
+ * n and 64-k word w, the pair (mag, sign) at uint64 index 2 (n (K/64) + w)
+ * and 2 (n (K/64) + w) + 1, bit j <-> k = 64 w + j; mag set for a non-zero
+ * weight, sign set for a negative one.  Source: "bit-floor" README, sections
+ * "The core math" (ternary GEMV on two bit-planes) and "What's inside"
+ * (ternary weights packed as two bit-plane u64 word arrays).  The planes
+ * keep the weight scale of the packed weight (its w_scale).
+ *   packed   device, from bitlinear_pack (N, K)
+ *   planes   device, bitlinear_bitplane_bytes(N, K) bytes, written
+ * K <= 65536.
+ */
+int bitlinear_bitplane_pack(const uint8_t *packed, int64_t N, int64_t K,
+                            uint64_t *planes, void *stream);
+
+/*
+ * Ternary-weight x 1-bit-activation GEMV of one token on the bit-planes:
+ *   acc[n] = POPCNT(mag & XNOR(sign, xb)) - POPCNT(mag & XOR(sign, xb))
+ *          = sum_k code[n][k] * (x[k] < 0 ? -1 : +1)
+ *   y[n]   = (float)acc[n] * (w_scale * s_x),  s_x = max |x|
+ * with xb the sign bits of x (set for negative values, -0.0 counts as
+ * positive).  Source: "bit-floor" README, section "The core math" (ternary
+ * GEMV, "no floating point in the inner loop").
+ *   planes   device, from bitlinear_bitplane_pack
+ *   w_scale  device, 1 float: gamma_eff of the packed weight
+ *   x        device [K] of dtype xt;  y device [N] of dtype yt
+ *   acc_dbg  NULL or device [N] int32
+ * K <= 65536.
+ */
+int bitlinear_bitplane_gemv(const uint64_t *planes, const float *w_scale,
+                            int64_t N, int64_t K, const void *x, int xt,
+                            void *y, int yt, int32_t *acc_dbg, void *stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the

@@ -125,3 +125,54 @@ def test_valid_arguments_without_device_fail_cleanly(bl):
         pytest.skip("a device is present")
     st = _gemv(bl)
     assert st in (bl.BL_ERR_CUDA, bl.BL_ERR_UNSUPPORTED)
+
+
+def test_rmsnorm_argument_errors_before_any_cuda_call(bl):
+    A = 0x7f0000000000
+    L = bl.lib
+    # null, dtype, shape (negative / non-finite eps, K), alignment
+    assert L.bitlinear_rmsnorm_quantize_act(None, 1, 1, 64, 64, None, 0, 1e-5, A, A, A, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_rmsnorm_quantize_act(A, 7, 1, 64, 64, None, 0, 1e-5, A, A, A, None) == bl.BL_ERR_DTYPE
+    assert L.bitlinear_rmsnorm_quantize_act(A, 1, 1, 64, 64, A, 5, 1e-5, A, A, A, None) == bl.BL_ERR_DTYPE
+    assert L.bitlinear_rmsnorm_quantize_act(A, 1, 1, 64, 64, None, 0, -1.0, A, A, A, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_rmsnorm_quantize_act(A, 1, 1, 64, 64, None, 0, float("nan"), A, A, A,
+                                            None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_rmsnorm_quantize_act(A, 1, 1, 96, 96, None, 0, 1e-5, A, A, A, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_rmsnorm_quantize_act(A, 1, 1, 64, 64, A + 8, 0, 1e-5, A, A, A,
+                                            None) == bl.BL_ERR_ALIGN
+    P = ctypes.c_void_p * 1
+    I = ctypes.c_int64 * 1
+    pk, sc, ys = P(A), P(A), P(A)
+    assert L.bitlinear_rmsnorm_gemv_fused_multi(1, pk, sc, I(64), 256, None, 1, None, 0, 1e-5, ys, 1,
+                                                I(64), None, 0, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_rmsnorm_gemv_fused_multi(0, pk, sc, I(64), 256, A, 1, None, 0, 1e-5, ys, 1,
+                                                I(64), None, 0, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_rmsnorm_gemv_fused_multi(1, pk, sc, I(64), 256, A, 1, None, 0, -2.0, ys, 1,
+                                                I(64), None, 0, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_rmsnorm_gemv_fused_multi(1, pk, sc, I(64), 256, A, 1, None, 0, 1e-5, ys, 1,
+                                                I(64), None, 4, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_rmsnorm_gemv_fused_multi(1, pk, sc, I(64), 256, A + 4, 1, None, 0, 1e-5, ys,
+                                                1, I(64), None, 0, None) == bl.BL_ERR_ALIGN
+
+
+def test_bitplane_sizes_and_argument_errors(bl):
+    A = 0x7f0000000000
+    L = bl.lib
+    assert L.bitlinear_bitplane_bytes(28672, 8192) == 28672 * 128 * 16
+    assert L.bitlinear_bitplane_bytes(8, 96) == 0
+    assert L.bitlinear_bitplane_pack(None, 8, 64, A, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_bitplane_pack(A, 8, 65600, A, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_bitplane_pack(A + 8, 8, 64, A, None) == bl.BL_ERR_ALIGN
+    assert L.bitlinear_bitplane_gemv(A, A, 8, 64, None, 1, A, 1, None, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_bitplane_gemv(A, A, 8, 64, A, 3, A, 1, None, None) == bl.BL_ERR_DTYPE
+    assert L.bitlinear_bitplane_gemv(A, A, 8, 131072, A, 1, A, 1, None, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_bitplane_gemv(A, A, 8, 64, A + 2, 1, A, 1, None, None) == bl.BL_ERR_ALIGN
+
+
+def test_lut_gemv_argument_errors(bl):
+    A = 0x7f0000000000
+    L = bl.lib
+    assert L.bitlinear_lut_gemv(A, A, 8, 64, None, A, A, 1, None, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_lut_gemv(A, A, 8, 64, A, A, A, 5, None, None) == bl.BL_ERR_DTYPE
+    assert L.bitlinear_lut_gemv(A, A, 8, 12352, A, A, A, 1, None, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_lut_gemv(A, A, 8, 64, A, A + 2, A, 1, None, None) == bl.BL_ERR_ALIGN
