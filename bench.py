@@ -8,16 +8,19 @@ BitLinear products of a 2.4B-parameter BitNet b1.58 model -- per layer q/o
 (6912 -> 2560) -- for 30 layers, every product with its own packed ternary
 weight (521 MB of distinct weights per step, more than four times the 126 MB
 L2, so every step streams from HBM and no flush is needed).  Each layer is
-four launches of the fused GEMV (absmax int8 quantisation of x, ternary
-product with int32 accumulation, rescale, bf16 out): q/k/v in one launch and
+four steps of the fused GEMV (absmax int8 quantisation of x, ternary
+product with int32 accumulation, rescale, bf16 out): q/k/v in one step and
 gate/up in one, since each group shares its input, then o and down -- 120
-launches per step.  Each launch reads the output of the one before it, as in a
+steps per token.  Each step reads the output of the one before it, as in a
 decoder (o reads q, gate/up read o's output, down reads gate's output, the
-next layer reads down's output), so the chain is truly dependent; launches
-use programmatic dependent launch (a launch fetches its weights while the
-previous one finishes, and reads x only after it) and are replayed from a CUDA
-graph captured through the public Python API.  The end-to-end figure copies
-the token's input in and its final output back every step.
+next layer reads down's output), so the chain is truly dependent.  The whole
+chain runs as ONE persistent cooperative launch (DecodeChain: every CTA's
+producer warp streams its weights for all steps ahead, consumers start a step
+when every CTA has finished the previous one), replayed from a CUDA graph
+captured through the public Python API; the same steps as 120 launches with
+programmatic dependent launch are timed beside it (per_launch_pdl, or
+--per-launch for the headline).  The end-to-end figure copies the token's
+input in and its final output back every step.
 
 Metric: effective weight bandwidth, packed weight bytes / device time, GB/s,
 against the measured HBM copy bandwidth.  Inputs are synthetic and seeded
@@ -55,8 +58,9 @@ import synth_inputs as si  # noqa: E402
 METRIC = "decode ternary GEMV effective weight GB/s (% of HBM peak); prefill int8 TOPS"
 WORKLOAD = ("decode GEMV M=1, BitNet b1.58 2.4B layer shapes (q/o 2560->2560, k/v 2560->640, "
             "gate/up 2560->6912, down 6912->2560) x 30 layers, distinct packed weights per "
-            "layer, fused int8 absmax quantisation, bf16 in/out; per layer 4 dependent launches "
-            "(qkv, o, gate+up, down; products sharing x fused) with programmatic dependent launch")
+            "layer, fused int8 absmax quantisation, bf16 in/out; per layer 4 dependent steps "
+            "(qkv, o, gate+up, down; products sharing x fused), the token's 120 steps in one "
+            "persistent launch")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -72,13 +76,18 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def profiled_traffic():
-    """DRAM bytes per GEMV launch from the committed ncu summary, or None when
-    the kernel source has changed since those counters were taken."""
+def profiled_traffic(chain: bool = True):
+    """DRAM bytes per launch of the timed kernel from the committed ncu
+    summary, or None when the kernel source has changed since those counters
+    were taken."""
     import hashlib
     import re
-    prof = os.path.join(ROOT, "profiles", "decode_stream_2b_gemv_launches.md")
-    src = os.path.join(ROOT, "bit_ternary_weight_b200", "csrc", "gemv_stream.cu")
+    if chain:
+        prof = os.path.join(ROOT, "profiles", "decode_chain_2b_launches.md")
+        src = os.path.join(ROOT, "bit_ternary_weight_b200", "csrc", "gemv_chain.cu")
+    else:
+        prof = os.path.join(ROOT, "profiles", "decode_stream_2b_gemv_launches.md")
+        src = os.path.join(ROOT, "bit_ternary_weight_b200", "csrc", "gemv_stream.cu")
     try:
         text = open(prof).read()
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
@@ -412,6 +421,84 @@ def isolated_binary(bl, K, N, iters=100, device="cuda"):
     return {"K": K, "N": N, "us": t * 1e6, "GBps": nbytes / t / 1e9, "weight_copies": copies}
 
 
+def _graph_time(calls, iters):
+    """Per-call device time of `calls` (a list of thunks, cycled) replayed
+    from one CUDA graph of `iters` launches."""
+    for c in calls[:min(len(calls), 4)]:
+        c()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(iters):
+            calls[i % len(calls)]()
+    g.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    g.replay()
+    e.record()
+    torch.cuda.synchronize()
+    del g
+    return s.elapsed_time(e) / 1000.0 / iters
+
+
+def _weight_copies(bl, K, N, nbytes, seed0, device, limit=400):
+    copies = min(limit, max(2, int((4 * 126e6) // nbytes) + 1))
+    gen = torch.Generator(device=device)
+    ws = []
+    for c in range(copies):
+        gen.manual_seed(seed0 + c)
+        W = torch.randn(N, K, generator=gen, device=device) * 0.02
+        ws.append(bl.pack(W))
+        del W
+    return ws
+
+
+def isolated_bitplane(bl, K, N, iters=100, device="cuda"):
+    """Ternary x 1-bit bit-plane GEMV (N*K/4 bytes of planes), weights
+    rotated beyond L2."""
+    nbytes = N * K // 4
+    ws = [bl.bitplane_pack(w) for w in _weight_copies(bl, K, N, nbytes, 13, device)]
+    x = si.activations(1, K, seed=5).to(device)
+    y = torch.empty(N, dtype=torch.bfloat16, device=device)
+    t = _graph_time([lambda w=w: bl.bitplane_gemv(w, x, out=y) for w in ws], iters)
+    return {"K": K, "N": N, "us": t * 1e6, "GBps": nbytes / t / 1e9, "weight_copies": len(ws)}
+
+
+def lut_vs_dp4a(bl, K, N, iters=100, device="cuda"):
+    """Table-lookup GEMV against the dp4a GEMV on the same pre-quantised token
+    and the same rotated weights."""
+    nbytes = bl.packed_bytes(N, K)
+    ws = _weight_copies(bl, K, N, nbytes, 17, device)
+    x = si.activations(1, K, seed=5).to(device)
+    q, d, r = bl.quantize_act(x)
+    y = torch.empty(1, N, dtype=torch.bfloat16, device=device)
+    t_lut = _graph_time([lambda w=w: bl.lut_gemv(w, q, d, out=y) for w in ws], iters)
+    t_dp4a = _graph_time([lambda w=w: bl.gemv(w, q, d, r, out=y) for w in ws], iters)
+    return {"K": K, "N": N, "lut_us": t_lut * 1e6, "lut_GBps": nbytes / t_lut / 1e9,
+            "dp4a_us": t_dp4a * 1e6, "dp4a_GBps": nbytes / t_dp4a / 1e9,
+            "weight_copies": len(ws)}
+
+
+def rmsnorm_gemv_cost(bl, K, Ns, iters=200, device="cuda"):
+    """RMSNorm + quantise + products sharing the token in one launch, against
+    the same launch without RMSNorm (same rotated weights)."""
+    per = sum(bl.packed_bytes(N, K) for N in Ns)
+    sets = []
+    for c in range(min(400, max(2, int((4 * 126e6) // per) + 1))):
+        gen = torch.Generator(device=device)
+        gen.manual_seed(23 + c)
+        sets.append([bl.pack(torch.randn(N, K, generator=gen, device=device) * 0.02) for N in Ns])
+    x = si.activations(1, K, seed=5).to(device)
+    gain = (1.0 + 0.1 * torch.randn(K, device=device)).to(torch.bfloat16)
+    outs = [torch.empty(1, N, dtype=torch.bfloat16, device=device) for N in Ns]
+    t_norm = _graph_time([lambda ws=ws: bl.rmsnorm_gemv_fused_multi(ws, x, gain, outs=outs)
+                          for ws in sets], iters)
+    t_plain = _graph_time([lambda ws=ws: bl.gemv_fused_multi(ws, x, outs=outs) for ws in sets], iters)
+    return {"K": K, "N": Ns, "rmsnorm_us": t_norm * 1e6, "plain_us": t_plain * 1e6,
+            "rmsnorm_GBps": per / t_norm / 1e9, "plain_GBps": per / t_plain / 1e9}
+
+
 def prefill_gemm(bl, K, N, M, iters=20, device="cuda"):
     gen = torch.Generator(device=device)
     gen.manual_seed(3)
@@ -425,7 +512,8 @@ def prefill_gemm(bl, K, N, M, iters=20, device="cuda"):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
     bl.gemm(w, q, d, r, out=y, workspace=ws)
     torch.cuda.synchronize()
-    times, qtimes = [], []
+    gain = (1.0 + 0.1 * torch.randn(K, generator=gen, device=device)).to(torch.bfloat16)
+    times, qtimes, ntimes = [], [], []
     for _ in range(iters):
         flush.zero_()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -435,16 +523,24 @@ def prefill_gemm(bl, K, N, M, iters=20, device="cuda"):
         flush.zero_()
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s2.record()
-        bl.quantize_act(x)
+        bl.quantize_act(x, out=(q, d, r))
         e2.record()
+        flush.zero_()
+        s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s3.record()
+        bl.rmsnorm_quantize_act(x, gain, out=(q, d, r))
+        e3.record()
         torch.cuda.synchronize()
         times.append(s.elapsed_time(e) / 1000.0)
         qtimes.append(s2.elapsed_time(e2) / 1000.0)
+        ntimes.append(s3.elapsed_time(e3) / 1000.0)
     t = statistics.median(times)
     tq = statistics.median(qtimes)
+    tn = statistics.median(ntimes)
     ops = 2.0 * M * N * K
     return {"M": M, "K": K, "N": N, "gemm_us": t * 1e6, "TOPS": ops / t / 1e12,
             "quant_us": tq * 1e6, "quant_GBps": M * K * 3 / tq / 1e9,
+            "rmsnorm_quant_us": tn * 1e6, "rmsnorm_quant_GBps": M * K * 3 / tn / 1e9,
             "TOPS_incl_quant": ops / (t + tq) / 1e12}
 
 
@@ -536,9 +632,15 @@ def run_ours(args, world, rank, local):
     else:
         launches, xs, ys, host_x, step_bytes = build_stream(bl, args.layers, seed=rank, device=device)
         rank_bytes = step_bytes
-        step = lambda: run_step(bl, launches)  # noqa: E731
+        if args.per_launch:
+            step = lambda: run_step(bl, launches)  # noqa: E731
+        else:
+            # the token's whole chain in one persistent launch
+            chain = bl.DecodeChain([bl.ChainStep(ws, x, outs) for (ws, x, outs) in launches])
+            step = chain.run
     # xs: the token's input (copied in every e2e step); ys: its final output
-    launches_per_step = len(launches)
+    products_per_step = len(launches)
+    kernel_launches_per_step = products_per_step if (args.split or args.per_launch) else 1
     # eager warm-up through the public API, then capture the step
     for _ in range(2):
         step()
@@ -595,6 +697,23 @@ def run_ours(args, world, rank, local):
     t_eager = s.elapsed_time(e) / 1000.0
     del graph
 
+    # the same step as one launch per product (PDL, graph), for comparison
+    per_launch = None
+    if not args.split and not args.per_launch:
+        g2 = torch.cuda.CUDAGraph()
+        run_step(bl, launches)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g2):
+            run_step(bl, launches)
+        for _ in range(args.warmup):
+            g2.replay()
+        t_pl = max_over_ranks(time_graph(g2, args.steps, world), world)
+        per_launch = {"GBps": job_throughput(step_bytes, args.steps, world, t_pl),
+                      "ms_per_step": t_pl / args.steps * 1000,
+                      "launches_per_step": products_per_step,
+                      "how": "one gemv_fused_multi launch per step of the chain, PDL, CUDA graph"}
+        del g2
+
     extra = {}
     if rank == 0 and not args.no_extra and not args.split:
         def measure(key, fn):
@@ -611,6 +730,13 @@ def run_ours(args, world, rank, local):
         measure("small_batch_2560x6912", lambda: [
             isolated_gemv(bl, 2560, 6912, M=m, iters=100, device=device) for m in si.SMALL_BATCH_M])
         measure("binary_100b", lambda: isolated_binary(bl, 8192, 28672, device=device))
+        measure("bitplane_100b", lambda: [isolated_bitplane(bl, K, N, device=device)
+                                          for (K, N) in si.DECODE_SHAPES_100B])
+        measure("lut_vs_dp4a", lambda: [lut_vs_dp4a(bl, K, N, device=device)
+                                        for (K, N) in si.DECODE_SHAPES_2B + [(8192, 28672)]])
+        measure("rmsnorm_gemv", lambda: [rmsnorm_gemv_cost(bl, 2560, [6912, 6912], device=device),
+                                         rmsnorm_gemv_cost(bl, 2560, [2560, 640, 640], device=device),
+                                         rmsnorm_gemv_cost(bl, 8192, [28672], device=device)])
         measure("prefill", lambda: [prefill_gemm(bl, K, N, M, device=device)
                                     for (K, N) in si.PREFILL_SHAPES for M in si.PREFILL_TOKENS])
 
@@ -627,7 +753,8 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "int8", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) bf16 x with 0.1% x20 outliers)",
         "config": {"workload": WORKLOAD, "layers": args.layers,
-                   "launches_per_step": launches_per_step,
+                   "products_per_step": products_per_step,
+                   "launches_per_step": kernel_launches_per_step,
                    "weight_bytes_per_step": step_bytes,
                    "weight_bytes_per_step_per_rank": rank_bytes,
                    "l2": "inputs larger than L2: 521 MB of distinct packed weights per step",
@@ -637,11 +764,14 @@ def run_ours(args, world, rank, local):
                                   f"{world} independent replicas (weak scaling)"},
         "roofline": {"bound": "hbm", "achieved": rank_bytes * args.steps / t / 1e9, "peak": hbm,
                      "unit": "GB/s", "frac": rank_bytes * args.steps / t / 1e9 / hbm,
-                     "traffic": profiled_traffic(),
+                     "traffic": profiled_traffic(chain=kernel_launches_per_step == 1),
                      "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                     "kernel": "gemv_stream_kernel<KC=8, bf16 fused> (4 launches per layer)",
+                     "kernel": ("gemv_chain_kernel (one persistent launch per token)"
+                                if kernel_launches_per_step == 1 else
+                                "gemv_stream_kernel<KC=8, bf16 fused> (4 launches per layer)"),
                      "note": "algorithmic bytes = packed weight bytes per launch; duration = "
-                             "step time / launches (CUDA events over the timed region)"},
+                             "step time / launches per step (CUDA events over the timed "
+                             "region, on the launching stream)"},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "GB/s",
                 "h2d_bytes_per_step": xs.numel() * xs.element_size(),
@@ -649,7 +779,8 @@ def run_ours(args, world, rank, local):
                 "how": "pinned host token input -> device, graph of the public-API "
                        "gemv_fused_multi chain, final output -> pinned host, CUDA events"},
         "e2e_eager_GBps": step_bytes * eager_steps / t_eager / 1e9,
-        "gpu_launches": launches_per_step * args.steps,
+        "per_launch_pdl": per_launch,
+        "gpu_launches": kernel_launches_per_step * args.steps,
         "clocks": clocks,
         "extra": extra,
     }
@@ -712,6 +843,9 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=2.0)
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-launch", action="store_true",
+                    help="time the step as one launch per product (PDL) instead of the "
+                         "persistent chain launch")
     ap.add_argument("--split", action="store_true",
                     help="split one model's products by output rows over the ranks "
                          "(column-parallel, all-gather of y per launch) instead of "

@@ -97,6 +97,31 @@ _SIGNATURES = {
     "bitlinear_last_device_status": (_int, [_vp]),
     "bitlinear_device_sm_count": (_int, []),
 }
+class ChainStepC(ctypes.Structure):
+    """Mirror of bitlinear_chain_step (include/bitlinear.h)."""
+    _fields_ = [("count", ctypes.c_int),
+                ("packed", ctypes.c_void_p * 8),
+                ("w_scale", ctypes.c_void_p * 8),
+                ("N", ctypes.c_int64 * 8),
+                ("y", ctypes.c_void_p * 8),
+                ("acc_dbg", ctypes.c_void_p * 8),
+                ("K", ctypes.c_int64),
+                ("x", ctypes.c_void_p),
+                ("xt", ctypes.c_int),
+                ("yt", ctypes.c_int),
+                ("norm", ctypes.c_int),
+                ("gain", ctypes.c_void_p),
+                ("gt", ctypes.c_int),
+                ("eps", ctypes.c_float)]
+
+
+_SIGNATURES.update({
+    "bitlinear_chain_plan_bytes": (_sz, [_int]),
+    "bitlinear_chain_plan": (_int, [_int, ctypes.POINTER(ChainStepC), _vp, _sz, _vp]),
+    "bitlinear_chain_run": (_int, [_vp, _int, _vp]),
+    "bitlinear_chain_run_timeout_test": (_int, [_vp, _int, ctypes.c_uint64, _vp]),
+})
+
 for _name, (_res, _args) in _SIGNATURES.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res
@@ -323,6 +348,73 @@ def rmsnorm_gemv_fused_multi(weights, x: torch.Tensor, gain=None, eps: float = R
             float(eps), ys, _dt(outs[0].dtype), ldys, accs, BL_FLAG_PDL if pdl else 0,
             _stream(x.device)), "bitlinear_rmsnorm_gemv_fused_multi")
     return outs
+
+
+@dataclass
+class ChainStep:
+    """One step of a decode chain: products sharing the token x (1 .. 8 weights
+    with the same K), each written to its output [N] (or [1, N]); RMSNorm in
+    front when `norm` or a gain is given."""
+    weights: list
+    x: torch.Tensor
+    outs: list
+    norm: bool = False
+    gain: torch.Tensor | None = None
+    eps: float = RMS_EPS
+    acc_dbgs: list | None = None
+
+
+class DecodeChain:
+    """A token's chain of dependent decode BitLinears run as ONE persistent
+    launch (bitlinear_chain_plan / bitlinear_chain_run).  The plan lives in a
+    device buffer owned by this object; the tensors the steps name must stay
+    alive and in place while the chain is used."""
+
+    def __init__(self, steps, device=None):
+        n = len(steps)
+        device = device or steps[0].x.device
+        arr = (ChainStepC * n)()
+        for i, st in enumerate(steps):
+            c = arr[i]
+            c.count = len(st.weights)
+            for j, (w, o) in enumerate(zip(st.weights, st.outs)):
+                c.packed[j] = w.packed.data_ptr()
+                c.w_scale[j] = w.w_scale.data_ptr()
+                c.N[j] = w.N
+                c.y[j] = o.data_ptr()
+                a = None if st.acc_dbgs is None else st.acc_dbgs[j]
+                c.acc_dbg[j] = 0 if a is None else a.data_ptr()
+            c.K = st.weights[0].K
+            c.x = st.x.data_ptr()
+            c.xt = _dt(st.x.dtype)
+            c.yt = _dt(st.outs[0].dtype)
+            c.norm = 1 if (st.norm or st.gain is not None) else 0
+            c.gain = 0 if st.gain is None else st.gain.data_ptr()
+            c.gt = BL_F32 if st.gain is None else _dt(st.gain.dtype)
+            c.eps = float(st.eps)
+        nbytes = int(_lib.bitlinear_chain_plan_bytes(n))
+        if nbytes == 0:
+            raise BitLinearError(BL_ERR_SHAPE, "bitlinear_chain_plan_bytes")
+        self.n = n
+        self.steps = steps
+        self.device = torch.device(device)
+        self.plan = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        with _on(self.device):
+            _check(_lib.bitlinear_chain_plan(n, arr, _ptr(self.plan), nbytes,
+                                             _stream(self.device)), "bitlinear_chain_plan")
+            torch.cuda.current_stream(self.device).synchronize()
+
+    def run(self):
+        with _on(self.device):
+            _check(_lib.bitlinear_chain_run(_ptr(self.plan), self.n, _stream(self.device)),
+                   "bitlinear_chain_run")
+
+    def run_timeout_test(self, wait_limit_ns: int = 1_000_000):
+        """Run with a wait that cannot complete (testing the timeout path)."""
+        with _on(self.device):
+            _check(_lib.bitlinear_chain_run_timeout_test(_ptr(self.plan), self.n, wait_limit_ns,
+                                                         _stream(self.device)),
+                   "bitlinear_chain_run_timeout_test")
 
 
 def gemm_workspace_bytes(M: int, N: int, K: int) -> int:

@@ -450,6 +450,92 @@ int bitlinear_rmsnorm_gemv_fused_multi(int count, const uint8_t *const *packed,
     return launch_gemv_stream(b, true, static_cast<cudaStream_t>(stream), gain, gt, eps, true);
 }
 
+size_t bitlinear_chain_plan_bytes(int nsteps) { return chain_plan_bytes(nsteps); }
+
+int bitlinear_chain_plan(int nsteps, const bitlinear_chain_step *steps, void *plan,
+                         size_t plan_bytes, void *stream)
+{
+    if (!steps || !plan)
+        return BL_ERR_NULL;
+    if (nsteps < 1 || nsteps > BITLINEAR_CHAIN_MAX_STEPS)
+        return BL_ERR_SHAPE;
+    int st;
+    for (int i = 0; i < nsteps; ++i) {
+        const bitlinear_chain_step &d = steps[i];
+        if (!d.x)
+            return BL_ERR_NULL;
+        if (d.count < 1 || d.count > kGemvMaxProblems)
+            return BL_ERR_SHAPE;
+        if (!valid_dtype(d.xt) || !valid_dtype(d.yt) || (d.gain && !valid_dtype(d.gt)))
+            return BL_ERR_DTYPE;
+        if (!chain_step_fits(d.K) || !(d.eps >= 0.0f) || !(d.eps <= 3.0e38f))
+            return BL_ERR_SHAPE;
+        for (int j = 0; j < d.count; ++j) {
+            if ((st = check_gemv_common(d.packed[j], d.w_scale[j], d.N[j], d.K, 1, d.y[j], d.yt,
+                                        d.N[j], 1)))
+                return st;
+            if (reinterpret_cast<uintptr_t>(d.acc_dbg[j]) & 3u)
+                return BL_ERR_ALIGN;
+        }
+        if (!aligned16(d.x) || !aligned16(d.gain))
+            return BL_ERR_ALIGN;
+    }
+    if (plan_bytes < chain_plan_bytes(nsteps))
+        return BL_ERR_WORKSPACE;
+    if (!aligned16(plan))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    if ((st = need_device(&di)))
+        return st;
+    if ((st = check_dev_ptrs({plan})))
+        return st;
+    for (int i = 0; i < nsteps; ++i) {
+        const bitlinear_chain_step &d = steps[i];
+        if ((st = check_dev_ptrs({d.x, d.gain})))
+            return st;
+        for (int j = 0; j < d.count; ++j)
+            if ((st = check_dev_ptrs({d.packed[j], d.w_scale[j], d.y[j], d.acc_dbg[j]})))
+                return st;
+    }
+    return build_chain_plan(nsteps, steps, plan, static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_chain_run(const void *plan, int nsteps, void *stream)
+{
+    if (!plan)
+        return BL_ERR_NULL;
+    if (nsteps < 1 || nsteps > BITLINEAR_CHAIN_MAX_STEPS)
+        return BL_ERR_SHAPE;
+    if (!aligned16(plan))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({plan})))
+        return st;
+    return launch_chain(plan, nsteps, static_cast<cudaStream_t>(stream), 2000000000ull, -1);
+}
+
+int bitlinear_chain_run_timeout_test(const void *plan, int nsteps, uint64_t wait_limit_ns,
+                                     void *stream)
+{
+    if (!plan)
+        return BL_ERR_NULL;
+    if (nsteps < 2 || nsteps > BITLINEAR_CHAIN_MAX_STEPS || wait_limit_ns < 1000 ||
+        wait_limit_ns > 2000000000ull)
+        return BL_ERR_SHAPE;
+    if (!aligned16(plan))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({plan})))
+        return st;
+    return launch_chain(plan, nsteps, static_cast<cudaStream_t>(stream), wait_limit_ns, 1);
+}
+
 size_t bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
     if (!valid_nk(N, K) || M < 1)

@@ -148,4 +148,10 @@ int launch_lut_gemv(const uint8_t *packed, const float *w_scale, int64_t N, int6
                     const int8_t *q, const float *d, void *y, int yt, int32_t *acc_dbg,
                     cudaStream_t s);
 
+// Persistent decode chain (gemv_chain.cu).
+size_t chain_plan_bytes(int nsteps);
+bool chain_step_fits(int64_t K);
+int build_chain_plan(int nsteps, const bitlinear_chain_step *steps, void *plan, cudaStream_t s);
+int launch_chain(const void *plan, int nsteps, cudaStream_t s, uint64_t limit_ns, int test_step);
+
 }  // namespace bl

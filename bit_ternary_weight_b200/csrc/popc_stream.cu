@@ -21,7 +21,9 @@
 //     on the stage's mbarrier.  The producer starts at once: the weights do
 //     not depend on x.
 //   * Eight consumer warps meanwhile build x's sign words in shared memory
-//     (two ballots per 64-bit word) and the block-wide max |x|, then take the
+//     (eight lanes per 64-bit word, eight elements each, combined with
+//     shuffles; all loads of a batch issued first) and the block-wide
+//     max |x|, then take the
 //     stage's rows in turn, one row per warp at a time: each lane XORs /
 //     popcounts 16-byte pieces of the row against the matching x words, and
 //     one warp reduction (redux.sync) gives the row's count.
@@ -79,15 +81,6 @@ __device__ __forceinline__ uint4 pc_lds128(uint32_t saddr)
 __device__ __forceinline__ uint64_t u64_of(uint32_t lo, uint32_t hi)
 {
     return (static_cast<uint64_t>(hi) << 32) | lo;
-}
-
-template <int XT>
-__device__ __forceinline__ float x_at(const void *x, int64_t k)
-{
-    if constexpr (XT == BL_BF16)
-        return __bfloat162float(static_cast<const __nv_bfloat16 *>(x)[k]);
-    else
-        return static_cast<const float *>(x)[k];
 }
 
 template <int VAR, int XT>
@@ -151,16 +144,41 @@ __global__ void __launch_bounds__(kPcThreads, 2) popc_stream_kernel(const PcPara
 
     // ---------------------------------------------------- consumer warps
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // x's sign words: eight lanes per 64-bit word, eight elements (one or two
+    // 16-byte loads) per lane, so a warp covers four words per step; the
+    // loads of kXBatch steps are issued before any of them is used
     const int words = int(p.K / 64);
+    constexpr int kXBatch = 4;
     float amax = 0.0f;
-    for (int w = warp; w < words; w += kPcConsumers) {
-        const float v0 = x_at<XT>(p.x, int64_t(w) * 64 + lane);
-        const float v1 = x_at<XT>(p.x, int64_t(w) * 64 + 32 + lane);
-        amax = fmaxf(amax, fmaxf(fabsf(v0), fabsf(v1)));
-        const unsigned lo = __ballot_sync(0xffffffffu, v0 < 0.0f);
-        const unsigned hi = __ballot_sync(0xffffffffu, v1 < 0.0f);
-        if (lane == 0)
-            xw[w] = u64_of(lo, hi);
+    const int sub = lane & 7;
+    for (int w0 = warp * 4; w0 < words; w0 += kPcConsumers * 4 * kXBatch) {
+        float f[kXBatch][8];
+#pragma unroll
+        for (int b = 0; b < kXBatch; ++b) {
+            const int w = w0 + b * kPcConsumers * 4 + (lane >> 3);
+            if (w < words)
+                load8<XT, true>(p.x, int64_t(w) * 64 + sub * 8, f[b]);
+            else
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    f[b][e] = 0.0f;
+        }
+#pragma unroll
+        for (int b = 0; b < kXBatch; ++b) {
+            const int w = w0 + b * kPcConsumers * 4 + (lane >> 3);
+            uint32_t neg = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                amax = fmaxf(amax, fabsf(f[b][e]));
+                neg |= uint32_t(f[b][e] < 0.0f) << e;
+            }
+            uint64_t word = static_cast<uint64_t>(neg) << (8 * sub);
+            word |= __shfl_xor_sync(0xffffffffu, word, 1);
+            word |= __shfl_xor_sync(0xffffffffu, word, 2);
+            word |= __shfl_xor_sync(0xffffffffu, word, 4);
+            if (sub == 0 && w < words)
+                xw[w] = word;
+        }
     }
     // maxima are >= 0 and finite (fmaxf from 0 drops NaN): bit patterns order like the values
     amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));

@@ -15,8 +15,8 @@
 // (and more bytes of x) are in flight per SM: the kernel's time per token is
 // mostly load latency.
 //
-// Many tokens (prefill) run a second kernel, row_quant_kernel, which can also
-// normalise each row first (RMSNorm; the "bit-floor" README, section "What's
+// RMSNorm in front of the quantiser runs a second kernel, row_quant_kernel
+// (RMSNorm; the "bit-floor" README, section "What's
 // inside": rmsnorm.cu reduces the mean square and applies an rsqrt scale per
 // element).  One warp per token, with no block-wide barrier on the token's
 // path: lane 0 brings the whole row into a shared-memory slot of the warp
@@ -423,20 +423,12 @@ int launch_row_quant(const void *x, int xt, int64_t M, int64_t K, int64_t ldx, c
 
 }  // namespace
 
-// Tokens from which the warp-per-token kernel runs plain quantisation: with
-// fewer, a CTA per token (128 threads on one row) has the shorter latency.
-constexpr int64_t kRowQuantMinTokensPerSm = 2;
-
+// Plain quantisation runs the CTA-per-token kernel: measured against the
+// warp-per-token kernel at 8192 tokens it was as fast at K = 2560 and faster
+// at K = 6912 (more warps per SM with the row in registers).
 int launch_quantize_act(const void *x, int xt, int64_t M, int64_t K, int64_t ldx,
                         int8_t *q, float *d, int32_t *rowsum, cudaStream_t s)
 {
-    const DeviceInfo *di = device_info();
-    if (!di)
-        return BL_ERR_CUDA;
-    const size_t row_bytes = size_t(K) * (xt == BL_BF16 ? 2 : 4);
-    int w = 0, sl = 0;
-    if (M >= kRowQuantMinTokensPerSm * di->sm_count && row_geometry(row_bytes, 0, &w, &sl))
-        return launch_row_quant(x, xt, M, K, ldx, nullptr, BL_F32, 0.0f, false, q, d, rowsum, s);
     dim3 grid(static_cast<unsigned>(M));
     if (xt == BL_BF16)
         quantize_act_kernel<BL_BF16><<<grid, kQuantThreads, 0, s>>>(x, K, ldx, q, d, rowsum);

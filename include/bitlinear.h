@@ -278,6 +278,80 @@ int bitlinear_rmsnorm_gemv_fused_multi(int count, const uint8_t *const *packed,
                                        void *stream);
 
 /*
+ * One step of a decode chain: `count` BitLinears sharing the token x (as in
+ * bitlinear_gemv_fused_multi with M = 1), RMSNorm first when `norm` is set or
+ * a gain is given.  All pointers are device pointers except the struct itself.
+ */
+typedef struct {
+    int count;                                          /* 1 .. BITLINEAR_GEMV_MAX_PROBLEMS */
+    const uint8_t *packed[BITLINEAR_GEMV_MAX_PROBLEMS]; /* from bitlinear_pack */
+    const float *w_scale[BITLINEAR_GEMV_MAX_PROBLEMS];
+    int64_t N[BITLINEAR_GEMV_MAX_PROBLEMS];
+    void *y[BITLINEAR_GEMV_MAX_PROBLEMS];               /* [N[i]] of dtype yt */
+    int32_t *acc_dbg[BITLINEAR_GEMV_MAX_PROBLEMS];      /* NULL or [N[i]] int32 */
+    int64_t K;                                          /* a multiple of 256, <= 16384 */
+    const void *x;                                      /* [K] of dtype xt */
+    int xt, yt;                                         /* BL_F32 or BL_BF16 */
+    int norm;                                           /* nonzero: RMSNorm x first */
+    const void *gain;                                   /* NULL or [K] of dtype gt */
+    int gt;
+    float eps;                                          /* RMSNorm epsilon, >= 0 */
+} bitlinear_chain_step;
+
+/* Most steps one chain may hold. */
+#define BITLINEAR_CHAIN_MAX_STEPS 4096
+
+/* Bytes of device memory a plan of `nsteps` steps needs (0 if out of range). */
+size_t bitlinear_chain_plan_bytes(int nsteps);
+
+/*
+ * Prepare a decode chain: the steps of one token, each reading the output of
+ * an earlier step (or the token's input), to be run as ONE persistent launch
+ * by bitlinear_chain_run.  Source: "How to Run BitNet Inference on GPU Using
+ * CUDA Kernels", sections "Understanding the Two-Phase Architecture" (the
+ * decode phase chains memory-bound INT8 x INT2 linears through Attention and
+ * FeedForward) and "Key Components and Source Code Architecture" (CUDA graphs
+ * to remove launch overhead).  Every step computes exactly what
+ * bitlinear_gemv_fused_multi (or, with norm, bitlinear_rmsnorm_gemv_fused_multi)
+ * computes on the same arguments.
+ *   steps     host array of nsteps descriptors, read during the call only
+ *   plan      device buffer of at least bitlinear_chain_plan_bytes(nsteps),
+ *             16-byte aligned, owned by the caller; written here (a copy
+ *             from host memory on `stream`), read and updated by every run
+ * A step's outputs must not overlap its own input x.  Make the plan outside
+ * stream capture; runs may be captured.  Errors: BL_ERR_SHAPE for a K that
+ * is not a multiple of 256 or above 16384, more than 64 row groups of 8 per
+ * SM in one step, or nsteps out of range; the usual checks otherwise.
+ */
+int bitlinear_chain_plan(int nsteps, const bitlinear_chain_step *steps,
+                         void *plan, size_t plan_bytes, void *stream);
+
+/*
+ * Run a prepared chain: one cooperative launch (one CTA per SM, all resident)
+ * after a reset of the plan's step counters, both on `stream`.  Each CTA owns
+ * a slice of every step's rows; its producer warp streams the weights of all
+ * steps ahead through shared memory, and its consumers start step s once all
+ * CTAs have finished step s - 1.  Every wait is bounded (2 s): a timeout is
+ * reported by the next bitlinear_last_device_status() as BL_ERR_TIMEOUT and
+ * leaves the outputs of the unfinished steps unspecified.  Runs of one plan
+ * must be ordered (one stream); the buffers the plan names must stay alive.
+ *   plan, nsteps   as given to bitlinear_chain_plan
+ */
+int bitlinear_chain_run(const void *plan, int nsteps, void *stream);
+
+/*
+ * For testing failure handling without a GPU fault: runs the chain with its
+ * bounded waits limited to wait_limit_ns (1 us .. 2 s) and with the wait
+ * before step 1 expecting one more arrival than there are CTAs, a count
+ * nothing reaches.  That wait runs out, the grid leaves through its abort
+ * path, and the next bitlinear_last_device_status() returns BL_ERR_TIMEOUT;
+ * the device stays usable.  Step 0's outputs are complete, later outputs
+ * unspecified.  nsteps >= 2.
+ */
+int bitlinear_chain_run_timeout_test(const void *plan, int nsteps,
+                                     uint64_t wait_limit_ns, void *stream);
+
+/*
  * Bytes of workspace bitlinear_gemm needs for this problem (0 if none).
  * Nonzero for small batches (M <= 32) whose output tiles alone would leave
  * SMs idle: K is then split across CTAs and the int32 partial sums meet in

@@ -176,3 +176,60 @@ def test_lut_gemv_argument_errors(bl):
     assert L.bitlinear_lut_gemv(A, A, 8, 64, A, A, A, 5, None, None) == bl.BL_ERR_DTYPE
     assert L.bitlinear_lut_gemv(A, A, 8, 12352, A, A, A, 1, None, None) == bl.BL_ERR_SHAPE
     assert L.bitlinear_lut_gemv(A, A, 8, 64, A, A + 2, A, 1, None, None) == bl.BL_ERR_ALIGN
+
+
+def test_chain_step_struct_matches_the_header(bl, tmp_path):
+    """The binding's ctypes mirror of bitlinear_chain_step has the C layout."""
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("no C compiler")
+    fields = [f[0] for f in bl.ChainStepC._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "bitlinear.h"\nint main(void){'
+                   'printf("%zu", sizeof(bitlinear_chain_step));'
+                   + "".join(f'printf(" %zu", offsetof(bitlinear_chain_step, {f}));' for f in fields)
+                   + "return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    want = [ctypes.sizeof(bl.ChainStepC)] + [getattr(bl.ChainStepC, f).offset for f in fields]
+    assert got == want
+
+
+def test_chain_argument_errors(bl):
+    L = bl.lib
+    assert L.bitlinear_chain_plan_bytes(0) == 0
+    assert L.bitlinear_chain_plan_bytes(4097) == 0
+    assert L.bitlinear_chain_plan_bytes(120) > 120 * ctypes.sizeof(bl.ChainStepC)
+    A = 0x7f0000000000
+    st = (bl.ChainStepC * 1)()
+    st[0].count = 1
+    st[0].packed[0] = A
+    st[0].w_scale[0] = A
+    st[0].N[0] = 64
+    st[0].y[0] = A
+    st[0].K = 2560
+    st[0].x = A
+    st[0].xt = st[0].yt = 1
+    nb = L.bitlinear_chain_plan_bytes(1)
+    assert L.bitlinear_chain_plan(1, st, None, nb, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_chain_plan(0, st, A, nb, None) == bl.BL_ERR_SHAPE
+    st[0].K = 2304 + 64     # not a multiple of 256
+    assert L.bitlinear_chain_plan(1, st, A, nb, None) == bl.BL_ERR_SHAPE
+    st[0].K = 32768         # above the chain's 16384
+    assert L.bitlinear_chain_plan(1, st, A, nb, None) == bl.BL_ERR_SHAPE
+    st[0].K = 2560
+    st[0].eps = -1.0
+    assert L.bitlinear_chain_plan(1, st, A, nb, None) == bl.BL_ERR_SHAPE
+    st[0].eps = 1e-5
+    st[0].xt = 9
+    assert L.bitlinear_chain_plan(1, st, A, nb, None) == bl.BL_ERR_DTYPE
+    st[0].xt = 1
+    assert L.bitlinear_chain_plan(1, st, A, nb - 1, None) == bl.BL_ERR_WORKSPACE
+    assert L.bitlinear_chain_plan(1, st, A + 8, nb, None) == bl.BL_ERR_ALIGN
+    assert L.bitlinear_chain_run(None, 1, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_chain_run(A, 0, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_chain_run_timeout_test(A, 1, 1000000, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_chain_run_timeout_test(A, 2, 10, None) == bl.BL_ERR_SHAPE
