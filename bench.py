@@ -13,14 +13,15 @@ product with int32 accumulation, rescale, bf16 out): q/k/v in one step and
 gate/up in one, since each group shares its input, then o and down -- 120
 steps per token.  Each step reads the output of the one before it, as in a
 decoder (o reads q, gate/up read o's output, down reads gate's output, the
-next layer reads down's output), so the chain is truly dependent.  The whole
-chain runs as ONE persistent cooperative launch (DecodeChain: every CTA's
-producer warp streams its weights for all steps ahead, consumers start a step
-when every CTA has finished the previous one), replayed from a CUDA graph
-captured through the public Python API; the same steps as 120 launches with
-programmatic dependent launch are timed beside it (per_launch_pdl, or
---per-launch for the headline).  The end-to-end figure copies the token's
-input in and its final output back every step.
+next layer reads down's output), so the chain is truly dependent.  Each step
+is one launch with programmatic dependent launch (a launch fetches its weights
+while the previous one finishes, and reads x only after it), the 120 launches
+replayed from a CUDA graph captured through the public Python API.  The same
+token as ONE persistent cooperative launch (DecodeChain: producer warps stream
+every step's weights ahead, a software grid barrier between steps) is timed
+beside it (persistent_chain, or --chain for the headline); on B200 it is the
+slower of the two.  The end-to-end figure copies the token's input in and its
+final output back every step.
 
 Metric: effective weight bandwidth, packed weight bytes / device time, GB/s,
 against the measured HBM copy bandwidth.  Inputs are synthetic and seeded
@@ -59,8 +60,8 @@ METRIC = "decode ternary GEMV effective weight GB/s (% of HBM peak); prefill int
 WORKLOAD = ("decode GEMV M=1, BitNet b1.58 2.4B layer shapes (q/o 2560->2560, k/v 2560->640, "
             "gate/up 2560->6912, down 6912->2560) x 30 layers, distinct packed weights per "
             "layer, fused int8 absmax quantisation, bf16 in/out; per layer 4 dependent steps "
-            "(qkv, o, gate+up, down; products sharing x fused), the token's 120 steps in one "
-            "persistent launch")
+            "(qkv, o, gate+up, down; products sharing x fused), one launch each with "
+            "programmatic dependent launch")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -632,15 +633,15 @@ def run_ours(args, world, rank, local):
     else:
         launches, xs, ys, host_x, step_bytes = build_stream(bl, args.layers, seed=rank, device=device)
         rank_bytes = step_bytes
-        if args.per_launch:
-            step = lambda: run_step(bl, launches)  # noqa: E731
-        else:
+        if args.chain:
             # the token's whole chain in one persistent launch
             chain = bl.DecodeChain([bl.ChainStep(ws, x, outs) for (ws, x, outs) in launches])
             step = chain.run
+        else:
+            step = lambda: run_step(bl, launches)  # noqa: E731
     # xs: the token's input (copied in every e2e step); ys: its final output
     products_per_step = len(launches)
-    kernel_launches_per_step = products_per_step if (args.split or args.per_launch) else 1
+    kernel_launches_per_step = 1 if (args.chain and not args.split) else products_per_step
     # eager warm-up through the public API, then capture the step
     for _ in range(2):
         step()
@@ -697,21 +698,22 @@ def run_ours(args, world, rank, local):
     t_eager = s.elapsed_time(e) / 1000.0
     del graph
 
-    # the same step as one launch per product (PDL, graph), for comparison
-    per_launch = None
-    if not args.split and not args.per_launch:
-        g2 = torch.cuda.CUDAGraph()
-        run_step(bl, launches)
+    # the same token as ONE persistent launch (DecodeChain), for comparison
+    other = None
+    if not args.split and not args.chain:
+        chain = bl.DecodeChain([bl.ChainStep(ws, x, outs) for (ws, x, outs) in launches])
+        chain.run()
         torch.cuda.synchronize()
+        g2 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g2):
-            run_step(bl, launches)
+            chain.run()
         for _ in range(args.warmup):
             g2.replay()
-        t_pl = max_over_ranks(time_graph(g2, args.steps, world), world)
-        per_launch = {"GBps": job_throughput(step_bytes, args.steps, world, t_pl),
-                      "ms_per_step": t_pl / args.steps * 1000,
-                      "launches_per_step": products_per_step,
-                      "how": "one gemv_fused_multi launch per step of the chain, PDL, CUDA graph"}
+        t_ch = max_over_ranks(time_graph(g2, args.steps, world), world)
+        other = {"GBps": job_throughput(step_bytes, args.steps, world, t_ch),
+                 "ms_per_step": t_ch / args.steps * 1000, "launches_per_step": 1,
+                 "how": "DecodeChain: the token's 120 steps in one persistent cooperative "
+                        "launch (software grid barrier per step), CUDA graph"}
         del g2
 
     extra = {}
@@ -779,7 +781,7 @@ def run_ours(args, world, rank, local):
                 "how": "pinned host token input -> device, graph of the public-API "
                        "gemv_fused_multi chain, final output -> pinned host, CUDA events"},
         "e2e_eager_GBps": step_bytes * eager_steps / t_eager / 1e9,
-        "per_launch_pdl": per_launch,
+        "persistent_chain": other,
         "gpu_launches": kernel_launches_per_step * args.steps,
         "clocks": clocks,
         "extra": extra,
@@ -843,9 +845,9 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=2.0)
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--per-launch", action="store_true",
-                    help="time the step as one launch per product (PDL) instead of the "
-                         "persistent chain launch")
+    ap.add_argument("--chain", action="store_true",
+                    help="time the step as one persistent launch (DecodeChain) instead of "
+                         "one launch per product with programmatic dependent launch")
     ap.add_argument("--split", action="store_true",
                     help="split one model's products by output rows over the ranks "
                          "(column-parallel, all-gather of y per launch) instead of "

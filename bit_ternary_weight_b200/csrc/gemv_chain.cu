@@ -21,19 +21,29 @@
 //     stage, from different lanes), never waiting on activations: it runs
 //     as far ahead of the consumers, across step boundaries, as the ring
 //     allows.
-//   * The eight consumer warps take one step at a time: wait until every CTA
+//   * The sixteen consumer warps take one step at a time: wait until every CTA
 //     has finished the previous step (a per-step arrival counter in the
-//     plan, polled with acquire loads by one thread), read x from L2,
+//     plan, polled by one thread, then an acquire fence), read x from L2,
 //     quantise it (the prologues of the one-token streaming kernel), consume
 //     the step's stages, fold the partial row sums, rescale and store their
-//     rows of y, and arrive on the step's counter (release: block barrier,
-//     fence, atomic add).
+//     rows of y, and arrive on the step's counter (block barrier, then one
+//     release reduction).
 //   * Every wait -- mbarriers and counters -- is bounded (2 s of
 //     %globaltimer); a CTA that gives up records BL_ERR_TIMEOUT in the device
 //     status word and raises the plan's abort word, which every other wait
 //     checks, so the whole grid leaves promptly; the producer waits (bounded)
 //     for its copies in flight before its CTA exits.
 // The host zeroes the counters and the abort word before every launch.
+//
+// Measured on B200 (2.4B decode stream, 120 steps, %globaltimer stamps per
+// CTA and step): a step costs ~0.9 us from the last arrival to the release of
+// the waiting CTAs, ~1.1 us of prologue (x from L2, absmax, quantise), the
+// stage work, ~0.35 us of stores and ~0.55 us for the release reduction to
+// retire behind them: 4.0-6.5 us per step, against ~3.1 us per launch when
+// every step is its own launch chained with programmatic dependent launch,
+// whose hand-off the hardware does faster than this software grid barrier.
+// The chain is exact and needs one launch per token; the per-launch chain is
+// the faster way to run a decode step here.
 #include <vector>
 
 #include "gemv_stream_common.cuh"
@@ -41,17 +51,17 @@
 namespace bl {
 namespace {
 
-constexpr int kChainKC = 8;                       // consumer warps
+constexpr int kChainKC = 16;                      // consumer warps
 constexpr int kChainThreads = 32 * (kChainKC + 1);
 constexpr int kChainStages = 6;
 constexpr uint32_t kChainStageBytes = 32 * 1024;
 constexpr int64_t kChainMaxK = 16384;             // int8 activations staged in shared memory
 constexpr int kChainMaxStepsLimit = 4096;
 
-// One step of the chain (device memory).  The field names the activation
-// prologues read (x, K, q, d, rowsum, gain, gt, eps) are those of
-// StreamParams.
-struct ChainStep {
+// One step of the chain (device memory; the consumers work from a copy in
+// shared memory).  The field names the activation prologues read (x, K, q,
+// d, rowsum, gain, gt, eps) are those of StreamParams.
+struct alignas(16) ChainStep {
     GemvProblem prob[kGemvMaxProblems];
     int64_t gstart[kGemvMaxProblems + 1];   // prefix sums of the products' row groups
     int count;
@@ -90,17 +100,27 @@ struct ChainSmem {
     float wscale[kGemvMaxProblems];
     int go;          // the step's counter wait succeeded (written by thread 0)
     int step_fail;   // a consumer warp gave up during the step
+    ChainStep cur;   // the consumers' current step
     int sacc[kMaxGroupsPerCta][8];
 };
 
 constexpr size_t kChainHeader = (sizeof(ChainSmem) + 127) / 128 * 128;
 constexpr size_t kChainSmem = kChainHeader + size_t(kChainStages) * kChainStageBytes + size_t(kChainMaxK);
 
-__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned *p)
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const unsigned *p)
 {
     uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Arrival on a step counter: release (orders this CTA's earlier stores, made
+// visible to this thread by the block barrier before it) and add.
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ int locate_step(const ChainStep &p, int64_t G)
@@ -120,18 +140,23 @@ __device__ __forceinline__ void chain_abort(unsigned *g_abort, volatile int *abo
     atomicExch(g_abort, 1u);
 }
 
-// Wait until counter >= target, bounded; false on timeout or abort.
+// Wait until counter >= target, bounded; false on timeout or abort.  Relaxed
+// polling, one acquire fence once the count is reached.
 __device__ __noinline__ bool wait_counter(const unsigned *counter, unsigned target, unsigned *g_abort,
                                           volatile int *abort_flag, int *status, uint64_t limit_ns)
 {
-    if (ld_acquire_u32(counter) >= target)
+    if (ld_relaxed_u32(counter) >= target) {
+        fence_acq_rel_gpu();
         return true;
+    }
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (ld_acquire_u32(counter) >= target)
+        if (ld_relaxed_u32(counter) >= target) {
+            fence_acq_rel_gpu();
             return true;
+        }
         if ((it & 15) == 0) {
-            if (*abort_flag || ld_acquire_u32(g_abort)) {
+            if (*abort_flag || ld_relaxed_u32(g_abort)) {
                 *abort_flag = 1;
                 return false;
             }
@@ -279,20 +304,26 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemv_chain_kernel(const Chai
     int sb = 0;
     uint32_t ph = 0;
     bool ok = true;
+    const ChainStep &p = sm.cur;
     for (int s = 0; s < nsteps && ok; ++s) {
-        const ChainStep &p = steps[s];
+        const ChainStep &pg = steps[s];
         int64_t g_begin;
         int ng;
-        cta_groups(p, bx, G, g_begin, ng);
+        cta_groups(pg, bx, G, g_begin, ng);
         if (ng > 0) {
             // every CTA has finished the previous step: its outputs (this
             // step's x, or an earlier step's) are in memory.  One thread
             // waits and the decision is read by all consumer warps after a
-            // barrier, so that they all leave (or stay) together.
+            // barrier, so that they all leave (or stay) together; meanwhile
+            // warp 1 copies the step's descriptor into shared memory.
             if (tid == 0) {
                 sm.step_fail = 0;
                 const unsigned target = unsigned(G) + (s == test_step ? 1u : 0u);
                 sm.go = s == 0 ? 1 : int(wait_counter(&counters[s - 1], target, g_abort, abort_flag, status, limit_ns));
+            } else if (warp == 1) {
+                constexpr int kVecs = int(sizeof(ChainStep) / 16);
+                for (int i = lane; i < kVecs; i += 32)
+                    reinterpret_cast<uint4 *>(&sm.cur)[i] = reinterpret_cast<const uint4 *>(&pg)[i];
             }
             consumers_sync<KC>();
             if (!sm.go) {
@@ -383,11 +414,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemv_chain_kernel(const Chai
             }
             consumers_sync<KC>();
         }
-        // this CTA is done with step s (its outputs are stored and fenced)
-        if (tid == 0) {
-            __threadfence();
-            atomicAdd(&counters[s], 1u);
-        }
+        // this CTA is done with step s (its outputs are stored; the barrier
+        // above ordered them before this release)
+        if (tid == 0)
+            red_release_add(&counters[s], 1u);
     }
     if (!ok)
         chain_abort(g_abort, abort_flag);

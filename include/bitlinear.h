@@ -335,6 +335,10 @@ int bitlinear_chain_plan(int nsteps, const bitlinear_chain_step *steps,
  * reported by the next bitlinear_last_device_status() as BL_ERR_TIMEOUT and
  * leaves the outputs of the unfinished steps unspecified.  Runs of one plan
  * must be ordered (one stream); the buffers the plan names must stay alive.
+ * On B200 a step of the 2.4B decode stream takes 4-6.5 us this way, against
+ * ~3.1 us as separate bitlinear_gemv_fused_multi launches with BL_FLAG_PDL
+ * in a CUDA graph: use the chain where one launch per token matters more
+ * than per-step latency.
  *   plan, nsteps   as given to bitlinear_chain_plan
  */
 int bitlinear_chain_run(const void *plan, int nsteps, void *stream);

@@ -36,7 +36,7 @@ def _oracle_step(ws_o, x_bf16, gain=None, eps=1e-5):
     (y32, acc, bf16 bits)."""
     xf = x_bf16.float().numpy()
     if gain is not None:
-        xf = oracle.rmsnorm(xf, gain.float().numpy(), eps)
+        xf = oracle.rmsnorm(xf, gain.float().cpu().numpy(), eps)
     q, d, r = oracle.quantize_act(xf)
     out = []
     for g, codes in ws_o:
