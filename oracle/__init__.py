@@ -71,6 +71,10 @@ def _load():
             "oracle_binary_rescale": (None, [vp, f32, f32, i64, vp]),
             "oracle_bitplanes": (None, [vp, i64, i64, vp, vp]),
             "oracle_bitplane_acc": (None, [vp, vp, vp, i64, i64, vp]),
+            "oracle_rope": (None, [vp, i64, i64, i64, ctypes.c_double, vp]),
+            "oracle_attention_decode": (None, [vp, vp, vp, i64, i64, i64, i64, i64, vp]),
+            "oracle_relu2_gate": (None, [vp, vp, i64, vp]),
+            "oracle_residual_add": (None, [vp, vp, i64, vp]),
             "oracle_num_threads": (ctypes.c_int, []),
         }
         for name, (res, args) in sig.items():
@@ -304,3 +308,91 @@ def bitplane_gemv(codes: np.ndarray, gamma_eff, x: np.ndarray):
     acc = bitplane_acc(mag, sign, xb, K)
     return {"mag": mag, "sign": sign, "xb": xb, "s_x": s_x, "acc": acc,
             "y": binary_rescale(acc, gamma_eff, s_x)}
+
+
+# --------------------------------------------------------------------------
+# decoder layer pieces around the BitLinears (synthetic layer stack)
+# --------------------------------------------------------------------------
+
+ROPE_BASE = 10000.0
+
+
+def rope(x: np.ndarray, heads: int, D: int, pos: int, base: float = ROPE_BASE) -> np.ndarray:
+    """Rotate pairs (2i, 2i+1) of each head by pos * base^(-2i/D); fp32 [heads*D]."""
+    x = _c(x, np.float32).reshape(-1)
+    assert x.size == heads * D
+    out = np.empty(heads * D, np.float32)
+    _load().oracle_rope(_p(x), heads, D, pos, float(base), _p(out))
+    return out
+
+
+def attention_decode(q, K, V, H: int, Hkv: int, D: int, T: int) -> np.ndarray:
+    """Softmax attention of one query token over positions 0..T-1 of a
+    [Hkv, T_stride, D] cache (grouped heads); fp32 [H*D] before rounding."""
+    q = _c(q, np.float32).reshape(-1)
+    K = _c(K, np.float32)
+    V = _c(V, np.float32)
+    T_stride = K.shape[1]
+    out = np.empty(H * D, np.float32)
+    _load().oracle_attention_decode(_p(q), _p(K), _p(V), H, Hkv, D, T, T_stride, _p(out))
+    return out
+
+
+def relu2_gate(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    g = _c(g, np.float32).reshape(-1)
+    u = _c(u, np.float32).reshape(-1)
+    out = np.empty(g.size, np.float32)
+    _load().oracle_relu2_gate(_p(g), _p(u), g.size, _p(out))
+    return out
+
+
+def residual_add(h: np.ndarray, y: np.ndarray) -> np.ndarray:
+    h = _c(h, np.float32).reshape(-1)
+    y = _c(y, np.float32).reshape(-1)
+    out = np.empty(h.size, np.float32)
+    _load().oracle_residual_add(_p(h), _p(y), h.size, _p(out))
+    return out
+
+
+def bf16_round(v: np.ndarray) -> np.ndarray:
+    """fp32 values rounded to bf16 (nearest even), returned as fp32."""
+    bits = to_bf16_bits(np.asarray(v, np.float32))
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def _linear32(x32: np.ndarray, codes: np.ndarray, gamma, gain=None, eps: float = RMS_EPS):
+    """One token's BitLinear: optional RMSNorm, absmax int8, ternary product,
+    rescale; fp32 y (before any rounding)."""
+    x32 = np.asarray(x32, np.float32).reshape(1, -1)
+    if gain is not None:
+        x32 = rmsnorm(x32, gain, eps)
+    q, d, r = quantize_act(x32)
+    return rescale(ternary_acc(codes, q), d, gamma)[0]
+
+
+def decoder_layer(h: np.ndarray, layer: dict, cache_k: np.ndarray, cache_v: np.ndarray,
+                  pos: int, cfg: dict) -> np.ndarray:
+    """One decode step of one layer (readings as in the C functions above):
+    h (bf16 values as fp32 [hidden]) -> new h; writes position pos of the
+    layer's cache [Hkv, T, D] (bf16 values as fp32).  layer: dict of
+    (gamma, codes) for q, k, v, o, gate, up, down and the two RMSNorm gains
+    (fp32 arrays) g_attn, g_ffn."""
+    H, Hkv, D = cfg["heads"], cfg["kv_heads"], cfg["head_dim"]
+    eps = cfg.get("eps", RMS_EPS)
+    base = cfg.get("rope_base", ROPE_BASE)
+    h = np.asarray(h, np.float32).reshape(-1)
+    q = bf16_round(_linear32(h, layer["q"][1], layer["q"][0], layer["g_attn"], eps))
+    k = bf16_round(_linear32(h, layer["k"][1], layer["k"][0], layer["g_attn"], eps))
+    v = bf16_round(_linear32(h, layer["v"][1], layer["v"][0], layer["g_attn"], eps))
+    q_rot = bf16_round(rope(q, H, D, pos, base))
+    k_rot = bf16_round(rope(k, Hkv, D, pos, base))
+    cache_k[:, pos, :] = k_rot.reshape(Hkv, D)
+    cache_v[:, pos, :] = v.reshape(Hkv, D)
+    attn = bf16_round(attention_decode(q_rot, cache_k, cache_v, H, Hkv, D, pos + 1))
+    y_o = _linear32(attn, layer["o"][1], layer["o"][0])
+    h1 = bf16_round(residual_add(h, y_o))
+    gate = bf16_round(_linear32(h1, layer["gate"][1], layer["gate"][0], layer["g_ffn"], eps))
+    up = bf16_round(_linear32(h1, layer["up"][1], layer["up"][0], layer["g_ffn"], eps))
+    m = relu2_gate(gate, up)
+    y_d = _linear32(m, layer["down"][1], layer["down"][0])
+    return bf16_round(residual_add(h1, y_d))

@@ -48,6 +48,7 @@
  * order of additions is part of the definition above.
  */
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 #include <math.h>
 
@@ -378,6 +379,95 @@ void oracle_bitplane_acc(const uint64_t *mag, const uint64_t *sign,
         }
         acc[n] = (int32_t)dot;
     }
+}
+
+/* ---------------------------------------------------------------------------
+ * The rest of a decoder layer around the BitLinears, for the synthetic layer
+ * stack.  [GUIDE] "Understanding the Two-Phase Architecture" (Attention and
+ * FeedForward call BitLinear; a KV cache of shape (1, seq_len, kv_heads, 1,
+ * head_dim)); [FLOOR] "What's inside" (rope.rs: RoPE applied to queries and
+ * keys before attention; attention.cu: attention with a softmax over the
+ * cached positions).  The pages fix no formula; the readings:
+ *   RoPE       pairs (2i, 2i + 1) of each head rotated by the angle
+ *              pos * base^(-2i / D) (fp64, then cos and sin rounded to fp32);
+ *              out = (a c - b s, a s + b c), each product and the sum or
+ *              difference an fp32 operation in that order.
+ *   attention  per query head h (kv head h / (H / Hkv)) over positions
+ *              j = 0 .. T - 1: s_j = (float)(sum_d q[d] K[j][d]) * scale with
+ *              the dot product in fp64; m = max s_j; e_j = (float)exp((double)
+ *              (s_j - m)) with s_j - m in fp32; S = (float)(sum_j e_j) in fp64;
+ *              out[d] = (float)(sum_j e_j V[j][d]) / S, the sum in fp64, the
+ *              division in fp32.  scale = (float)(1 / sqrt(D)).
+ *   FFN gate   m = (r * r) * u with r = max(g, 0) (squared ReLU gating), fp32.
+ * ------------------------------------------------------------------------- */
+void oracle_rope(const float *x, int64_t heads, int64_t D, int64_t pos, double base,
+                 float *out)
+{
+    for (int64_t h = 0; h < heads; ++h)
+        for (int64_t i = 0; i < D / 2; ++i) {
+            double ang = (double)pos * pow(base, -(double)(2 * i) / (double)D);
+            float c = (float)cos(ang), s = (float)sin(ang);
+            float a = x[h * D + 2 * i], b = x[h * D + 2 * i + 1];
+            float ac = a * c, bs = b * s, as = a * s, bc = b * c;
+            out[h * D + 2 * i] = ac - bs;
+            out[h * D + 2 * i + 1] = as + bc;
+        }
+}
+
+/* K, V: [Hkv][T_stride][D]; positions 0 .. T - 1 are used. */
+void oracle_attention_decode(const float *q, const float *K, const float *V, int64_t H,
+                             int64_t Hkv, int64_t D, int64_t T, int64_t T_stride,
+                             float *out)
+{
+    float scale = (float)(1.0 / sqrt((double)D));
+    float *sc = (float *)malloc((size_t)T * sizeof(float));
+    float *e = (float *)malloc((size_t)T * sizeof(float));
+    for (int64_t h = 0; h < H; ++h) {
+        int64_t kv = h / (H / Hkv);
+        const float *qh = q + h * D;
+        const float *Kh = K + kv * T_stride * D;
+        const float *Vh = V + kv * T_stride * D;
+        float m = -INFINITY;
+        for (int64_t j = 0; j < T; ++j) {
+            double dot = 0.0;
+            for (int64_t d = 0; d < D; ++d)
+                dot += (double)qh[d] * (double)Kh[j * D + d];
+            sc[j] = (float)dot * scale;
+            if (sc[j] > m)
+                m = sc[j];
+        }
+        double S = 0.0;
+        for (int64_t j = 0; j < T; ++j) {
+            float t = sc[j] - m;
+            e[j] = (float)exp((double)t);
+            S += (double)e[j];
+        }
+        float Sf = (float)S;
+        for (int64_t d = 0; d < D; ++d) {
+            double num = 0.0;
+            for (int64_t j = 0; j < T; ++j)
+                num += (double)e[j] * (double)Vh[j * D + d];
+            out[h * D + d] = (float)num / Sf;
+        }
+    }
+    free(sc);
+    free(e);
+}
+
+void oracle_relu2_gate(const float *g, const float *u, int64_t n, float *out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        float r = g[i] > 0.0f ? g[i] : 0.0f;
+        float rr = r * r;
+        out[i] = rr * u[i];
+    }
+}
+
+/* Residual add: out = h + y, one fp32 addition (h a bf16 value as fp32). */
+void oracle_residual_add(const float *h, const float *y, int64_t n, float *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = h[i] + y[i];
 }
 
 /* Threads the OpenMP loops above use (1 when built without OpenMP). */

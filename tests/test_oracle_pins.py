@@ -403,3 +403,94 @@ def test_bitplane_invariants():
     # flipping every activation's sign negates every dot product (no x is 0)
     assert np.all(x != 0)
     np.testing.assert_array_equal(oracle.bitplane_gemv(codes, g, -x)["acc"], -acc)
+
+
+# ---------------------------------------------------------------- decoder layer pieces
+
+def test_rope_hand_and_closed_forms():
+    # D = 4: pair 0 turns by pos, pair 1 by pos * 10000^(-1/2) = pos / 100
+    out = oracle.rope(_f32([1.0, 0.0, 0.0, 1.0]), 1, 4, 1)
+    np.testing.assert_allclose(out, [math.cos(1.0), math.sin(1.0), -math.sin(0.01), math.cos(0.01)],
+                               rtol=1e-6, atol=1e-7)
+    x = si.activations(1, 8 * 128, seed=2, dtype=torch.float32).numpy()[0]
+    np.testing.assert_array_equal(oracle.rope(x, 8, 128, 0), x)       # position 0: identity
+    for pos in (1, 17, 1000):
+        y = oracle.rope(x, 8, 128, pos).astype(np.float64)
+        n_in = x.astype(np.float64).reshape(-1, 2)
+        n_out = y.reshape(-1, 2)
+        np.testing.assert_allclose(np.hypot(n_out[:, 0], n_out[:, 1]),
+                                   np.hypot(n_in[:, 0], n_in[:, 1]), rtol=2e-6, atol=1e-6)
+        # against the rotation written in fp64
+        i = np.arange(64)
+        ang = pos * 10000.0 ** (-(2.0 * i) / 128)
+        a, b = n_in[:, 0].reshape(8, 64), n_in[:, 1].reshape(8, 64)
+        want = np.stack([a * np.cos(ang) - b * np.sin(ang), a * np.sin(ang) + b * np.cos(ang)], -1)
+        np.testing.assert_allclose(y.reshape(8, 64, 2), want, rtol=1e-5, atol=2e-6)
+
+
+def test_rope_composes():
+    x = si.activations(1, 4 * 128, seed=3, dtype=torch.float32).numpy()[0]
+    two = oracle.rope(oracle.rope(x, 4, 128, 5), 4, 128, 7)
+    np.testing.assert_allclose(two, oracle.rope(x, 4, 128, 12), rtol=1e-5, atol=2e-6)
+
+
+def test_attention_closed_forms_and_textbook():
+    H, Hkv, D, T = 8, 2, 128, 37
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal(H * D).astype(np.float32)
+    K = rng.standard_normal((Hkv, 64, D)).astype(np.float32)
+    V = rng.standard_normal((Hkv, 64, D)).astype(np.float32)
+    # one position: the softmax is 1, the output is that value row exactly
+    out1 = oracle.attention_decode(q, K, V, H, Hkv, D, 1).reshape(H, D)
+    for h in range(H):
+        np.testing.assert_array_equal(out1[h], V[h // (H // Hkv), 0])
+    # textbook softmax attention in fp64 with grouped heads and 1/sqrt(D)
+    out = oracle.attention_decode(q, K, V, H, Hkv, D, T).reshape(H, D).astype(np.float64)
+    for h in range(H):
+        kv = h // (H // Hkv)
+        s = (K[kv, :T].astype(np.float64) @ q[h * D:(h + 1) * D]) / math.sqrt(D)
+        p = np.exp(s - s.max())
+        p /= p.sum()
+        np.testing.assert_allclose(out[h], p @ V[kv, :T], rtol=1e-5, atol=1e-6)
+    # equal scores (zero query): the mean of the cached values
+    out0 = oracle.attention_decode(np.zeros(H * D, np.float32), K, V, H, Hkv, D, T).reshape(H, D)
+    np.testing.assert_allclose(out0[0], V[0, :T].mean(axis=0), rtol=1e-5, atol=1e-6)
+
+
+def test_relu2_gate_and_residual():
+    np.testing.assert_array_equal(oracle.relu2_gate(_f32([-1.0, 0.0, 2.0, 0.5]), _f32([3.0, 3.0, 3.0, -4.0])),
+                                  _f32([0.0, 0.0, 12.0, -1.0]))
+    np.testing.assert_array_equal(oracle.residual_add(_f32([1.0, -2.0]), _f32([0.5, 2.0])), _f32([1.5, 0.0]))
+
+
+def _layer(seed, zero=(), K=256, H=2, Hkv=1, D=128, F=384):
+    hidden = H * D
+    shapes = {"q": (hidden, hidden), "k": (Hkv * D, hidden), "v": (Hkv * D, hidden),
+              "o": (hidden, hidden), "gate": (F, hidden), "up": (F, hidden), "down": (hidden, F)}
+    layer = {}
+    for i, (name, (N, Kk)) in enumerate(shapes.items()):
+        W = si.weight(N, Kk, seed=seed * 10 + i).numpy()
+        if name in zero:
+            W = np.zeros_like(W)
+        g = oracle.weight_scale(W)
+        layer[name] = (g, oracle.ternary_codes(W, g))
+    layer["g_attn"] = np.ones(hidden, np.float32)
+    layer["g_ffn"] = np.ones(hidden, np.float32)
+    return layer, dict(heads=H, kv_heads=Hkv, head_dim=D)
+
+
+def test_decoder_layer_closed_forms():
+    layer, cfg = _layer(1, zero=("q", "k", "v", "o", "gate", "up", "down"))
+    h = oracle.bf16_round(si.activations(1, 256, seed=4, dtype=torch.float32).numpy()[0])
+    ck = np.zeros((1, 8, 128), np.float32)
+    cv = np.zeros((1, 8, 128), np.float32)
+    # all weights zero: every BitLinear gives 0, the residual stream is unchanged
+    np.testing.assert_array_equal(oracle.decoder_layer(h, layer, ck, cv, 3, cfg), h)
+    assert not ck.any() and not cv.any()
+    # only the attention output projection and the FFN zero: h is unchanged,
+    # and position 3 (only) of the cache is written
+    layer, cfg = _layer(2, zero=("o", "gate", "up", "down"))
+    ck[:] = 7.0
+    out = oracle.decoder_layer(h, layer, ck, cv, 3, cfg)
+    np.testing.assert_array_equal(out, h)
+    assert (ck[:, [0, 1, 2, 4, 5, 6, 7]] == 7.0).all() and not (ck[:, 3] == 7.0).all()
