@@ -500,6 +500,43 @@ def rmsnorm_gemv_cost(bl, K, Ns, iters=200, device="cuda"):
             "rmsnorm_GBps": per / t_norm / 1e9, "plain_GBps": per / t_plain / 1e9}
 
 
+def decoder_tokens(bl, contexts=(512, 2048), tokens=64, device="cuda"):
+    """The synthetic 2.4B decoder stack (30 layers: RMSNorm, q/k/v, RoPE +
+    attention over a bf16 KV cache, o + residual, RMSNorm, gate/up, squared
+    ReLU gate, down + residual; 151 launches per token with PDL) replayed
+    from a CUDA graph, one token per replay, at a given number of cached
+    positions."""
+    from bit_ternary_weight_b200.decoder import Decoder, DecoderConfig
+    cfg = DecoderConfig(max_seq=max(contexts) + tokens + 8)
+    dec = Decoder.random(cfg, seed=1, device=device)
+    dec.h.copy_(si.activations(1, cfg.hidden, seed=5)[0])
+    out = []
+    dec.set_position(0)
+    dec.step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        dec.step()
+    for ctx in contexts:
+        dec.set_position(ctx)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(tokens):
+            g.replay()
+        e.record()
+        torch.cuda.synchronize()
+        t = s.elapsed_time(e) / 1000.0 / tokens
+        out.append({"context": ctx, "tokens": tokens, "us_per_token": t * 1e6,
+                    "tokens_per_s": 1.0 / t, "weight_GBps": dec.weight_bytes() / t / 1e9,
+                    "launches_per_token": 5 * cfg.layers + 1})
+    assert bl.last_device_status() == 0
+    del g, dec
+    return out
+
+
 def prefill_gemm(bl, K, N, M, iters=20, device="cuda"):
     gen = torch.Generator(device=device)
     gen.manual_seed(3)
@@ -736,6 +773,7 @@ def run_ours(args, world, rank, local):
                                           for (K, N) in si.DECODE_SHAPES_100B])
         measure("lut_vs_dp4a", lambda: [lut_vs_dp4a(bl, K, N, device=device)
                                         for (K, N) in si.DECODE_SHAPES_2B + [(8192, 28672)]])
+        measure("decoder_2b", lambda: decoder_tokens(bl, device=device))
         measure("rmsnorm_gemv", lambda: [rmsnorm_gemv_cost(bl, 2560, [6912, 6912], device=device),
                                          rmsnorm_gemv_cost(bl, 2560, [2560, 640, 640], device=device),
                                          rmsnorm_gemv_cost(bl, 8192, [28672], device=device)])

@@ -116,6 +116,12 @@ class ChainStepC(ctypes.Structure):
 
 
 _SIGNATURES.update({
+    "bitlinear_decode_linear": (_int, [_int, _vp, _vp, _vp, _i64, _int, _vp, _int, _vp, _vp, _int,
+                                       ctypes.c_float, _vp, _int, _vp, _vp, _vp, ctypes.c_uint,
+                                       _vp]),
+    "bitlinear_attention_decode": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
+                                          ctypes.c_double, _vp, ctypes.c_uint, _vp]),
+    "bitlinear_position_advance": (_int, [_vp, _vp]),
     "bitlinear_chain_plan_bytes": (_sz, [_int]),
     "bitlinear_chain_plan": (_int, [_int, ctypes.POINTER(ChainStepC), _vp, _sz, _vp]),
     "bitlinear_chain_run": (_int, [_vp, _int, _vp]),
@@ -348,6 +354,63 @@ def rmsnorm_gemv_fused_multi(weights, x: torch.Tensor, gain=None, eps: float = R
             float(eps), ys, _dt(outs[0].dtype), ldys, accs, BL_FLAG_PDL if pdl else 0,
             _stream(x.device)), "bitlinear_rmsnorm_gemv_fused_multi")
     return outs
+
+
+BL_ACT_PLAIN = 0
+BL_ACT_RMSNORM = 1
+BL_ACT_RELU2_GATE = 2
+
+
+def decode_linear(weights, x: torch.Tensor, act: int = BL_ACT_PLAIN, x2=None, gain=None,
+                  eps: float = RMS_EPS, outs=None, resid=None, out_dtype=torch.bfloat16,
+                  acc_dbgs=None, pdl: bool = False):
+    """One token through a decoder layer's BitLinears sharing an input, in one
+    launch: act (plain / RMSNorm with gain / squared-ReLU gate of x and x2),
+    the products, the rescale and, per product, an optional residual
+    (resid[i]: bf16 [N] added before the rounding; may be outs[i] itself)."""
+    x = x.reshape(-1)
+    n = len(weights)
+    if outs is None:
+        outs = [torch.empty(w.N, dtype=out_dtype, device=x.device) for w in weights]
+    P = ctypes.c_void_p * n
+    I64 = ctypes.c_int64 * n
+    packed = P(*[w.packed.data_ptr() for w in weights])
+    scales = P(*[w.w_scale.data_ptr() for w in weights])
+    Ns = I64(*[w.N for w in weights])
+    ys = P(*[o.data_ptr() for o in outs])
+    ldys = I64(*[w.N for w in weights])
+    res = None if resid is None else P(*[0 if r is None else r.data_ptr() for r in resid])
+    accs = None if acc_dbgs is None else P(*[0 if a is None else a.data_ptr() for a in acc_dbgs])
+    gt = BL_F32 if gain is None else _dt(gain.dtype)
+    with _on(x.device):
+        _check(_lib.bitlinear_decode_linear(
+            n, packed, scales, Ns, weights[0].K, act, _ptr(x), _dt(x.dtype), _ptr(x2), _ptr(gain),
+            gt, float(eps), ys, _dt(outs[0].dtype), ldys, res, accs, BL_FLAG_PDL if pdl else 0,
+            _stream(x.device)), "bitlinear_decode_linear")
+    return outs
+
+
+def attention_decode(q, k, v, cache_k, cache_v, pos, H: int, Hkv: int, out=None,
+                     rope_base: float = 10000.0, pdl: bool = False):
+    """One token's attention with RoPE over a bf16 cache [Hkv, T_max, 128];
+    pos: int32 device scalar (this token's position; the cache row written)."""
+    D = 128
+    T_max = cache_k.shape[-2]
+    if out is None:
+        out = torch.empty(H * D, dtype=torch.bfloat16, device=q.device)
+    with _on(q.device):
+        _check(_lib.bitlinear_attention_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(cache_k),
+                                               _ptr(cache_v), _ptr(pos), H, Hkv, D, T_max,
+                                               float(rope_base), _ptr(out),
+                                               BL_FLAG_PDL if pdl else 0, _stream(q.device)),
+               "bitlinear_attention_decode")
+    return out
+
+
+def position_advance(pos: torch.Tensor):
+    with _on(pos.device):
+        _check(_lib.bitlinear_position_advance(_ptr(pos), _stream(pos.device)),
+               "bitlinear_position_advance")
 
 
 @dataclass

@@ -450,6 +450,109 @@ int bitlinear_rmsnorm_gemv_fused_multi(int count, const uint8_t *const *packed,
     return launch_gemv_stream(b, true, static_cast<cudaStream_t>(stream), gain, gt, eps, true);
 }
 
+int bitlinear_decode_linear(int count, const uint8_t *const *packed, const float *const *w_scale,
+                            const int64_t *N, int64_t K, int act, const void *x, int xt,
+                            const void *x2, const void *gain, int gt, float eps, void *const *y,
+                            int yt, const int64_t *ldy, const void *const *resid,
+                            int32_t *const *acc_dbg, unsigned flags, void *stream)
+{
+    if (!packed || !w_scale || !N || !y || !ldy || !x)
+        return BL_ERR_NULL;
+    if (act == BL_ACT_RELU2_GATE && !x2)
+        return BL_ERR_NULL;
+    if (count < 1 || count > kGemvMaxProblems || (flags & ~BL_FLAG_PDL) ||
+        (act != BL_ACT_PLAIN && act != BL_ACT_RMSNORM && act != BL_ACT_RELU2_GATE))
+        return BL_ERR_SHAPE;
+    if (!valid_dtype(xt) || !valid_dtype(yt) || (gain && !valid_dtype(gt)) ||
+        (act == BL_ACT_RELU2_GATE && xt != BL_BF16))
+        return BL_ERR_DTYPE;
+    bool any_resid = false;
+    if (resid)
+        for (int i = 0; i < count; ++i)
+            any_resid = any_resid || resid[i] != nullptr;
+    if (any_resid && yt != BL_BF16)
+        return BL_ERR_DTYPE;
+    if (act == BL_ACT_RMSNORM && (!(eps >= 0.0f) || !(eps <= 3.0e38f)))
+        return BL_ERR_SHAPE;
+    int st;
+    for (int i = 0; i < count; ++i) {
+        if ((st = check_gemv_common(packed[i], w_scale[i], N[i], K, 1, y[i], yt, ldy[i], 1)))
+            return st;
+        if ((acc_dbg && (reinterpret_cast<uintptr_t>(acc_dbg[i]) & 3u)) ||
+            (resid && (reinterpret_cast<uintptr_t>(resid[i]) & 1u)))
+            return BL_ERR_ALIGN;
+    }
+    if (!aligned16(x) || !aligned16(x2) || !aligned16(gain))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    if ((st = need_device(&di)))
+        return st;
+    GemvBatch b{};
+    b.count = count;
+    for (int i = 0; i < count; ++i) {
+        b.prob[i] = GemvProblem{packed[i], w_scale[i], N[i], y[i], ldy[i], acc_dbg ? acc_dbg[i] : nullptr,
+                                resid ? resid[i] : nullptr};
+    }
+    b.K = K;
+    b.M = 1;
+    b.x = x;
+    b.xt = xt;
+    b.ldx = K;
+    b.yt = yt;
+    b.flags = flags;
+    if (!gemv_stream_applies(b, di->sm_count))
+        return BL_ERR_SHAPE;
+    if ((st = check_dev_ptrs({x, x2, gain})))
+        return st;
+    for (int i = 0; i < count; ++i)
+        if ((st = check_dev_ptrs({packed[i], w_scale[i], y[i], acc_dbg ? acc_dbg[i] : nullptr,
+                                  resid ? resid[i] : nullptr})))
+            return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (act == BL_ACT_RELU2_GATE)
+        return launch_gemv_stream_relu2(b, x2, s);
+    return launch_gemv_stream(b, true, s, gain, gt, eps, act == BL_ACT_RMSNORM);
+}
+
+int bitlinear_attention_decode(const void *q, const void *k, const void *v, void *cache_k,
+                               void *cache_v, const int32_t *pos, int H, int Hkv, int D,
+                               int T_max, double rope_base, void *out, unsigned flags,
+                               void *stream)
+{
+    if (!q || !k || !v || !cache_k || !cache_v || !pos || !out)
+        return BL_ERR_NULL;
+    if (H < 1 || Hkv < 1 || H % Hkv || D != 128 || T_max < 1 || T_max > 32768 ||
+        !(rope_base > 1.0) || !(rope_base < 1e30) || (flags & ~BL_FLAG_PDL) || H > 65535)
+        return BL_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
+         reinterpret_cast<uintptr_t>(cache_k) | reinterpret_cast<uintptr_t>(cache_v) |
+         reinterpret_cast<uintptr_t>(out)) & 7u || (reinterpret_cast<uintptr_t>(pos) & 3u))
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({q, k, v, cache_k, cache_v, pos, out})))
+        return st;
+    return launch_attention_decode(q, k, v, cache_k, cache_v, pos, H, Hkv, D, T_max, rope_base, out,
+                                   flags, static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_position_advance(int32_t *pos, void *stream)
+{
+    if (!pos)
+        return BL_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(pos) & 3u)
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({pos})))
+        return st;
+    return launch_position_advance(pos, static_cast<cudaStream_t>(stream));
+}
+
 size_t bitlinear_chain_plan_bytes(int nsteps) { return chain_plan_bytes(nsteps); }
 
 int bitlinear_chain_plan(int nsteps, const bitlinear_chain_step *steps, void *plan,

@@ -65,6 +65,13 @@ __device__ __forceinline__ uint32_t ld_dep_u32(const void *p)
     return v;
 }
 
+__device__ __forceinline__ uint32_t ld_dep_u16(const void *p)
+{
+    unsigned short v;
+    asm volatile("ld.global.cg.u16 %0, [%1];" : "=h"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // 4-way byte dot product, unsigned bytes of a times signed bytes of b.
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
 {

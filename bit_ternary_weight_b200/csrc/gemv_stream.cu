@@ -155,6 +155,8 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
         stream_rmsnorm_quantize<KC, BL_BF16, CH>(p, sm, qs);
     else if constexpr (MODE == SMODE_NORM_F32)
         stream_rmsnorm_quantize<KC, BL_F32, 0>(p, sm, qs);
+    else if constexpr (MODE == SMODE_RELU2)
+        stream_relu2_quantize<KC>(p, sm, qs);
     else if constexpr (MODE == SMODE_X_BF16 && CH > 0)
         stream_quantize_bf16<KC, CH>(p, sm, qs);
     else
@@ -230,7 +232,14 @@ __global__ void __launch_bounds__(Geo<KC>::kThreads, Geo<KC>::kCtasPerSm)
             const int a = (&sm.sacc[0][0])[idx] - rs;
             if (pr.acc_dbg)
                 pr.acc_dbg[row] = a;
-            store_y(pr.y, p.yt, row, rescale1(a, dd, sm.wscale[pi]));
+            float v = rescale1(a, dd, sm.wscale[pi]);
+            if (pr.resid) {
+                // residual stream: one fp32 addition before the bf16 rounding
+                // (read coherently: the preceding launch may have written it)
+                const uint32_t hb = ld_dep_u16(static_cast<const uint16_t *>(pr.resid) + row);
+                v = __fadd_rn(__uint_as_float(hb << 16), v);
+            }
+            store_y(pr.y, p.yt, row, v);
         }
     }
 }
@@ -365,6 +374,26 @@ int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s, const voi
 int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s)
 {
     return launch_gemv_stream(b, fused, s, nullptr, BL_F32, 0.0f, false);
+}
+
+int launch_gemv_stream_relu2(const GemvBatch &b, const void *x2, cudaStream_t s)
+{
+    StreamParams p{};
+    p.count = b.count;
+    p.gstart[0] = 0;
+    for (int i = 0; i < b.count; ++i) {
+        p.prob[i] = b.prob[i];
+        p.gstart[i + 1] = p.gstart[i] + (b.prob[i].N + 7) / 8;
+    }
+    for (int i = b.count; i < kGemvMaxProblems; ++i)
+        p.gstart[i + 1] = p.gstart[b.count];
+    p.K = b.K;
+    p.x = b.x;
+    p.x2 = x2;
+    p.yt = b.yt;
+    if (b.K <= kSmallK)
+        return launch_mode<8, SMODE_RELU2, 0>(p, s, b.flags);
+    return launch_mode<16, SMODE_RELU2, 0>(p, s, b.flags);
 }
 
 }  // namespace bl

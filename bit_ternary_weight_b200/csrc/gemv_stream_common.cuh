@@ -29,7 +29,8 @@ struct Geo {
 
 // Activations: pre-quantised q; raw bf16 / fp32 x quantised in the prologue;
 // or x normalised (RMSNorm) and then quantised in the prologue.
-enum { SMODE_Q = 0, SMODE_X_BF16 = 1, SMODE_X_F32 = 2, SMODE_NORM_BF16 = 3, SMODE_NORM_F32 = 4 };
+enum { SMODE_Q = 0, SMODE_X_BF16 = 1, SMODE_X_F32 = 2, SMODE_NORM_BF16 = 3, SMODE_NORM_F32 = 4,
+       SMODE_RELU2 = 5 };
 
 // 512-byte pieces (256 k) of one group per stage: the whole k range when it
 // is at most two pieces per consumer warp (one stage per set), else one per
@@ -45,6 +46,7 @@ struct StreamParams {
     const float *d;
     const int32_t *rowsum;
     const void *x;
+    const void *x2;      // SMODE_RELU2: the up projection [K] (x is the gate), bf16
     const void *gain;    // RMSNorm gain [K] (SMODE_NORM_*), NULL for none
     int gt;              // its dtype
     float eps;           // RMSNorm epsilon
@@ -373,6 +375,47 @@ __device__ __forceinline__ void stream_rmsnorm_quantize(const Prm &p, Smem &sm, 
             h8(i, j, h);
             *reinterpret_cast<uint2 *>(qs + (j * 32 + lane) * 8) = quant8(h, s, sum);
         }
+    }
+    sum = __reduce_add_sync(0xffffffffu, sum);
+    if (lane == 0)
+        sm.bsum[warp] = sum;
+    __syncwarp();
+}
+
+// Squared-ReLU gate, then quantisation: h = (r * r) * u with r = max(g, 0),
+// g = x and u = x2 (bf16), two fp32 products; read twice from L2 (absmax
+// pass, quantise pass), each warp for the activations of its own pieces.
+template <int KC, class Prm, class Smem>
+__device__ __forceinline__ void stream_relu2_quantize(const Prm &p, Smem &sm, int8_t *qs)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int P = int(p.K / 256);
+    auto h8 = [&](int j, float (&h)[8]) {
+        float u[8];
+        load8<BL_BF16, true>(p.x, (int64_t(j) * 32 + lane) * 8, h);
+        load8<BL_BF16, true>(p.x2, (int64_t(j) * 32 + lane) * 8, u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float r = fmaxf(h[e], 0.0f);
+            h[e] = __fmul_rn(__fmul_rn(r, r), u[e]);
+        }
+    };
+    float amax = 0.0f;
+#pragma unroll 4
+    for (int j = warp; j < P; j += KC) {
+        float h[8];
+        h8(j, h);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            amax = fmaxf(amax, fabsf(h[e]));
+    }
+    const float s = stream_scale<KC>(sm, amax);
+    int sum = 0;
+#pragma unroll 4
+    for (int j = warp; j < P; j += KC) {
+        float h[8];
+        h8(j, h);
+        *reinterpret_cast<uint2 *>(qs + (j * 32 + lane) * 8) = quant8(h, s, sum);
     }
     sum = __reduce_add_sync(0xffffffffu, sum);
     if (lane == 0)

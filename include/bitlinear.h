@@ -277,6 +277,78 @@ int bitlinear_rmsnorm_gemv_fused_multi(int count, const uint8_t *const *packed,
                                        int32_t *const *acc_dbg, unsigned flags,
                                        void *stream);
 
+/* Activation modes of bitlinear_decode_linear. */
+#define BL_ACT_PLAIN 0       /* quantise x */
+#define BL_ACT_RMSNORM 1     /* RMSNorm x (gain, eps), then quantise */
+#define BL_ACT_RELU2_GATE 2  /* quantise relu(x)^2 * x2 (x: gate, x2: up, bf16) */
+
+/*
+ * One token through the decode BitLinears of a decoder layer, in one launch:
+ * the activation step in front (act), `count` products sharing it, the
+ * rescale, and optionally the residual add.  Sources: "How to Run BitNet
+ * Inference on GPU Using CUDA Kernels", section "Understanding the Two-Phase
+ * Architecture" (Attention and FeedForward call BitLinear); "bit-floor"
+ * README, section "What's inside" (rmsnorm.cu).  The gate's activation is a
+ * reading of this library (the pages name none): squared ReLU,
+ *   h[k] = (r * r) * x2[k],  r = max(x[k], 0),   two fp32 products,
+ * quantised like any activation (the fp32 h, not rounded to bf16 first).
+ *   act            BL_ACT_PLAIN, BL_ACT_RMSNORM or BL_ACT_RELU2_GATE
+ *   x, xt          device [K] (one token); bf16 for BL_ACT_RELU2_GATE
+ *   x2             BL_ACT_RELU2_GATE: device bf16 [K] (the up projection)
+ *   gain, gt, eps  BL_ACT_RMSNORM: as for bitlinear_rmsnorm_quantize_act
+ *   resid          NULL, or a host array of `count` pointers, each NULL or a
+ *                  device bf16 [N[i]]: y[i] = bf16(resid[i] + y32) with one
+ *                  fp32 addition (yt must be BL_BF16).  resid[i] may be y[i]
+ *                  itself (an in-place residual stream); it must not overlap
+ *                  x or x2.
+ *   other arguments as for bitlinear_gemv_fused_multi (M = 1)
+ * Runs the streaming one-token kernel only (K a multiple of 256 up to
+ * 32768, at most 64 row groups per SM), else BL_ERR_SHAPE.  Under
+ * BL_FLAG_PDL, x, x2 and resid may come from the kernel just before; the
+ * weights, scales and gain may not.
+ */
+int bitlinear_decode_linear(int count, const uint8_t *const *packed,
+                            const float *const *w_scale, const int64_t *N,
+                            int64_t K, int act, const void *x, int xt,
+                            const void *x2, const void *gain, int gt, float eps,
+                            void *const *y, int yt, const int64_t *ldy,
+                            const void *const *resid, int32_t *const *acc_dbg,
+                            unsigned flags, void *stream);
+
+/*
+ * Decode attention of one token over a bf16 KV cache, with RoPE and the
+ * append of this token's key and value.  Sources: "How to Run BitNet
+ * Inference on GPU Using CUDA Kernels", section "Understanding the Two-Phase
+ * Architecture" (Attention with a KV cache of shape (1, seq_len, kv_heads,
+ * 1, head_dim)); "bit-floor" README, section "What's inside" (rope.rs,
+ * attention.cu).  Readings (identical on the CPU oracle): interleaved RoPE
+ * pairs (2i, 2i + 1) turned by pos * rope_base^(-2i / D) (angle, cos, sin in
+ * fp64, rounded to fp32; rotation in fp32; rotated q and k rounded to bf16);
+ * s_j = (float)(q . K[j]) * (float)(1 / sqrt(D)) with the dot product in
+ * fp64; softmax weights e_j = (float)exp(s_j - max s); out = bf16((float)(sum_j
+ * e_j V[j]) / (float)(sum_j e_j)), sums in fp64.  Query head h reads kv head
+ * h / (H / Hkv).
+ *   q, k, v          device bf16 [H*D], [Hkv*D], [Hkv*D] (this token)
+ *   cache_k, cache_v device bf16 [Hkv][T_max][D]; position *pos of every kv
+ *                    head is written, positions 0 .. *pos read
+ *   pos              device int32 scalar: this token's position, read by
+ *                    the kernel (a CUDA graph can replay the call for the
+ *                    next token after bitlinear_position_advance)
+ *   out              device bf16 [H*D]
+ *   flags            0 or BL_FLAG_PDL (q, k, v may come from the kernel just
+ *                    before; the cache and pos from earlier work)
+ * D must be 128; H a multiple of Hkv; T_max <= 32768.  A position outside
+ * [0, T_max) writes nothing and makes the next bitlinear_last_device_status()
+ * return BL_ERR_SHAPE.
+ */
+int bitlinear_attention_decode(const void *q, const void *k, const void *v,
+                               void *cache_k, void *cache_v, const int32_t *pos,
+                               int H, int Hkv, int D, int T_max, double rope_base,
+                               void *out, unsigned flags, void *stream);
+
+/* *pos += 1 on the device (after a token's last attention call). */
+int bitlinear_position_advance(int32_t *pos, void *stream);
+
 /*
  * One step of a decode chain: `count` BitLinears sharing the token x (as in
  * bitlinear_gemv_fused_multi with M = 1), RMSNorm first when `norm` is set or
@@ -469,8 +541,10 @@ int bitlinear_bitplane_gemv(const uint64_t *planes, const float *w_scale,
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the
- * current device: BL_OK, or BL_ERR_TIMEOUT if a kernel's bounded wait ran
- * out since the last call.  BL_ERR_CUDA if the synchronisation failed.
+ * current device: BL_OK, BL_ERR_TIMEOUT if a kernel's bounded wait ran out,
+ * or BL_ERR_SHAPE if a kernel found a device-side argument out of range (a
+ * position outside the KV cache), since the last call.  BL_ERR_CUDA if the
+ * synchronisation failed.
  */
 int bitlinear_last_device_status(void *stream);
 

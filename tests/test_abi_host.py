@@ -233,3 +233,25 @@ def test_chain_argument_errors(bl):
     assert L.bitlinear_chain_run(A, 0, None) == bl.BL_ERR_SHAPE
     assert L.bitlinear_chain_run_timeout_test(A, 1, 1000000, None) == bl.BL_ERR_SHAPE
     assert L.bitlinear_chain_run_timeout_test(A, 2, 10, None) == bl.BL_ERR_SHAPE
+
+
+def test_decoder_entry_argument_errors(bl):
+    A = 0x7f0000000000
+    L = bl.lib
+    P = ctypes.c_void_p * 1
+    I = ctypes.c_int64 * 1
+    pk, sc, ys = P(A), P(A), P(A)
+    f = L.bitlinear_decode_linear
+    assert f(1, pk, sc, I(64), 256, 2, A, 1, None, None, 0, 1e-5, ys, 1, I(64), None, None, 0, None) == bl.BL_ERR_NULL
+    assert f(1, pk, sc, I(64), 256, 7, A, 1, None, None, 0, 1e-5, ys, 1, I(64), None, None, 0, None) == bl.BL_ERR_SHAPE
+    assert f(1, pk, sc, I(64), 256, 2, A, 0, A, None, 0, 1e-5, ys, 1, I(64), None, None, 0, None) == bl.BL_ERR_DTYPE
+    assert f(1, pk, sc, I(64), 256, 0, A, 1, None, None, 0, 1e-5, ys, 0, I(64), P(A), None, 0, None) == bl.BL_ERR_DTYPE
+    assert f(1, pk, sc, I(64), 256, 1, A, 1, None, None, 0, -1.0, ys, 1, I(64), None, None, 0, None) == bl.BL_ERR_SHAPE
+    g = L.bitlinear_attention_decode
+    assert g(None, A, A, A, A, A, 20, 5, 128, 64, 1e4, A, 0, None) == bl.BL_ERR_NULL
+    assert g(A, A, A, A, A, A, 20, 5, 64, 64, 1e4, A, 0, None) == bl.BL_ERR_SHAPE
+    assert g(A, A, A, A, A, A, 20, 6, 128, 64, 1e4, A, 0, None) == bl.BL_ERR_SHAPE
+    assert g(A, A, A, A, A, A, 20, 5, 128, 40000, 1e4, A, 0, None) == bl.BL_ERR_SHAPE
+    assert g(A + 2, A, A, A, A, A, 20, 5, 128, 64, 1e4, A, 0, None) == bl.BL_ERR_ALIGN
+    assert L.bitlinear_position_advance(None, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_position_advance(A + 2, None) == bl.BL_ERR_ALIGN
