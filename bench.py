@@ -324,7 +324,8 @@ def time_graph(graph, steps, world):
     return start.elapsed_time(end) / 1000.0
 
 
-def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda", pdl=False):
+def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda", pdl=False,
+                  force_fused=None):
     """Per-launch time of one shape, rotating distinct weight copies (>= 4x L2).
 
     pdl: consecutive launches (M = 1) overlap through programmatic dependent
@@ -345,7 +346,7 @@ def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda", pdl=Fals
     y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
     # the path bl.linear takes: fused dp4a GEMV for few tokens, else quantise +
     # tensor-core GEMM (both launches timed)
-    fused = M <= bl.GEMV_FUSED_MAX_M
+    fused = M <= bl.GEMV_FUSED_MAX_M if force_fused is None else force_fused
     if fused and pdl:
         call = lambda wt: bl.gemv_fused_multi([wt], x, outs=[y], pdl=True)  # noqa: E731
     elif fused:
@@ -389,7 +390,24 @@ def gemv_path(K, N, M, fused):
     ng = (N + 7) // 8
     if M == 1 and K % 256 == 0 and K <= 32768 and ng <= 64 * sms:
         return "fused streaming GEMV (producer warp, bulk copies, mbarrier ring)"
+    if 2 <= M <= 16 and K % 256 == 0 and ng <= 32 * sms:
+        return "fused multi-token streaming GEMV (one weight pass for all tokens)"
     return "fused dp4a GEMV (per-warp cp.async ring)"
+
+
+def small_batch_sweep(bl, device="cuda"):
+    """Config 3's timing: M in {1, 2, 4, 8, 16} on the four 2.4B shapes, the
+    path linear() takes (fused streaming GEMV; from 8 tokens the time of
+    quantise + tensor-core GEMM is given beside it)."""
+    out = []
+    for (K, N) in si.DECODE_SHAPES_2B:
+        for m in si.SMALL_BATCH_M:
+            r = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=True)
+            if m >= 8:
+                g = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=False)
+                r["tensor_core_us"] = g["us"]
+            out.append(r)
+    return out
 
 
 def isolated_binary(bl, K, N, iters=100, device="cuda"):
@@ -503,7 +521,7 @@ def rmsnorm_gemv_cost(bl, K, Ns, iters=200, device="cuda"):
 def decoder_tokens(bl, contexts=(512, 2048), tokens=64, device="cuda"):
     """The synthetic 2.4B decoder stack (30 layers: RMSNorm, q/k/v, RoPE +
     attention over a bf16 KV cache, o + residual, RMSNorm, gate/up, squared
-    ReLU gate, down + residual; 151 launches per token with PDL) replayed
+    ReLU gate, down + residual; 181 launches per token with PDL) replayed
     from a CUDA graph, one token per replay, at a given number of cached
     positions."""
     from bit_ternary_weight_b200.decoder import Decoder, DecoderConfig
@@ -531,7 +549,7 @@ def decoder_tokens(bl, contexts=(512, 2048), tokens=64, device="cuda"):
         t = s.elapsed_time(e) / 1000.0 / tokens
         out.append({"context": ctx, "tokens": tokens, "us_per_token": t * 1e6,
                     "tokens_per_s": 1.0 / t, "weight_GBps": dec.weight_bytes() / t / 1e9,
-                    "launches_per_token": 5 * cfg.layers + 1})
+                    "launches_per_token": 6 * cfg.layers + 1})
     assert bl.last_device_status() == 0
     del g, dec
     return out
@@ -766,8 +784,7 @@ def run_ours(args, world, rank, local):
                                           for (K, N) in si.DECODE_SHAPES_100B])
         measure("chained_100b_pdl", lambda: [isolated_gemv(bl, K, N, iters=200, device=device, pdl=True)
                                              for (K, N) in si.DECODE_SHAPES_100B])
-        measure("small_batch_2560x6912", lambda: [
-            isolated_gemv(bl, 2560, 6912, M=m, iters=100, device=device) for m in si.SMALL_BATCH_M])
+        measure("small_batch", lambda: small_batch_sweep(bl, device=device))
         measure("binary_100b", lambda: isolated_binary(bl, 8192, 28672, device=device))
         measure("bitplane_100b", lambda: [isolated_bitplane(bl, K, N, device=device)
                                           for (K, N) in si.DECODE_SHAPES_100B])

@@ -120,7 +120,8 @@ _SIGNATURES.update({
                                        ctypes.c_float, _vp, _int, _vp, _vp, _vp, ctypes.c_uint,
                                        _vp]),
     "bitlinear_attention_decode": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
-                                          ctypes.c_double, _vp, ctypes.c_uint, _vp]),
+                                          ctypes.c_double, _vp, _vp, _sz, ctypes.c_uint, _vp]),
+    "bitlinear_attention_workspace_bytes": (_sz, [_int, _int, _int]),
     "bitlinear_position_advance": (_int, [_vp, _vp]),
     "bitlinear_chain_plan_bytes": (_sz, [_int]),
     "bitlinear_chain_plan": (_int, [_int, ctypes.POINTER(ChainStepC), _vp, _sz, _vp]),
@@ -390,19 +391,30 @@ def decode_linear(weights, x: torch.Tensor, act: int = BL_ACT_PLAIN, x2=None, ga
     return outs
 
 
+def attention_workspace(H: int, Hkv: int, T_max: int, device) -> torch.Tensor:
+    """A zeroed workspace for attention_decode (reusable by ordered calls)."""
+    n = int(_lib.bitlinear_attention_workspace_bytes(H, Hkv, T_max))
+    if n == 0:
+        raise BitLinearError(BL_ERR_SHAPE, "bitlinear_attention_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
 def attention_decode(q, k, v, cache_k, cache_v, pos, H: int, Hkv: int, out=None,
-                     rope_base: float = 10000.0, pdl: bool = False):
+                     rope_base: float = 10000.0, workspace=None, pdl: bool = False):
     """One token's attention with RoPE over a bf16 cache [Hkv, T_max, 128];
     pos: int32 device scalar (this token's position; the cache row written)."""
     D = 128
     T_max = cache_k.shape[-2]
     if out is None:
         out = torch.empty(H * D, dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        workspace = attention_workspace(H, Hkv, T_max, q.device)
     with _on(q.device):
         _check(_lib.bitlinear_attention_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(cache_k),
                                                _ptr(cache_v), _ptr(pos), H, Hkv, D, T_max,
-                                               float(rope_base), _ptr(out),
-                                               BL_FLAG_PDL if pdl else 0, _stream(q.device)),
+                                               float(rope_base), _ptr(out), _ptr(workspace),
+                                               workspace.numel(), BL_FLAG_PDL if pdl else 0,
+                                               _stream(q.device)),
                "bitlinear_attention_decode")
     return out
 

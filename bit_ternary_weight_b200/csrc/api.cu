@@ -514,28 +514,40 @@ int bitlinear_decode_linear(int count, const uint8_t *const *packed, const float
     return launch_gemv_stream(b, true, s, gain, gt, eps, act == BL_ACT_RMSNORM);
 }
 
+size_t bitlinear_attention_workspace_bytes(int H, int Hkv, int T_max)
+{
+    if (H < 1 || Hkv < 1 || H % Hkv || H / Hkv > attention_max_group() || T_max < 1 ||
+        T_max > 32768)
+        return 0;
+    return attention_workspace_bytes(H, Hkv, T_max);
+}
+
 int bitlinear_attention_decode(const void *q, const void *k, const void *v, void *cache_k,
                                void *cache_v, const int32_t *pos, int H, int Hkv, int D,
-                               int T_max, double rope_base, void *out, unsigned flags,
-                               void *stream)
+                               int T_max, double rope_base, void *out, void *ws,
+                               size_t ws_bytes, unsigned flags, void *stream)
 {
     if (!q || !k || !v || !cache_k || !cache_v || !pos || !out)
         return BL_ERR_NULL;
-    if (H < 1 || Hkv < 1 || H % Hkv || D != 128 || T_max < 1 || T_max > 32768 ||
-        !(rope_base > 1.0) || !(rope_base < 1e30) || (flags & ~BL_FLAG_PDL) || H > 65535)
+    if (H < 1 || Hkv < 1 || H % Hkv || H / Hkv > attention_max_group() || D != 128 ||
+        T_max < 1 || T_max > 32768 || !(rope_base > 1.0) || !(rope_base < 1e30) ||
+        (flags & ~BL_FLAG_PDL) || Hkv > 65535)
         return BL_ERR_SHAPE;
     if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
          reinterpret_cast<uintptr_t>(cache_k) | reinterpret_cast<uintptr_t>(cache_v) |
-         reinterpret_cast<uintptr_t>(out)) & 7u || (reinterpret_cast<uintptr_t>(pos) & 3u))
+         reinterpret_cast<uintptr_t>(out)) & 15u || (reinterpret_cast<uintptr_t>(pos) & 3u) ||
+        !aligned16(ws))
         return BL_ERR_ALIGN;
     const DeviceInfo *di;
     int st = need_device(&di);
     if (st)
         return st;
-    if ((st = check_dev_ptrs({q, k, v, cache_k, cache_v, pos, out})))
+    if ((st = check_dev_ptrs({q, k, v, cache_k, cache_v, pos, out, ws})))
         return st;
+    if (!ws || ws_bytes < attention_workspace_bytes(H, Hkv, T_max))
+        return BL_ERR_WORKSPACE;
     return launch_attention_decode(q, k, v, cache_k, cache_v, pos, H, Hkv, D, T_max, rope_base, out,
-                                   flags, static_cast<cudaStream_t>(stream));
+                                   ws, flags, static_cast<cudaStream_t>(stream));
 }
 
 int bitlinear_position_advance(int32_t *pos, void *stream)

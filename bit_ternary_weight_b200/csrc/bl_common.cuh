@@ -65,6 +65,13 @@ __device__ __forceinline__ uint32_t ld_dep_u32(const void *p)
     return v;
 }
 
+__device__ __forceinline__ unsigned long long ld_dep_u64(const void *p)
+{
+    unsigned long long v;
+    asm volatile("ld.global.cg.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ uint32_t ld_dep_u16(const void *p)
 {
     unsigned short v;

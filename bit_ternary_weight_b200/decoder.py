@@ -1,7 +1,8 @@
 """A synthetic BitNet b1.58 decoder-layer stack for decode, on the library's
-kernels: every layer is five launches (RMSNorm + q/k/v BitLinears; RoPE +
-KV-cache append + attention; o BitLinear + residual; RMSNorm + gate/up
-BitLinears; squared-ReLU gate + down BitLinear + residual), chained with
+kernels: every layer is six launches (RMSNorm + q/k/v BitLinears; RoPE +
+KV-cache append + attention scores; softmax + values; o BitLinear +
+residual; RMSNorm + gate/up BitLinears; squared-ReLU gate + down BitLinear
++ residual), chained with
 programmatic dependent launch, one position advance per token, and the whole
 token capturable in a CUDA graph.
 
@@ -24,8 +25,8 @@ from dataclasses import dataclass, field
 
 import torch
 
-from . import (BL_ACT_PLAIN, BL_ACT_RELU2_GATE, BL_ACT_RMSNORM, attention_decode, decode_linear,
-               pack, position_advance)
+from . import (BL_ACT_PLAIN, BL_ACT_RELU2_GATE, BL_ACT_RMSNORM, attention_decode,
+               attention_workspace, decode_linear, pack, position_advance)
 
 
 @dataclass
@@ -121,18 +122,20 @@ class Decoder:
                         "v": torch.empty(c.kv_heads * c.head_dim, dtype=bf, device=dev),
                         "attn": torch.empty(c.heads * c.head_dim, dtype=bf, device=dev),
                         "gate": torch.empty(c.ffn, dtype=bf, device=dev),
-                        "up": torch.empty(c.ffn, dtype=bf, device=dev)}
+                        "up": torch.empty(c.ffn, dtype=bf, device=dev),
+                        "attn_ws": attention_workspace(c.heads, c.kv_heads, c.max_seq, dev)}
 
     def set_position(self, pos: int):
         self.pos.fill_(int(pos))
 
     def layer_step(self, L: DecoderLayer, pdl: bool = True):
-        """One layer for the current token (five launches)."""
+        """One layer for the current token (six launches)."""
         c, s, h = self.cfg, self.scratch, self.h
         decode_linear([L.q, L.k, L.v], h, BL_ACT_RMSNORM, gain=L.g_attn, eps=c.eps,
                       outs=[s["q"], s["k"], s["v"]], pdl=pdl)
         attention_decode(s["q"], s["k"], s["v"], L.cache_k, L.cache_v, self.pos, c.heads,
-                         c.kv_heads, out=s["attn"], rope_base=c.rope_base, pdl=pdl)
+                         c.kv_heads, out=s["attn"], rope_base=c.rope_base,
+                         workspace=s["attn_ws"], pdl=pdl)
         decode_linear([L.o], s["attn"], BL_ACT_PLAIN, outs=[h], resid=[h], pdl=pdl)
         decode_linear([L.gate, L.up], h, BL_ACT_RMSNORM, gain=L.g_ffn, eps=c.eps,
                       outs=[s["gate"], s["up"]], pdl=pdl)
@@ -141,7 +144,7 @@ class Decoder:
 
     def step(self, pdl: bool = True):
         """One decode step: the token in self.h through every layer, then the
-        position advances.  5 * layers + 1 launches."""
+        position advances.  6 * layers + 1 launches."""
         for L in self.layers:
             self.layer_step(L, pdl)
         position_advance(self.pos)

@@ -335,16 +335,28 @@ int bitlinear_decode_linear(int count, const uint8_t *const *packed,
  *                    the kernel (a CUDA graph can replay the call for the
  *                    next token after bitlinear_position_advance)
  *   out              device bf16 [H*D]
+ *   ws, ws_bytes     device workspace of at least
+ *                    bitlinear_attention_workspace_bytes(H, Hkv, T_max) bytes,
+ *                    16-byte aligned: scores, per-block maxima and fp64
+ *                    partial sums, and one arrival ticket per kv head.  It
+ *                    must be all zero before its first use; every call that
+ *                    completes leaves the tickets zero.  Calls ordered on one
+ *                    stream may share it; calls that can overlap may not.
  *   flags            0 or BL_FLAG_PDL (q, k, v may come from the kernel just
  *                    before; the cache and pos from earlier work)
- * D must be 128; H a multiple of Hkv; T_max <= 32768.  A position outside
- * [0, T_max) writes nothing and makes the next bitlinear_last_device_status()
- * return BL_ERR_SHAPE.
+ * Two launches on `stream` (scores, then values), over blocks of 64 cached
+ * positions.  D must be 128; H a multiple of Hkv with H / Hkv <= 8; T_max
+ * <= 32768.  A position outside [0, T_max) writes nothing and makes the next
+ * bitlinear_last_device_status() return BL_ERR_SHAPE.
  */
 int bitlinear_attention_decode(const void *q, const void *k, const void *v,
                                void *cache_k, void *cache_v, const int32_t *pos,
                                int H, int Hkv, int D, int T_max, double rope_base,
-                               void *out, unsigned flags, void *stream);
+                               void *out, void *ws, size_t ws_bytes,
+                               unsigned flags, void *stream);
+
+/* Bytes of workspace bitlinear_attention_decode needs (0 if out of range). */
+size_t bitlinear_attention_workspace_bytes(int H, int Hkv, int T_max);
 
 /* *pos += 1 on the device (after a token's last attention call). */
 int bitlinear_position_advance(int32_t *pos, void *stream);

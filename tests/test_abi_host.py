@@ -248,10 +248,14 @@ def test_decoder_entry_argument_errors(bl):
     assert f(1, pk, sc, I(64), 256, 0, A, 1, None, None, 0, 1e-5, ys, 0, I(64), P(A), None, 0, None) == bl.BL_ERR_DTYPE
     assert f(1, pk, sc, I(64), 256, 1, A, 1, None, None, 0, -1.0, ys, 1, I(64), None, None, 0, None) == bl.BL_ERR_SHAPE
     g = L.bitlinear_attention_decode
-    assert g(None, A, A, A, A, A, 20, 5, 128, 64, 1e4, A, 0, None) == bl.BL_ERR_NULL
-    assert g(A, A, A, A, A, A, 20, 5, 64, 64, 1e4, A, 0, None) == bl.BL_ERR_SHAPE
-    assert g(A, A, A, A, A, A, 20, 6, 128, 64, 1e4, A, 0, None) == bl.BL_ERR_SHAPE
-    assert g(A, A, A, A, A, A, 20, 5, 128, 40000, 1e4, A, 0, None) == bl.BL_ERR_SHAPE
-    assert g(A + 2, A, A, A, A, A, 20, 5, 128, 64, 1e4, A, 0, None) == bl.BL_ERR_ALIGN
+    nb = L.bitlinear_attention_workspace_bytes(20, 5, 64)
+    assert nb > 20 * 64 * 4 and L.bitlinear_attention_workspace_bytes(20, 6, 64) == 0
+    assert L.bitlinear_attention_workspace_bytes(40, 2, 64) == 0      # 20 query heads per kv head
+    assert g(None, A, A, A, A, A, 20, 5, 128, 64, 1e4, A, A, nb, 0, None) == bl.BL_ERR_NULL
+    assert g(A, A, A, A, A, A, 20, 5, 64, 64, 1e4, A, A, nb, 0, None) == bl.BL_ERR_SHAPE
+    assert g(A, A, A, A, A, A, 20, 6, 128, 64, 1e4, A, A, nb, 0, None) == bl.BL_ERR_SHAPE
+    assert g(A, A, A, A, A, A, 20, 5, 128, 40000, 1e4, A, A, nb, 0, None) == bl.BL_ERR_SHAPE
+    assert g(A + 8, A, A, A, A, A, 20, 5, 128, 64, 1e4, A, A, nb, 0, None) == bl.BL_ERR_ALIGN
+    assert g(A, A, A, A, A, A, 20, 5, 128, 64, 1e4, A, A + 8, nb, 0, None) == bl.BL_ERR_ALIGN
     assert L.bitlinear_position_advance(None, None) == bl.BL_ERR_NULL
     assert L.bitlinear_position_advance(A + 2, None) == bl.BL_ERR_ALIGN

@@ -509,3 +509,69 @@ def test_row_split_shards_equal_unsplit(bl, world, M):
         R = p[0].rows_per_rank
         full = buf.view(world, M, R).permute(1, 0, 2).reshape(M, world * R)[:, :N]
         compare_outputs(full, y_o)
+
+
+# ------------------------------------------------------------------ small batches on the streaming kernel
+
+@pytest.mark.parametrize("M", [2, 3, 5, 8, 13, 16])
+@pytest.mark.parametrize("K,Ns", [(2560, [6912]), (6912, [2560]), (2560, [2560, 640, 640]),
+                                  (256, [1001]), (8192, [3000])])
+def test_small_batch_streaming_kernel(bl, M, K, Ns):
+    """2 .. 16 tokens with K a multiple of 256 run the multi-token streaming
+    kernel: fused (bf16 and fp32 x) for one or several products, and on
+    pre-quantised activations (bitlinear_gemv, below 8 tokens), integers and
+    outputs equal to the oracle's."""
+    for xdtype in (torch.bfloat16, torch.float32):
+        x = si.activations(M, K, seed=M * 31 + K, dtype=xdtype)
+        ws, refs = [], []
+        for i, N in enumerate(Ns):
+            W = si.weight(N, K, seed=3000 + 17 * i + N + M)
+            g, codes, _ = oracle_weight(W)
+            refs.append(_oracle_gemv(g, codes, x))
+            ws.append(_pack_gpu(bl, W))
+        accs = [torch.empty(M, N, dtype=torch.int32, device=dev()) for N in Ns]
+        big = [torch.full((M, N + 40), -3.0, dtype=torch.bfloat16, device=dev()) for N in Ns]
+        outs = [b[:, :N] for b, N in zip(big, Ns)]
+        bl.gemv_fused_multi(ws, x.to(dev()), outs=outs, acc_dbgs=accs)
+        torch.cuda.synchronize()
+        for (y_o, acc_o), y, acc, b, N in zip(refs, outs, accs, big, Ns):
+            np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+            compare_outputs(y, y_o)
+            assert (b[:, N:] == -3.0).all()
+        if M < 8 and len(Ns) == 1:
+            q, d, r = bl.quantize_act(x.to(dev()))
+            acc = torch.empty(M, Ns[0], dtype=torch.int32, device=dev())
+            y = bl.gemv(ws[0], q, d, r, acc_dbg=acc)
+            torch.cuda.synchronize()
+            np.testing.assert_array_equal(acc.cpu().numpy(), refs[0][1])
+            compare_outputs(y, refs[0][0])
+    assert bl.last_device_status() == 0
+
+
+def test_small_batch_pdl_chain_in_graph(bl):
+    """Eight tokens through a six-deep dependent chain of streaming launches
+    with programmatic dependent launch inside a CUDA graph."""
+    K, M = 2560, 8
+    Ws = [si.weight(K, K, seed=170 + i) for i in range(6)]
+    oracles = [oracle_weight(W) for W in Ws]
+    ws = [_pack_gpu(bl, W) for W in Ws]
+    x0 = si.activations(M, K, seed=171)
+    xs = [x0.to(dev())] + [torch.empty(M, K, dtype=torch.bfloat16, device=dev()) for _ in Ws]
+
+    def run():
+        for i, w in enumerate(ws):
+            bl.gemv_fused_multi([w], xs[i], outs=[xs[i + 1]], pdl=True)
+    run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    for t in xs[1:]:
+        t.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    x = x0
+    for i, (gam, codes, _) in enumerate(oracles):
+        y_o, _ = _oracle_gemv(gam, codes, x)
+        compare_outputs(xs[i + 1], y_o)
+        x = torch.from_numpy(oracle.to_bf16_bits(y_o).view(np.int16)).view(torch.bfloat16).reshape(M, K)
