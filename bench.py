@@ -396,16 +396,19 @@ def gemv_path(K, N, M, fused):
 
 
 def small_batch_sweep(bl, device="cuda"):
-    """Config 3's timing: M in {1, 2, 4, 8, 16} on the four 2.4B shapes, the
-    path linear() takes (fused streaming GEMV; from 8 tokens the time of
-    quantise + tensor-core GEMM is given beside it)."""
+    """Config 3's timing: M in {1, 2, 4, 8, 16} on the four 2.4B shapes.
+    `us` / `GBps` are the path linear() takes (bl.fused_gemv_preferred); from
+    8 tokens both paths are timed (`fused_us`, `tensor_core_us`)."""
     out = []
     for (K, N) in si.DECODE_SHAPES_2B:
         for m in si.SMALL_BATCH_M:
-            r = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=True)
+            f = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=True)
+            r = dict(f)
             if m >= 8:
                 g = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=False)
-                r["tensor_core_us"] = g["us"]
+                r["fused_us"], r["tensor_core_us"] = f["us"], g["us"]
+                if not bl.fused_gemv_preferred(m, N, K):
+                    r.update(us=g["us"], GBps=g["GBps"], path=g["path"])
             out.append(r)
     return out
 

@@ -120,7 +120,9 @@ _SIGNATURES.update({
                                        ctypes.c_float, _vp, _int, _vp, _vp, _vp, ctypes.c_uint,
                                        _vp]),
     "bitlinear_attention_decode": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
-                                          ctypes.c_double, _vp, _vp, _sz, ctypes.c_uint, _vp]),
+                                          ctypes.c_double, _vp, _vp, _vp, _sz, ctypes.c_uint,
+                                          _vp]),
+    "bitlinear_rope_table": (_int, [_int, _int, ctypes.c_double, _vp, _vp]),
     "bitlinear_attention_workspace_bytes": (_sz, [_int, _int, _int]),
     "bitlinear_position_advance": (_int, [_vp, _vp]),
     "bitlinear_chain_plan_bytes": (_sz, [_int]),
@@ -399,8 +401,17 @@ def attention_workspace(H: int, Hkv: int, T_max: int, device) -> torch.Tensor:
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
+def rope_table(T_max: int, rope_base: float = 10000.0, device="cuda") -> torch.Tensor:
+    """(cos, sin) of every (position, pair) angle, fp32 [T_max, 64, 2]."""
+    tab = torch.empty(T_max, 64, 2, dtype=torch.float32, device=device)
+    with _on(tab.device):
+        _check(_lib.bitlinear_rope_table(128, T_max, float(rope_base), _ptr(tab),
+                                         _stream(tab.device)), "bitlinear_rope_table")
+    return tab
+
+
 def attention_decode(q, k, v, cache_k, cache_v, pos, H: int, Hkv: int, out=None,
-                     rope_base: float = 10000.0, workspace=None, pdl: bool = False):
+                     rope_base: float = 10000.0, workspace=None, table=None, pdl: bool = False):
     """One token's attention with RoPE over a bf16 cache [Hkv, T_max, 128];
     pos: int32 device scalar (this token's position; the cache row written)."""
     D = 128
@@ -412,7 +423,8 @@ def attention_decode(q, k, v, cache_k, cache_v, pos, H: int, Hkv: int, out=None,
     with _on(q.device):
         _check(_lib.bitlinear_attention_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(cache_k),
                                                _ptr(cache_v), _ptr(pos), H, Hkv, D, T_max,
-                                               float(rope_base), _ptr(out), _ptr(workspace),
+                                               float(rope_base), _ptr(table), _ptr(out),
+                                               _ptr(workspace),
                                                workspace.numel(), BL_FLAG_PDL if pdl else 0,
                                                _stream(q.device)),
                "bitlinear_attention_decode")
@@ -514,14 +526,23 @@ def gemm(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc
     return out
 
 
-GEMV_FUSED_MAX_M = 7   # from 8 tokens on, quantise + tensor-core GEMM is faster
+GEMV_FUSED_MAX_M = 8          # up to here the fused streaming GEMV is the faster path
+GEMV_FUSED_SMALL_W_MAX_M = 16  # ... and up to here for weights of at most
+GEMV_SMALL_W = 4 * 1024 * 1024  # this many entries (measured on B200)
+
+
+def fused_gemv_preferred(M: int, N: int, K: int) -> bool:
+    """Whether the fused dp4a GEMV beats quantise + tensor-core GEMM for M tokens."""
+    if M * K > 163840:
+        return False
+    return M <= GEMV_FUSED_MAX_M or (M <= GEMV_FUSED_SMALL_W_MAX_M and N * K <= GEMV_SMALL_W)
 
 
 def linear(w: TernaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16):
-    """y = BitLinear(x): the fused dp4a GEMV for up to 7 tokens, else quantise +
-    tensor-core GEMM."""
+    """y = BitLinear(x): the fused dp4a GEMV for few tokens (see
+    fused_gemv_preferred), else quantise + tensor-core GEMM."""
     x2 = x.reshape(-1, x.shape[-1])
-    if x2.shape[0] <= GEMV_FUSED_MAX_M and x2.shape[0] * w.K <= 163840:
+    if fused_gemv_preferred(x2.shape[0], w.N, w.K):
         y = gemv_fused(w, x2, out_dtype)
     else:
         q, d, r = quantize_act(x2)

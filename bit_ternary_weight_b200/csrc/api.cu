@@ -293,7 +293,8 @@ int check_gemv_common(const uint8_t *packed, const float *w_scale, int64_t N,
 }
 
 constexpr int64_t kGemvMaxM = 16;
-constexpr int64_t kGemvTensorM = 8;     // bitlinear_gemv runs on the tcgen05 path from here on
+constexpr int64_t kGemvTensorM = 8;     // above this, bitlinear_gemv may take the tcgen05 path
+constexpr int64_t kGemvSmallW = int64_t(4) << 20;   // weights up to this stay on dp4a to 16 tokens
 constexpr int64_t kGemvMaxMK = 163840;
 
 }  // namespace
@@ -318,9 +319,10 @@ int bitlinear_gemv(const uint8_t *packed, const float *w_scale, int64_t N, int64
     if ((st = check_dev_ptrs({packed, w_scale, q, d, rowsum, y, acc_dbg})))
         return st;
     GemvArgs a{packed, w_scale, N, K, M, q, d, rowsum, nullptr, BL_F32, 0, y, yt, ldy, acc_dbg};
-    // from kGemvTensorM tokens on, dp4a work grows with M while the tensor
-    // cores are idle: the product runs on the tcgen05 path (same results)
-    if (M >= kGemvTensorM)
+    // beyond kGemvTensorM tokens (on weights of more than kGemvSmallW entries)
+    // the dp4a work outgrows the weight stream while the tensor cores are idle:
+    // the product runs on the tcgen05 path (same results)
+    if (M > kGemvTensorM && N * K > kGemvSmallW)
         return launch_gemm(a, nullptr, 0, static_cast<cudaStream_t>(stream));
     return launch_gemv(a, false, static_cast<cudaStream_t>(stream));
 }
@@ -522,10 +524,27 @@ size_t bitlinear_attention_workspace_bytes(int H, int Hkv, int T_max)
     return attention_workspace_bytes(H, Hkv, T_max);
 }
 
+int bitlinear_rope_table(int D, int T_max, double rope_base, float *table, void *stream)
+{
+    if (!table)
+        return BL_ERR_NULL;
+    if (D != 128 || T_max < 1 || T_max > 32768 || !(rope_base > 1.0) || !(rope_base < 1e30))
+        return BL_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(table) & 7u)
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if ((st = check_dev_ptrs({table})))
+        return st;
+    return launch_rope_table(table, D, T_max, rope_base, static_cast<cudaStream_t>(stream));
+}
+
 int bitlinear_attention_decode(const void *q, const void *k, const void *v, void *cache_k,
                                void *cache_v, const int32_t *pos, int H, int Hkv, int D,
-                               int T_max, double rope_base, void *out, void *ws,
-                               size_t ws_bytes, unsigned flags, void *stream)
+                               int T_max, double rope_base, const float *rope_table, void *out,
+                               void *ws, size_t ws_bytes, unsigned flags, void *stream)
 {
     if (!q || !k || !v || !cache_k || !cache_v || !pos || !out)
         return BL_ERR_NULL;
@@ -536,18 +555,18 @@ int bitlinear_attention_decode(const void *q, const void *k, const void *v, void
     if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
          reinterpret_cast<uintptr_t>(cache_k) | reinterpret_cast<uintptr_t>(cache_v) |
          reinterpret_cast<uintptr_t>(out)) & 15u || (reinterpret_cast<uintptr_t>(pos) & 3u) ||
-        !aligned16(ws))
+        !aligned16(ws) || (reinterpret_cast<uintptr_t>(rope_table) & 7u))
         return BL_ERR_ALIGN;
     const DeviceInfo *di;
     int st = need_device(&di);
     if (st)
         return st;
-    if ((st = check_dev_ptrs({q, k, v, cache_k, cache_v, pos, out, ws})))
+    if ((st = check_dev_ptrs({q, k, v, cache_k, cache_v, pos, out, ws, rope_table})))
         return st;
     if (!ws || ws_bytes < attention_workspace_bytes(H, Hkv, T_max))
         return BL_ERR_WORKSPACE;
-    return launch_attention_decode(q, k, v, cache_k, cache_v, pos, H, Hkv, D, T_max, rope_base, out,
-                                   ws, flags, static_cast<cudaStream_t>(stream));
+    return launch_attention_decode(q, k, v, cache_k, cache_v, pos, H, Hkv, D, T_max, rope_base,
+                                   rope_table, out, ws, flags, static_cast<cudaStream_t>(stream));
 }
 
 int bitlinear_position_advance(int32_t *pos, void *stream)

@@ -24,6 +24,10 @@
 // they may differ in the last fp64 bit, which moves an fp32 result only on
 // such a boundary too.
 //
+// RoPE's cosines and sines come from a table of every (position, pair) that
+// bitlinear_rope_table computes once (same definition), or are computed in
+// the scores kernel when no table is given.
+//
 // Design: two launches over blocks of 64 cached positions, so that the work
 // of one token spreads over (kv heads x position blocks) CTAs instead of one
 // CTA per head walking every position.  The position pos is a device scalar
@@ -63,6 +67,7 @@ struct AttnParams {
     const int32_t *pos;
     int H, Hkv, T_max, nblk;
     double rope_base;
+    const float2 *rope;                   // NULL, or (cos, sin) [T_max][D/2] of every angle
     __nv_bfloat16 *out;                   // [H*D]
     // workspace
     float *sc;                            // [H][T_max] scores, then weights
@@ -80,12 +85,19 @@ __device__ __forceinline__ uint32_t f32_bf16_bits(float v)
     return __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
-// Rotate pair i of a head vector x (bf16) at position pos; the two rotated
-// values rounded to bf16 (as fp32).
-__device__ __forceinline__ void rope_pair(const __nv_bfloat16 *x, int i, int pos, double base, float &o0, float &o1)
+// cos and sin of the angle pos * base^(-2i / D), each computed in fp64 and
+// rounded to fp32.
+__device__ __forceinline__ float2 rope_angle(int pos, int i, double base)
 {
     const double ang = double(pos) * pow(base, -double(2 * i) / double(kHeadDim));
-    const float c = __double2float_rn(cos(ang)), s = __double2float_rn(sin(ang));
+    return make_float2(__double2float_rn(cos(ang)), __double2float_rn(sin(ang)));
+}
+
+// Rotate pair i of a head vector x (bf16) by (cos, sin) cs; the two rotated
+// values rounded to bf16 (as fp32).
+__device__ __forceinline__ void rope_pair(const __nv_bfloat16 *x, int i, float2 cs, float &o0, float &o1)
+{
+    const float c = cs.x, s = cs.y;
     const float a = bf16_bits_f32(ld_dep_u16(x + 2 * i)), b = bf16_bits_f32(ld_dep_u16(x + 2 * i + 1));
     const float r0 = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
     const float r1 = __fadd_rn(__fmul_rn(a, s), __fmul_rn(b, c));
@@ -110,6 +122,7 @@ __global__ void __launch_bounds__(kScoreThreads) attn_scores_kernel(const AttnPa
 {
     __shared__ float qs[kMaxGroup][kHeadDim];     // rotated queries of the group
     __shared__ float ks[kHeadDim];                // rotated new key (block holding pos)
+    __shared__ float2 cs[kHeadDim / 2];           // (cos, sin) of the token's angles
     __shared__ float wmax[kScoreThreads / 32][kMaxGroup];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kv = blockIdx.x, blk = blockIdx.y;
@@ -124,17 +137,20 @@ __global__ void __launch_bounds__(kScoreThreads) attn_scores_kernel(const AttnPa
         return;
     const int j1 = min(j0 + kPosBlock, pos + 1);
     const bool has_new = pos < j0 + kPosBlock;
+    if (tid < kHeadDim / 2)
+        cs[tid] = p.rope ? __ldg(p.rope + size_t(pos) * (kHeadDim / 2) + tid) : rope_angle(pos, tid, p.rope_base);
+    __syncthreads();
     for (int t = tid; t < G * (kHeadDim / 2); t += kScoreThreads) {
         const int g = t / (kHeadDim / 2), i = t % (kHeadDim / 2);
         float a, b;
-        rope_pair(p.q + (kv * G + g) * kHeadDim, i, pos, p.rope_base, a, b);
+        rope_pair(p.q + (kv * G + g) * kHeadDim, i, cs[i], a, b);
         qs[g][2 * i] = a;
         qs[g][2 * i + 1] = b;
     }
     const size_t head_base = size_t(kv) * p.T_max * kHeadDim;
     if (has_new && tid < kHeadDim / 2) {
         float a, b;
-        rope_pair(p.k + kv * kHeadDim, tid, pos, p.rope_base, a, b);
+        rope_pair(p.k + kv * kHeadDim, tid, cs[tid], a, b);
         ks[2 * tid] = a;
         ks[2 * tid + 1] = b;
         p.cache_k[head_base + size_t(pos) * kHeadDim + 2 * tid] = __float2bfloat16_rn(a);
@@ -302,11 +318,14 @@ __global__ void __launch_bounds__(kValueThreads) attn_values_kernel(const AttnPa
             num = __dadd_rn(num, part[q4][g][d]);
         p.bnum[(size_t(kv * G + g) * p.nblk + blk) * kHeadDim + d] = num;
     }
-    if (tid < G) {
-        double S = 0.0;
-        for (int jj = 0; jj < j1 - j0; ++jj)
-            S = __dadd_rn(S, double(ew[tid][jj]));
-        p.bsum[size_t(kv * G + tid) * p.nblk + blk] = S;
+    for (int g = tid >> 5; g < G; g += kValueThreads / 32) {
+        const int lane = tid & 31;
+        double S = __dadd_rn(double(ew[g][lane]), double(ew[g][lane + 32]));   // e_j = 0 beyond j1
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            S = __dadd_rn(S, __shfl_xor_sync(0xffffffffu, S, o));
+        if (lane == 0)
+            p.bsum[size_t(kv * G + g) * p.nblk + blk] = S;
     }
     // the last block of this kv head to finish combines the blocks
     __threadfence();
@@ -331,6 +350,16 @@ __global__ void __launch_bounds__(kValueThreads) attn_values_kernel(const AttnPa
     }
     if (tid == 0)
         p.ticket[kv] = 0u;
+}
+
+// (cos, sin) of pos * base^(-2i / D) for every position and pair, fp64 then
+// fp32 (the same values the attention kernels compute without a table).
+__global__ void rope_table_kernel(float2 *tab, int T_max, double base)
+{
+    const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= int64_t(T_max) * (kHeadDim / 2))
+        return;
+    tab[idx] = rope_angle(int(idx / (kHeadDim / 2)), int(idx % (kHeadDim / 2)), base);
 }
 
 __global__ void position_advance_kernel(int32_t *pos)
@@ -382,9 +411,18 @@ size_t attention_workspace_bytes(int H, int Hkv, int T_max) { return ws_layout(H
 
 int attention_max_group() { return kMaxGroup; }
 
+int launch_rope_table(float *tab, int D, int T_max, double base, cudaStream_t s)
+{
+    if (D != kHeadDim)
+        return BL_ERR_SHAPE;
+    const int64_t n = int64_t(T_max) * (kHeadDim / 2);
+    rope_table_kernel<<<unsigned((n + 255) / 256), 256, 0, s>>>(reinterpret_cast<float2 *>(tab), T_max, base);
+    return launch_status();
+}
+
 int launch_attention_decode(const void *q, const void *k, const void *v, void *cache_k, void *cache_v,
                             const int32_t *pos, int H, int Hkv, int D, int T_max, double rope_base,
-                            void *out, void *ws, unsigned flags, cudaStream_t s)
+                            const float *rope, void *out, void *ws, unsigned flags, cudaStream_t s)
 {
     const DeviceInfo *di = device_info();
     if (!di)
@@ -405,6 +443,7 @@ int launch_attention_decode(const void *q, const void *k, const void *v, void *c
     p.T_max = T_max;
     p.nblk = (T_max + kPosBlock - 1) / kPosBlock;
     p.rope_base = rope_base;
+    p.rope = reinterpret_cast<const float2 *>(rope);
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.sc = reinterpret_cast<float *>(base + w.sc);
     p.bmax = reinterpret_cast<float *>(base + w.bmax);

@@ -122,7 +122,7 @@ bool gemv_stream_applies(const GemvBatch &b, int sm_count);
 int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s, const void *gain, int gt,
                        float eps, bool norm);
 // Small batches (2 .. 16 tokens) on the streaming design (gemv_stream_mt.cu).
-bool gemv_stream_mt_applies(const GemvBatch &b, int sm_count, int max_smem);
+bool gemv_stream_mt_applies(const GemvBatch &b, bool fused, int sm_count, int max_smem);
 int launch_gemv_stream_mt(const GemvBatch &b, bool fused, cudaStream_t s);
 
 // The same with the squared-ReLU gate in front: the token is relu(x)^2 * x2
@@ -132,9 +132,10 @@ int launch_gemv_stream_relu2(const GemvBatch &b, const void *x2, cudaStream_t s)
 // Decode attention of one token (attention.cu).
 size_t attention_workspace_bytes(int H, int Hkv, int T_max);
 int attention_max_group();
+int launch_rope_table(float *tab, int D, int T_max, double base, cudaStream_t s);
 int launch_attention_decode(const void *q, const void *k, const void *v, void *cache_k, void *cache_v,
                             const int32_t *pos, int H, int Hkv, int D, int T_max, double rope_base,
-                            void *out, void *ws, unsigned flags, cudaStream_t s);
+                            const float *rope, void *out, void *ws, unsigned flags, cudaStream_t s);
 int launch_position_advance(int32_t *pos, cudaStream_t s);
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);

@@ -640,7 +640,7 @@ int launch_gemv_batch(const GemvBatch &b, bool fused, cudaStream_t s)
     // 2 .. 16 tokens: its multi-token form (one weight pass for all tokens)
     if (gemv_stream_applies(b, di->sm_count))
         return launch_gemv_stream(b, fused, s);
-    if (gemv_stream_mt_applies(b, di->sm_count, di->max_smem_optin))
+    if (gemv_stream_mt_applies(b, fused, di->sm_count, di->max_smem_optin))
         return launch_gemv_stream_mt(b, fused, s);
     Params p{};
     p.count = b.count;

@@ -12,9 +12,11 @@
 //     of the CTA's row groups (at most four groups per stage), exactly as in
 //     gemv_stream.cu; eight consumer warps take piece w (and w + 8) of every
 //     group of a stage.
-//   * The prologue quantises all M tokens (absmax per token: one block
-//     reduction for all of them), each warp only the activations of its own
-//     pieces, into int8 rows in shared memory (or copies pre-quantised q).
+//   * The prologue quantises the M tokens into int8 rows in shared memory
+//     (or copies pre-quantised q): one warp per token, the whole row loaded
+//     into registers at once (raw 16-byte vectors; rows above 4096 bf16
+//     elements in two halves), a warp reduction for its absmax (K <= 8192;
+//     fp32 input K <= 4096).
 //   * Per stage a consumer lane expands each group's 16-byte piece once into
 //     sixteen code words c = (word >> 2i) & 0x03030303 (stored codes s =
 //     code + 1 of four consecutive k), then, token by token, loads the
@@ -37,6 +39,7 @@ constexpr int kMtThreads = 32 * (kMtKC + 1);
 constexpr int kMtMaxTokens = 16;
 constexpr int kMtMaxSet = 4;                     // groups per stage
 constexpr int kMtMaxGroupsPerCta = 32;
+constexpr int64_t kMtMaxK = 8192;                // a token's row in one warp's registers
 
 enum { MT_Q = 0, MT_X_BF16 = 1, MT_X_F32 = 2 };
 
@@ -62,8 +65,7 @@ struct MtSmem {
     uint64_t full[kStages];
     uint64_t empty[kStages];
     int abort_flag;
-    float bmax[kMtMaxTokens][kMtKC];
-    int bsum[kMtMaxTokens][kMtKC];
+    int bsum[kMtMaxTokens][1];     // each token's row sum
     float d[kMtMaxTokens];
     float wscale[kGemvMaxProblems];
     int sacc[kMtMaxTokens][kMtMaxGroupsPerCta][8];
@@ -83,51 +85,114 @@ __device__ __forceinline__ int mt_locate(const MtParams &p, int64_t G)
 
 __device__ __forceinline__ void mt_sync() { named_barrier(1, 32 * kMtKC); }
 
-// Quantise the M tokens into qs [M][K]: each warp the activations of its own
-// pieces (256 k each: pieces w, w + 8, ...), one block reduction for the M
-// absmax values; x is read twice (from L2).
-template <int XT>
+// Quantise the M tokens into qs [M][K]: warp w takes tokens w, w + 8, ...,
+// each a whole row: the row's 16-byte chunks are all loaded before any is
+// used (CHM per lane, so one round trip to L2 per token), the absmax is a
+// warp reduction, and the warp quantises from its registers.  Other warps
+// read these activations after the block barrier that follows.
+template <int XT, int CHM>
+struct MtRow {
+    static constexpr int V = XT == BL_BF16 ? 1 : 2;   // 16-byte vectors per chunk of 8 elements
+    uint4 raw[CHM * V];
+
+    // chunks lane + 32 (i0 + i), i < CHM, of token m's row
+    __device__ __forceinline__ void load(const MtParams &p, int m, int i0, int lane, int chunks)
+    {
+#pragma unroll
+        for (int i = 0; i < CHM; ++i) {
+            const int c = lane + 32 * (i0 + i);
+#pragma unroll
+            for (int v = 0; v < V; ++v)
+                raw[V * i + v] = c < chunks
+                    ? ld_dep_v4(static_cast<const unsigned char *>(p.x) +
+                                (int64_t(m) * p.ldx + int64_t(c) * 8) * (XT == BL_BF16 ? 2 : 4) + 16 * v)
+                    : make_uint4(0, 0, 0, 0);
+        }
+    }
+    __device__ __forceinline__ void f32(int i, float (&f)[8]) const
+    {
+        if constexpr (XT == BL_BF16) {
+            bf16x8_f32(raw[i], f);
+        } else {
+            const uint4 a = raw[2 * i], b = raw[2 * i + 1];
+            f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y);
+            f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+            f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y);
+            f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+        }
+    }
+    __device__ __forceinline__ float amax() const
+    {
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < CHM; ++i) {
+            float f[8];
+            f32(i, f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                a = fmaxf(a, fabsf(f[e]));
+        }
+        return a;
+    }
+    __device__ __forceinline__ void quantise(int8_t *qrow, int i0, int lane, int chunks, float s, int &sum) const
+    {
+#pragma unroll
+        for (int i = 0; i < CHM; ++i) {
+            const int c = lane + 32 * (i0 + i);
+            if (c < chunks) {
+                float f[8];
+                f32(i, f);
+                *reinterpret_cast<uint2 *>(qrow + int64_t(c) * 8) = quant8(f, s, sum);
+            }
+        }
+    }
+};
+
+// Quantise the M tokens into qs [M][K]: warp w takes tokens w, w + 8, ...,
+// each a whole row: CHM 16-byte chunks per lane loaded before any is used
+// (one round trip to L2 per token), the absmax a warp reduction, the
+// quantisation from the registers.  HALVES = 2 (rows longer than 16 chunks
+// per lane): the two halves in turn -- load the first, load the second
+// (absmax of both), quantise the second, load the first again and quantise
+// it -- so that only half a row is live.  Other warps read these activations
+// after the block barrier at the end.
+template <int XT, int CHM, int HALVES>
 __device__ __forceinline__ void mt_quantize(const MtParams &p, MtSmem &sm, int8_t *qs)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int P = int(p.K / 256);
-    for (int m = 0; m < p.M; ++m) {
-        float amax = 0.0f;
-#pragma unroll 4
-        for (int j = warp; j < P; j += kMtKC) {
-            float f[8];
-            load8<XT, true>(p.x, int64_t(m) * p.ldx + (int64_t(j) * 32 + lane) * 8, f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                amax = fmaxf(amax, fabsf(f[e]));
+    const int chunks = int(p.K / 8);
+    for (int m = warp; m < p.M; m += kMtKC) {
+        int8_t *qrow = qs + int64_t(m) * p.K;
+        MtRow<XT, CHM> row;
+        float a;
+        if constexpr (HALVES == 1) {
+            row.load(p, m, 0, lane, chunks);
+            a = row.amax();
+        } else {
+            row.load(p, m, 0, lane, chunks);
+            a = row.amax();
+            row.load(p, m, CHM, lane, chunks);
+            a = fmaxf(a, row.amax());
         }
         // maxima are >= 0 and finite: bit patterns order like the values
-        const uint32_t wm = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
-        if (lane == 0)
-            sm.bmax[m][warp] = __uint_as_float(wm);
-    }
-    mt_sync();
-    for (int m = 0; m < p.M; ++m) {
-        float a = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kMtKC; ++w)
-            a = fmaxf(a, sm.bmax[m][w]);
+        a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(a)));
         const float a_eff = fmaxf(a, kEps);
         const float s = __fdiv_rn(kQb, a_eff);
-        if (threadIdx.x == 0)
-            sm.d[m] = __fdiv_rn(a_eff, kQb);
         int sum = 0;
-#pragma unroll 4
-        for (int j = warp; j < P; j += kMtKC) {
-            float f[8];
-            load8<XT, true>(p.x, int64_t(m) * p.ldx + (int64_t(j) * 32 + lane) * 8, f);
-            *reinterpret_cast<uint2 *>(qs + int64_t(m) * p.K + (j * 32 + lane) * 8) = quant8(f, s, sum);
+        if constexpr (HALVES == 1) {
+            row.quantise(qrow, 0, lane, chunks, s, sum);
+        } else {
+            row.quantise(qrow, CHM, lane, chunks, s, sum);
+            row.load(p, m, 0, lane, chunks);
+            row.quantise(qrow, 0, lane, chunks, s, sum);
         }
         sum = __reduce_add_sync(0xffffffffu, sum);
-        if (lane == 0)
-            sm.bsum[m][warp] = sum;
+        if (lane == 0) {
+            sm.bsum[m][0] = sum;
+            sm.d[m] = __fdiv_rn(a_eff, kQb);
+        }
     }
-    __syncwarp();
+    mt_sync();
 }
 
 __device__ __forceinline__ void mt_copy_q(const MtParams &p, MtSmem &sm, int8_t *qs)
@@ -139,10 +204,9 @@ __device__ __forceinline__ void mt_copy_q(const MtParams &p, MtSmem &sm, int8_t 
             if (lane < 16)
                 *reinterpret_cast<uint4 *>(qs + int64_t(m) * p.K + j * 256 + lane * 16) =
                     ld_dep_v4(p.q + int64_t(m) * p.K + int64_t(j) * 256 + lane * 16);
-        if (lane == 0) {
-            sm.bsum[m][warp] = warp == 0 ? int(ld_dep_u32(p.rowsum + m)) : 0;
-            if (warp == 0)
-                sm.d[m] = __uint_as_float(ld_dep_u32(p.d + m));
+        if (lane == 0 && warp == 0) {
+            sm.bsum[m][0] = int(ld_dep_u32(p.rowsum + m));
+            sm.d[m] = __uint_as_float(ld_dep_u32(p.d + m));
         }
     }
     __syncwarp();
@@ -221,7 +285,7 @@ __device__ __forceinline__ void mt_flush(int rg, int M, int (&acc)[kMtMaxSet][MT
     }
 }
 
-template <int MT, int MODE>
+template <int MT, int MODE, int CHM>
 __global__ void __launch_bounds__(kMtThreads, 1) gemv_stream_mt_kernel(const MtParams p)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -307,8 +371,9 @@ __global__ void __launch_bounds__(kMtThreads, 1) gemv_stream_mt_kernel(const MtP
     if constexpr (MODE == MT_Q)
         mt_copy_q(p, sm, qs);
     else
-        mt_quantize<MODE == MT_X_BF16 ? BL_BF16 : BL_F32>(p, sm, qs);
-    // (each warp reads only the activations it wrote itself)
+        mt_quantize<MODE == MT_X_BF16 ? BL_BF16 : BL_F32, (CHM > 16 ? 16 : CHM), (CHM > 16 ? 2 : 1)>(p, sm, qs);
+    // (pre-quantised: each warp reads only the activations it copied itself;
+    // quantised here: the barrier at the end of mt_quantize)
 
     const uint32_t ring_lane = ring + uint32_t(warp) * 512 + uint32_t(lane) * 16;
     const uint32_t q_lane = smem_u32(qs) + uint32_t(warp) * 256 + uint32_t(lane >> 3) * 64;
@@ -362,11 +427,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) gemv_stream_mt_kernel(const MtP
         const GemvProblem &pr = p.prob[pi];
         const int64_t row = (Gr - p.gstart[pi]) * 8 + (rr & 7);
         if (row < pr.N) {
-            int rs = 0;
-#pragma unroll
-            for (int w = 0; w < kMtKC; ++w)
-                rs += sm.bsum[m][w];
-            const int a = sm.sacc[m][rr >> 3][rr & 7] - rs;
+            const int a = sm.sacc[m][rr >> 3][rr & 7] - sm.bsum[m][0];
             if (pr.acc_dbg)
                 pr.acc_dbg[int64_t(m) * pr.N + row] = a;
             store_y(pr.y, p.yt, int64_t(m) * pr.ldy + row, rescale1(a, sm.d[m], sm.wscale[pi]));
@@ -381,7 +442,7 @@ size_t mt_smem(int64_t K, int M, int R)
     return kMtHeader + size_t(kStages) * R * slot + size_t(M) * K;
 }
 
-template <int MT, int MODE>
+template <int MT, int MODE, int CHM>
 int launch_mt_t(const MtParams &base, cudaStream_t s, unsigned flags)
 {
     const DeviceInfo *di = device_info();
@@ -399,7 +460,7 @@ int launch_mt_t(const MtParams &base, cudaStream_t s, unsigned flags)
     if (!R)
         R = mt_smem(base.K, base.M, kMtMaxSet) <= size_t(di->max_smem_optin) ? kMtMaxSet : 2;
     const size_t smem = mt_smem(base.K, base.M, R);
-    auto kern = gemv_stream_mt_kernel<MT, MODE>;
+    auto kern = gemv_stream_mt_kernel<MT, MODE, CHM>;
     int per_sm = 0;
     int st = occupancy(reinterpret_cast<const void *>(kern), kMtThreads, smem, &per_sm);
     if (st)
@@ -426,23 +487,39 @@ int launch_mt_t(const MtParams &base, cudaStream_t s, unsigned flags)
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
 }
 
+// Chunks of 8 elements per lane that hold a whole row: 8, 16 or 32 (K up to
+// 2048, 4096 or 8192); longer rows are not taken by this kernel.
+template <int MT, int MODE>
+int launch_mt_k(const MtParams &p, cudaStream_t s, unsigned flags)
+{
+    if (p.K <= 2048)
+        return launch_mt_t<MT, MODE, 8>(p, s, flags);
+    if constexpr (MODE == MT_X_F32)
+        return launch_mt_t<MT, MODE, 16>(p, s, flags);
+    else
+        return p.K <= 4096 ? launch_mt_t<MT, MODE, 16>(p, s, flags) : launch_mt_t<MT, MODE, 32>(p, s, flags);
+}
+
 template <int MT>
 int launch_mt_mode(const MtParams &p, bool fused, int xt, cudaStream_t s, unsigned flags)
 {
     if (!fused)
-        return launch_mt_t<MT, MT_Q>(p, s, flags);
+        return launch_mt_t<MT, MT_Q, 0>(p, s, flags);
     if (xt == BL_BF16)
-        return launch_mt_t<MT, MT_X_BF16>(p, s, flags);
-    return launch_mt_t<MT, MT_X_F32>(p, s, flags);
+        return launch_mt_k<MT, MT_X_BF16>(p, s, flags);
+    return launch_mt_k<MT, MT_X_F32>(p, s, flags);
 }
 
 }  // namespace
 
-// 2 .. 16 tokens, K a multiple of 256, at most 32 row groups per CTA (one CTA
-// per SM) and the activations plus the ring within shared memory.
-bool gemv_stream_mt_applies(const GemvBatch &b, int sm_count, int max_smem)
+// 2 .. 16 tokens, K a multiple of 256 up to 8192 (4096 for fp32 input), at
+// most 32 row groups per CTA (one CTA per SM) and the activations plus the
+// ring within shared memory.
+bool gemv_stream_mt_applies(const GemvBatch &b, bool fused, int sm_count, int max_smem)
 {
-    if (b.M < 2 || b.M > kMtMaxTokens || b.K % 256 != 0 || b.count < 1 || sm_count <= 0)
+    if (b.M < 2 || b.M > kMtMaxTokens || b.K % 256 != 0 || b.K > kMtMaxK || b.count < 1 || sm_count <= 0)
+        return false;
+    if (fused && b.xt != BL_BF16 && b.K > kMtMaxK / 2)     // fp32 rows: 16 chunks per lane at most
         return false;
     int64_t ng = 0;
     for (int i = 0; i < b.count; ++i)

@@ -26,7 +26,7 @@ from dataclasses import dataclass, field
 import torch
 
 from . import (BL_ACT_PLAIN, BL_ACT_RELU2_GATE, BL_ACT_RMSNORM, attention_decode,
-               attention_workspace, decode_linear, pack, position_advance)
+               attention_workspace, decode_linear, pack, position_advance, rope_table)
 
 
 @dataclass
@@ -123,7 +123,8 @@ class Decoder:
                         "attn": torch.empty(c.heads * c.head_dim, dtype=bf, device=dev),
                         "gate": torch.empty(c.ffn, dtype=bf, device=dev),
                         "up": torch.empty(c.ffn, dtype=bf, device=dev),
-                        "attn_ws": attention_workspace(c.heads, c.kv_heads, c.max_seq, dev)}
+                        "attn_ws": attention_workspace(c.heads, c.kv_heads, c.max_seq, dev),
+                        "rope": rope_table(c.max_seq, c.rope_base, dev)}
 
     def set_position(self, pos: int):
         self.pos.fill_(int(pos))
@@ -135,7 +136,7 @@ class Decoder:
                       outs=[s["q"], s["k"], s["v"]], pdl=pdl)
         attention_decode(s["q"], s["k"], s["v"], L.cache_k, L.cache_v, self.pos, c.heads,
                          c.kv_heads, out=s["attn"], rope_base=c.rope_base,
-                         workspace=s["attn_ws"], pdl=pdl)
+                         workspace=s["attn_ws"], table=s["rope"], pdl=pdl)
         decode_linear([L.o], s["attn"], BL_ACT_PLAIN, outs=[h], resid=[h], pdl=pdl)
         decode_linear([L.gate, L.up], h, BL_ACT_RMSNORM, gain=L.g_ffn, eps=c.eps,
                       outs=[s["gate"], s["up"]], pdl=pdl)

@@ -164,9 +164,11 @@ int bitlinear_quantize_act(const void *x, int xt, int64_t M, int64_t K,
  *   q, d, rowsum      from bitlinear_quantize_act (device), q is [M][K]
  *   y                 device, [M][ldy] of dtype yt (BL_F32 or BL_BF16), ldy >= N
  *   acc_dbg           NULL, or device [M][N] int32 receiving acc (before rescale)
- * M * K must not exceed 163840 (the activations are staged on chip).  From
- * M = 8 on the product runs on the tensor-core path of bitlinear_gemm (dp4a
- * work grows with M); results are identical either way.
+ * M * K must not exceed 163840 (the activations are staged on chip).  Above
+ * 8 tokens on weights of more than 4M entries the product runs on the
+ * tensor-core path of bitlinear_gemm (dp4a work grows with M); otherwise 2 ..
+ * 16 tokens share one streaming pass over the weights.  Results are
+ * identical either way.
  */
 int bitlinear_gemv(const uint8_t *packed, const float *w_scale, int64_t N,
                    int64_t K, const int8_t *q, const float *d,
@@ -334,6 +336,9 @@ int bitlinear_decode_linear(int count, const uint8_t *const *packed,
  *   pos              device int32 scalar: this token's position, read by
  *                    the kernel (a CUDA graph can replay the call for the
  *                    next token after bitlinear_position_advance)
+ *   rope_table       NULL, or device (cos, sin) pairs from
+ *                    bitlinear_rope_table(D, T_max, rope_base) (same values,
+ *                    fewer fp64 evaluations per token)
  *   out              device bf16 [H*D]
  *   ws, ws_bytes     device workspace of at least
  *                    bitlinear_attention_workspace_bytes(H, Hkv, T_max) bytes,
@@ -352,8 +357,19 @@ int bitlinear_decode_linear(int count, const uint8_t *const *packed,
 int bitlinear_attention_decode(const void *q, const void *k, const void *v,
                                void *cache_k, void *cache_v, const int32_t *pos,
                                int H, int Hkv, int D, int T_max, double rope_base,
-                               void *out, void *ws, size_t ws_bytes,
-                               unsigned flags, void *stream);
+                               const float *rope_table, void *out, void *ws,
+                               size_t ws_bytes, unsigned flags, void *stream);
+
+/*
+ * RoPE's cosines and sines for every position and pair, so that
+ * bitlinear_attention_decode need not evaluate them per token: table[t][i] =
+ * (cos, sin) of t * rope_base^(-2i / D), each computed in fp64 and rounded to
+ * fp32 -- the values the attention kernels compute without a table.
+ *   table   device float [T_max][D/2][2], written; 8-byte aligned
+ * D must be 128; T_max <= 32768.
+ */
+int bitlinear_rope_table(int D, int T_max, double rope_base, float *table,
+                         void *stream);
 
 /* Bytes of workspace bitlinear_attention_decode needs (0 if out of range). */
 size_t bitlinear_attention_workspace_bytes(int H, int Hkv, int T_max);

@@ -251,11 +251,21 @@ def test_decoder_entry_argument_errors(bl):
     nb = L.bitlinear_attention_workspace_bytes(20, 5, 64)
     assert nb > 20 * 64 * 4 and L.bitlinear_attention_workspace_bytes(20, 6, 64) == 0
     assert L.bitlinear_attention_workspace_bytes(40, 2, 64) == 0      # 20 query heads per kv head
-    assert g(None, A, A, A, A, A, 20, 5, 128, 64, 1e4, A, A, nb, 0, None) == bl.BL_ERR_NULL
-    assert g(A, A, A, A, A, A, 20, 5, 64, 64, 1e4, A, A, nb, 0, None) == bl.BL_ERR_SHAPE
-    assert g(A, A, A, A, A, A, 20, 6, 128, 64, 1e4, A, A, nb, 0, None) == bl.BL_ERR_SHAPE
-    assert g(A, A, A, A, A, A, 20, 5, 128, 40000, 1e4, A, A, nb, 0, None) == bl.BL_ERR_SHAPE
-    assert g(A + 8, A, A, A, A, A, 20, 5, 128, 64, 1e4, A, A, nb, 0, None) == bl.BL_ERR_ALIGN
-    assert g(A, A, A, A, A, A, 20, 5, 128, 64, 1e4, A, A + 8, nb, 0, None) == bl.BL_ERR_ALIGN
+    assert g(None, A, A, A, A, A, 20, 5, 128, 64, 1e4, None, A, A, nb, 0, None) == bl.BL_ERR_NULL
+    assert g(A, A, A, A, A, A, 20, 5, 64, 64, 1e4, None, A, A, nb, 0, None) == bl.BL_ERR_SHAPE
+    assert g(A, A, A, A, A, A, 20, 6, 128, 64, 1e4, None, A, A, nb, 0, None) == bl.BL_ERR_SHAPE
+    assert g(A, A, A, A, A, A, 20, 5, 128, 40000, 1e4, None, A, A, nb, 0, None) == bl.BL_ERR_SHAPE
+    assert g(A + 8, A, A, A, A, A, 20, 5, 128, 64, 1e4, None, A, A, nb, 0, None) == bl.BL_ERR_ALIGN
+    assert g(A, A, A, A, A, A, 20, 5, 128, 64, 1e4, None, A, A + 8, nb, 0, None) == bl.BL_ERR_ALIGN
     assert L.bitlinear_position_advance(None, None) == bl.BL_ERR_NULL
     assert L.bitlinear_position_advance(A + 2, None) == bl.BL_ERR_ALIGN
+
+
+def test_rope_table_argument_errors(bl):
+    A = 0x7f0000000000
+    L = bl.lib
+    assert L.bitlinear_rope_table(128, 64, 1e4, None, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_rope_table(64, 64, 1e4, A, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_rope_table(128, 0, 1e4, A, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_rope_table(128, 64, 0.5, A, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_rope_table(128, 64, 1e4, A + 4, None) == bl.BL_ERR_ALIGN

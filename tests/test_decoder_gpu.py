@@ -192,3 +192,28 @@ def test_decoder_stack_tokens_match_oracle(bl, graph):
     for L, (ck, cv) in zip(dec.layers, caches):
         np.testing.assert_array_equal(_f32_of_bf16(L.cache_k), ck)
         np.testing.assert_array_equal(_f32_of_bf16(L.cache_v), cv)
+
+
+def test_rope_table_and_attention_with_it(bl):
+    """The table holds the oracle's cos/sin (fp64, rounded to fp32), and
+    attention with the table equals attention without it bit for bit."""
+    import math
+    T_max = 256
+    tab = bl.rope_table(T_max, device=dev()).cpu().numpy()
+    for t in (0, 1, 77, 255):
+        for i in (0, 1, 31, 63):
+            ang = t * 10000.0 ** (-(2.0 * i) / 128)
+            assert tab[t, i, 0] == np.float32(math.cos(ang))
+            assert tab[t, i, 1] == np.float32(math.sin(ang))
+    g = torch.Generator().manual_seed(9)
+    q = _bf16(torch.randn(H * D, generator=g)).to(dev())
+    k = _bf16(torch.randn(HKV * D, generator=g)).to(dev())
+    v = _bf16(torch.randn(HKV * D, generator=g)).to(dev())
+    ck = _bf16(torch.randn(HKV, T_max, D, generator=g)).to(dev())
+    cv = _bf16(torch.randn(HKV, T_max, D, generator=g)).to(dev())
+    posd = torch.tensor([200], dtype=torch.int32, device=dev())
+    a = bl.attention_decode(q, k, v, ck.clone(), cv.clone(), posd, H, HKV)
+    b = bl.attention_decode(q, k, v, ck.clone(), cv.clone(), posd, H, HKV,
+                            table=bl.rope_table(T_max, device=dev()))
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))

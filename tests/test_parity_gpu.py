@@ -224,8 +224,10 @@ def test_gemv_ragged_and_edge(bl, N, K, M, fused):
 
 @pytest.mark.parametrize("M", [8, 16])
 def test_small_batch_tensor_core_path(bl, M):
-    """From 8 tokens on, bitlinear_gemv and linear() run the tcgen05 path:
-    the four 2.4B shapes x 10 seeds, integers bit-exact, outputs equal."""
+    """bitlinear_gemv and linear() at 8 and 16 tokens (the tcgen05 path for
+    16 tokens on weights above 4M entries, the multi-token streaming kernel
+    otherwise): the four 2.4B shapes x 10 seeds, integers bit-exact, outputs
+    equal."""
     for K, N in si.DECODE_SHAPES_2B:
         for seed in range(10):
             W = si.weight(N, K, seed=2000 + seed)
