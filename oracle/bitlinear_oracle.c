@@ -394,10 +394,12 @@ void oracle_bitplane_acc(const uint64_t *mag, const uint64_t *sign,
  *              difference an fp32 operation in that order.
  *   attention  per query head h (kv head h / (H / Hkv)) over positions
  *              j = 0 .. T - 1: s_j = (float)(sum_d q[d] K[j][d]) * scale with
- *              the dot product in fp64; m = max s_j; e_j = (float)exp((double)
- *              (s_j - m)) with s_j - m in fp32; S = (float)(sum_j e_j) in fp64;
- *              out[d] = (float)(sum_j e_j V[j][d]) / S, the sum in fp64, the
- *              division in fp32.  scale = (float)(1 / sqrt(D)).
+ *              the dot product in fp64 and scale = (float)(1 / sqrt(D));
+ *              m = max s_j; the softmax weights e_j = exp(s_j - m), their sum
+ *              S and out[d] = (float)((sum_j e_j V[j][d]) / S) all in fp64
+ *              (the weights are not rounded to fp32: any fp64 grouping of the
+ *              sums, and any factoring of the exponentials, then agrees to
+ *              about 1e-15, far inside one fp32 rounding).
  *   FFN gate   m = (r * r) * u with r = max(g, 0) (squared ReLU gating), fp32.
  * ------------------------------------------------------------------------- */
 void oracle_rope(const float *x, int64_t heads, int64_t D, int64_t pos, double base,
@@ -421,7 +423,7 @@ void oracle_attention_decode(const float *q, const float *K, const float *V, int
 {
     float scale = (float)(1.0 / sqrt((double)D));
     float *sc = (float *)malloc((size_t)T * sizeof(float));
-    float *e = (float *)malloc((size_t)T * sizeof(float));
+    double *e = (double *)malloc((size_t)T * sizeof(double));
     for (int64_t h = 0; h < H; ++h) {
         int64_t kv = h / (H / Hkv);
         const float *qh = q + h * D;
@@ -438,16 +440,14 @@ void oracle_attention_decode(const float *q, const float *K, const float *V, int
         }
         double S = 0.0;
         for (int64_t j = 0; j < T; ++j) {
-            float t = sc[j] - m;
-            e[j] = (float)exp((double)t);
-            S += (double)e[j];
+            e[j] = exp((double)sc[j] - (double)m);
+            S += e[j];
         }
-        float Sf = (float)S;
         for (int64_t d = 0; d < D; ++d) {
             double num = 0.0;
             for (int64_t j = 0; j < T; ++j)
-                num += (double)e[j] * (double)Vh[j * D + d];
-            out[h * D + d] = (float)num / Sf;
+                num += e[j] * (double)Vh[j * D + d];
+            out[h * D + d] = (float)(num / S);
         }
     }
     free(sc);
