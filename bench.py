@@ -524,7 +524,7 @@ def rmsnorm_gemv_cost(bl, K, Ns, iters=200, device="cuda"):
 def decoder_tokens(bl, contexts=(512, 2048), tokens=64, device="cuda"):
     """The synthetic 2.4B decoder stack (30 layers: RMSNorm, q/k/v, RoPE +
     attention over a bf16 KV cache, o + residual, RMSNorm, gate/up, squared
-    ReLU gate, down + residual; 181 launches per token with PDL) replayed
+    ReLU gate, down + residual; 151 launches per token with PDL) replayed
     from a CUDA graph, one token per replay, at a given number of cached
     positions."""
     from bit_ternary_weight_b200.decoder import Decoder, DecoderConfig
@@ -552,7 +552,7 @@ def decoder_tokens(bl, contexts=(512, 2048), tokens=64, device="cuda"):
         t = s.elapsed_time(e) / 1000.0 / tokens
         out.append({"context": ctx, "tokens": tokens, "us_per_token": t * 1e6,
                     "tokens_per_s": 1.0 / t, "weight_GBps": dec.weight_bytes() / t / 1e9,
-                    "launches_per_token": 6 * cfg.layers + 1})
+                    "launches_per_token": 5 * cfg.layers + 1})
     assert bl.last_device_status() == 0
     del g, dec
     return out

@@ -13,43 +13,40 @@
 //              order; rotated q and k rounded to bf16 (k goes to the cache).
 //   scores     s_j = (float)(sum_d q[d] K[j][d]) * (float)(1 / sqrt(D)), the
 //              dot product of bf16 values in fp64 (every product exact).
-//   softmax    m = max_j s_j; e_j = (float)exp((double)(s_j - m)) with the
-//              difference in fp32; S = (float)(sum_j e_j) in fp64.
-//   output     out[d] = bf16((float)(sum_j e_j V[j][d]) / S), the sum in fp64
-//              (products exact), the division in fp32.
-// The fp64 sums run in another order than the oracle's; each is exact or
-// within an fp64 rounding of it, so the fp32 values agree unless one lies
-// within about 1e-15 (relative) of an fp32 rounding boundary.  exp, cos, sin
-// and pow are CUDA's fp64 functions on the GPU and the C library's on the CPU;
-// they may differ in the last fp64 bit, which moves an fp32 result only on
-// such a boundary too.
+//   softmax    m = max_j s_j; weights e_j = exp(s_j - m), their sum S and
+//              out[d] = bf16((float)((sum_j e_j V[j][d]) / S)) all in fp64.
+// The kernel evaluates the softmax per block of positions against the
+// block's own maximum m_b and combines the blocks with the factors
+// exp(m_b - m); with every softmax quantity in fp64 this grouping, the fp64
+// sums' order, and the difference between CUDA's fp64 exp, cos, sin and pow
+// and the C library's, change the fp32 results only when a value lies within
+// about 1e-15 (relative) of an fp32 rounding boundary.
 //
 // RoPE's cosines and sines come from a table of every (position, pair) that
 // bitlinear_rope_table computes once (same definition), or are computed in
-// the scores kernel when no table is given.
+// the kernel when no table is given.
 //
-// Design: two launches over blocks of 64 cached positions, so that the work
-// of one token spreads over (kv heads x position blocks) CTAs instead of one
-// CTA per head walking every position.  The position pos is a device scalar
-// read after the dependency wait, so a CUDA graph can replay the calls for
-// successive tokens; the grids cover the whole cache and the blocks beyond
-// pos return at once.
-//   scores   CTA (kv head, block): the rotated queries of the kv head's query
-//            heads (all of them share its keys); the block holding pos also
-//            rotates the new key and appends key and value at pos.  Eight
-//            lanes per position (16 dimensions each, fp64 partial dot
-//            products for every query head, three shuffle rounds), four
-//            positions per warp step.  Scores and the block's maxima go to
-//            the workspace.
-//   values   CTA (kv head, block): the global maximum of each query head from
-//            the blocks' maxima, the block's e_j in shared memory, the fp64
-//            partial sums of e_j and of e_j V[j] (lanes over dimensions, four
-//            position groups per CTA), written to the workspace; the CTA that
-//            arrives last on the kv head's ticket (fence, atomic add) adds the
-//            blocks' partial sums in block order, divides, rounds and stores,
-//            and resets the ticket.
+// Design: one launch of CTAs (kv head, block of 64 cached positions), so that
+// one token's attention spreads over many SMs; the position pos is a device
+// scalar read after the dependency wait, so a CUDA graph can replay the call
+// for successive tokens (the grid covers the whole cache; blocks beyond pos
+// return at once).  A CTA:
+//   * brings its block's cached keys and values (positions below pos) into
+//     shared memory with two bulk copies as soon as pos is known;
+//   * meanwhile rotates the queries of the kv head's query heads and, in the
+//     block holding pos, the new key, which it appends with the new value;
+//   * scores its positions (eight lanes per position, sixteen dimensions each,
+//     fp64 partial dot products for every query head), takes the block
+//     maximum, the fp64 weights, their sum and the fp64 weighted values
+//     (lanes over dimensions, four position groups), and writes them to the
+//     workspace;
+//   * arrives on the kv head's ticket (fence, atomic add); the last CTA to
+//     arrive combines the blocks in block order, divides, rounds and stores,
+//     and resets the ticket.
 // A position outside the cache records BL_ERR_SHAPE in the device status word
-// and writes nothing.
+// and writes nothing; a bulk copy that does not land in 2 s records
+// BL_ERR_TIMEOUT and that CTA leaves without output (the workspace's ticket
+// must then be zeroed again).
 #include "bl_common.cuh"
 
 namespace bl {
@@ -57,9 +54,9 @@ namespace {
 
 constexpr int kHeadDim = 128;
 constexpr int kPosBlock = 64;             // cached positions per CTA
-constexpr int kScoreThreads = 128;
-constexpr int kValueThreads = 128;
+constexpr int kAttnThreads = 128;
 constexpr int kMaxGroup = 8;              // query heads per kv head
+constexpr uint32_t kRowBytes = kHeadDim * 2;
 
 struct AttnParams {
     const __nv_bfloat16 *q, *k, *v;       // [H*D], [Hkv*D], [Hkv*D]
@@ -67,15 +64,30 @@ struct AttnParams {
     const int32_t *pos;
     int H, Hkv, T_max, nblk;
     double rope_base;
-    const float2 *rope;                   // NULL, or (cos, sin) [T_max][D/2] of every angle
+    const float2 *rope;                   // NULL, or (cos, sin) [T_max][D/2]
     __nv_bfloat16 *out;                   // [H*D]
     // workspace
-    float *sc;                            // [H][T_max] scores, then weights
-    float *bmax;                          // [H][nblk]
-    double *bsum;                         // [H][nblk]
-    double *bnum;                         // [H][nblk][D]
+    float *bmax;                          // [H][nblk] block maxima
+    double *bsum;                         // [H][nblk] block sums of exp(s - m_b)
+    double *bnum;                         // [H][nblk][D] block sums of exp(s - m_b) V
     unsigned *ticket;                     // [Hkv], zero between calls
     int *status;
+};
+
+struct AttnSmem {
+    uint64_t bar;
+    int abort_flag;
+    int last;
+    float2 cs[kHeadDim / 2];               // (cos, sin) of the token's angles
+    float qs[kMaxGroup][kHeadDim];         // rotated queries of the group
+    float ks[kHeadDim];                    // rotated new key (block holding pos)
+    float vs[kHeadDim];                    // new value
+    float sc[kMaxGroup][kPosBlock];        // scores
+    float mb[kMaxGroup];                   // block maxima
+    double ew[kMaxGroup][kPosBlock];       // weights exp(s - m_b)
+    double part[4][kMaxGroup][kHeadDim];   // per position group weighted values
+    alignas(128) __nv_bfloat16 kb[kPosBlock][kHeadDim];   // the block's cached keys
+    alignas(128) __nv_bfloat16 vb[kPosBlock][kHeadDim];   // ... and values
 };
 
 __device__ __forceinline__ float bf16_bits_f32(uint32_t b) { return __uint_as_float(b << 16); }
@@ -105,92 +117,94 @@ __device__ __forceinline__ void rope_pair(const __nv_bfloat16 *x, int i, float2 
     o1 = bf16_bits_f32(f32_bf16_bits(r1));
 }
 
-// The token's position, checked against the cache; -1 (and BL_ERR_SHAPE in
-// the status word, once per grid) when outside.
-__device__ __forceinline__ int read_pos(const AttnParams &p)
+__device__ __forceinline__ void bf16x8(const uint4 v, float *f)
 {
-    const int pos = int(ld_dep_u32(p.pos));
-    if (pos < 0 || pos >= p.T_max) {
-        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0)
-            atomicExch(p.status, BL_ERR_SHAPE);
-        return -1;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        f[2 * e] = __uint_as_float(w[e] << 16);
+        f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
     }
-    return pos;
 }
 
-__global__ void __launch_bounds__(kScoreThreads) attn_scores_kernel(const AttnParams p)
+__global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const AttnParams p)
 {
-    __shared__ float qs[kMaxGroup][kHeadDim];     // rotated queries of the group
-    __shared__ float ks[kHeadDim];                // rotated new key (block holding pos)
-    __shared__ float2 cs[kHeadDim / 2];           // (cos, sin) of the token's angles
-    __shared__ float wmax[kScoreThreads / 32][kMaxGroup];
+    extern __shared__ __align__(128) unsigned char attn_raw[];
+    AttnSmem &sm = *reinterpret_cast<AttnSmem *>(attn_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kv = blockIdx.x, blk = blockIdx.y;
     const int G = p.H / p.Hkv;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int pos = read_pos(p);
-    if (pos < 0)
+    const int pos = int(ld_dep_u32(p.pos));
+    if (pos < 0 || pos >= p.T_max) {
+        if (tid == 0 && kv == 0 && blk == 0)
+            atomicExch(p.status, BL_ERR_SHAPE);
         return;
+    }
     const int j0 = blk * kPosBlock;
     if (j0 > pos)
         return;
     const int j1 = min(j0 + kPosBlock, pos + 1);
-    const bool has_new = pos < j0 + kPosBlock;
+    const int n = j1 - j0;                            // positions of this block
+    const int nk = min(j1, pos) - j0;                 // of them in the cache already
+    const size_t head_base = size_t(kv) * p.T_max * kHeadDim;
+    if (tid == 0) {
+        sm.abort_flag = 0;
+        mbar_init(smem_u32(&sm.bar), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (nk > 0) {
+            const uint32_t bytes = uint32_t(nk) * kRowBytes;
+            mbar_arrive_tx(smem_u32(&sm.bar), 2 * bytes);
+            bulk_load(smem_u32(&sm.kb[0][0]), p.cache_k + head_base + size_t(j0) * kHeadDim, bytes, smem_u32(&sm.bar));
+            bulk_load(smem_u32(&sm.vb[0][0]), p.cache_v + head_base + size_t(j0) * kHeadDim, bytes, smem_u32(&sm.bar));
+        } else {
+            mbar_arrive(smem_u32(&sm.bar));
+        }
+    }
     if (tid < kHeadDim / 2)
-        cs[tid] = p.rope ? __ldg(p.rope + size_t(pos) * (kHeadDim / 2) + tid) : rope_angle(pos, tid, p.rope_base);
+        sm.cs[tid] = p.rope ? __ldg(p.rope + size_t(pos) * (kHeadDim / 2) + tid) : rope_angle(pos, tid, p.rope_base);
     __syncthreads();
-    for (int t = tid; t < G * (kHeadDim / 2); t += kScoreThreads) {
+    for (int t = tid; t < G * (kHeadDim / 2); t += kAttnThreads) {
         const int g = t / (kHeadDim / 2), i = t % (kHeadDim / 2);
         float a, b;
-        rope_pair(p.q + (kv * G + g) * kHeadDim, i, cs[i], a, b);
-        qs[g][2 * i] = a;
-        qs[g][2 * i + 1] = b;
+        rope_pair(p.q + (kv * G + g) * kHeadDim, i, sm.cs[i], a, b);
+        sm.qs[g][2 * i] = a;
+        sm.qs[g][2 * i + 1] = b;
     }
-    const size_t head_base = size_t(kv) * p.T_max * kHeadDim;
-    if (has_new && tid < kHeadDim / 2) {
+    if (nk < n && tid < kHeadDim / 2) {
+        // the block holding pos: rotate the new key, append key and value
         float a, b;
-        rope_pair(p.k + kv * kHeadDim, tid, cs[tid], a, b);
-        ks[2 * tid] = a;
-        ks[2 * tid + 1] = b;
+        rope_pair(p.k + kv * kHeadDim, tid, sm.cs[tid], a, b);
+        sm.ks[2 * tid] = a;
+        sm.ks[2 * tid + 1] = b;
+        const float v0 = bf16_bits_f32(ld_dep_u16(p.v + kv * kHeadDim + 2 * tid));
+        const float v1 = bf16_bits_f32(ld_dep_u16(p.v + kv * kHeadDim + 2 * tid + 1));
+        sm.vs[2 * tid] = v0;
+        sm.vs[2 * tid + 1] = v1;
         p.cache_k[head_base + size_t(pos) * kHeadDim + 2 * tid] = __float2bfloat16_rn(a);
         p.cache_k[head_base + size_t(pos) * kHeadDim + 2 * tid + 1] = __float2bfloat16_rn(b);
-        p.cache_v[head_base + size_t(pos) * kHeadDim + 2 * tid] =
-            __ushort_as_bfloat16(static_cast<unsigned short>(ld_dep_u16(p.v + kv * kHeadDim + 2 * tid)));
-        p.cache_v[head_base + size_t(pos) * kHeadDim + 2 * tid + 1] =
-            __ushort_as_bfloat16(static_cast<unsigned short>(ld_dep_u16(p.v + kv * kHeadDim + 2 * tid + 1)));
+        p.cache_v[head_base + size_t(pos) * kHeadDim + 2 * tid] = __float2bfloat16_rn(v0);
+        p.cache_v[head_base + size_t(pos) * kHeadDim + 2 * tid + 1] = __float2bfloat16_rn(v1);
     }
     __syncthreads();
-    // eight lanes per position (lane group r = lane / 8), sixteen dims each
+    if (!mbar_wait(smem_u32(&sm.bar), 0, &sm.abort_flag, p.status))
+        return;     // BL_ERR_TIMEOUT recorded; no output from this CTA
+
+    // ---- scores: eight lanes per position, sixteen dims each
     const float scale = __double2float_rn(1.0 / sqrt(double(kHeadDim)));
     const int sub = lane & 7, r = lane >> 3;
-    float lmax[kMaxGroup];
-#pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g)
-        lmax[g] = -INFINITY;
-    for (int jb = j0 + warp * 4; jb < j1; jb += 4 * (kScoreThreads / 32)) {
-        const int j = jb + r;
+    for (int jb = warp * 4; jb < n; jb += 4 * (kAttnThreads / 32)) {
+        const int jj = jb + r;
         float kf[16];
-        if (j < j1) {
-            if (j == pos) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    kf[e] = ks[sub * 16 + e];
-            } else {
-                const uint4 *kr = reinterpret_cast<const uint4 *>(p.cache_k + head_base + size_t(j) * kHeadDim +
-                                                                  sub * 16);
-                const uint4 a = __ldcg(kr), b = __ldcg(kr + 1);
-                const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    kf[2 * e] = __uint_as_float(w[e] << 16);
-                    kf[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-                }
-            }
+        if (jj < nk) {
+            const uint4 *kr = reinterpret_cast<const uint4 *>(&sm.kb[jj][sub * 16]);
+            bf16x8(kr[0], kf);
+            bf16x8(kr[1], kf + 8);
         } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-                kf[e] = 0.0f;
+                kf[e] = jj < n ? sm.ks[sub * 16 + e] : 0.0f;
         }
 #pragma unroll
         for (int g = 0; g < kMaxGroup; ++g) {
@@ -199,106 +213,68 @@ __global__ void __launch_bounds__(kScoreThreads) attn_scores_kernel(const AttnPa
             double dot = 0.0;
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-                dot = __fma_rn(double(qs[g][sub * 16 + e]), double(kf[e]), dot);   // exact products
+                dot = __fma_rn(double(sm.qs[g][sub * 16 + e]), double(kf[e]), dot);   // exact products
             dot = __dadd_rn(dot, __shfl_xor_sync(0xffffffffu, dot, 1));
             dot = __dadd_rn(dot, __shfl_xor_sync(0xffffffffu, dot, 2));
             dot = __dadd_rn(dot, __shfl_xor_sync(0xffffffffu, dot, 4));
-            if (j < j1) {
-                const float sv = __fmul_rn(__double2float_rn(dot), scale);
-                if (sub == 0)
-                    p.sc[size_t(kv * G + g) * p.T_max + j] = sv;
-                lmax[g] = fmaxf(lmax[g], sv);
-            }
+            if (jj < n && sub == 0)
+                sm.sc[g][jj] = __fmul_rn(__double2float_rn(dot), scale);
         }
     }
-#pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) {
-        if (g >= G)
-            break;
-        float m = lmax[g];
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-        if (lane == 0)
-            wmax[warp][g] = m;
-    }
     __syncthreads();
-    if (tid < G) {
-        float m = wmax[0][tid];
-#pragma unroll
-        for (int w = 1; w < kScoreThreads / 32; ++w)
-            m = fmaxf(m, wmax[w][tid]);
-        p.bmax[size_t(kv * G + tid) * p.nblk + blk] = m;
-    }
-}
-
-__global__ void __launch_bounds__(kValueThreads) attn_values_kernel(const AttnParams p)
-{
-    __shared__ float ew[kMaxGroup][kPosBlock];              // weights e_j of the block
-    __shared__ double part[4][kMaxGroup][kHeadDim / 4 * 4];  // per position group partial sums
-    __shared__ float gmax[kMaxGroup];
-    __shared__ int last;
-    const int tid = threadIdx.x;
-    const int kv = blockIdx.x, blk = blockIdx.y;
-    const int G = p.H / p.Hkv;
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int pos = read_pos(p);
-    if (pos < 0)
-        return;
-    const int nact = pos / kPosBlock + 1;       // blocks holding positions 0 .. pos
-    const int j0 = blk * kPosBlock;
-    if (blk >= nact)
-        return;
-    const int j1 = min(j0 + kPosBlock, pos + 1);
-    // the global maximum of each query head (exact: a max is order free)
-    if (tid < 32 * G) {
-        const int g = tid >> 5, lane = tid & 31;
+    // ---- block maxima, fp64 weights and their sums (warp g per head)
+    for (int g = warp; g < G; g += kAttnThreads / 32) {
         float m = -INFINITY;
-        for (int b = lane; b < nact; b += 32)
-            m = fmaxf(m, __ldcg(p.bmax + size_t(kv * G + g) * p.nblk + b));
+        for (int jj = lane; jj < n; jj += 32)
+            m = fmaxf(m, sm.sc[g][jj]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0)
-            gmax[g] = m;
-    }
-    __syncthreads();
-    // the block's weights e_j = (float)exp((double)(s_j - m))
-    for (int t = tid; t < G * kPosBlock; t += kValueThreads) {
-        const int g = t / kPosBlock, jj = t % kPosBlock, j = j0 + jj;
-        float e = 0.0f;
-        if (j < j1) {
-            const float sv = __ldcg(p.sc + size_t(kv * G + g) * p.T_max + j);
-            e = __double2float_rn(exp(double(__fsub_rn(sv, gmax[g]))));
+        double S = 0.0;
+        for (int jj = lane; jj < kPosBlock; jj += 32) {
+            const double e = jj < n ? exp(double(sm.sc[g][jj]) - double(m)) : 0.0;
+            sm.ew[g][jj] = e;
+            S = __dadd_rn(S, e);
         }
-        ew[g][jj] = e;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            S = __dadd_rn(S, __shfl_xor_sync(0xffffffffu, S, o));
+        if (lane == 0) {
+            sm.mb[g] = m;
+            p.bmax[size_t(kv * G + g) * p.nblk + blk] = m;
+            p.bsum[size_t(kv * G + g) * p.nblk + blk] = S;
+        }
     }
     __syncthreads();
-    // fp64 partial sums: thread (pg, c) takes dims 4c .. 4c + 3 of the
-    // positions jj = pg, pg + 4, ... of the block (pg = tid / 32, c = tid % 32)
+    // ---- weighted values: thread (pg, c) dims 4c .. 4c+3, positions pg, pg + 4, ...
     const int pg = tid >> 5, c = tid & 31;
-    const size_t head_base = size_t(kv) * p.T_max * kHeadDim;
     double acc[kMaxGroup][4];
 #pragma unroll
     for (int g = 0; g < kMaxGroup; ++g)
 #pragma unroll
         for (int x = 0; x < 4; ++x)
             acc[g][x] = 0.0;
-#pragma unroll 4
-    for (int jj = pg; jj < j1 - j0; jj += 4) {
-        const uint2 ab = __ldcg(reinterpret_cast<const uint2 *>(p.cache_v + head_base + size_t(j0 + jj) * kHeadDim +
-                                                                4 * c));
-        const uint32_t a = ab.x, b = ab.y;
-        const double vf[4] = {double(__uint_as_float(a << 16)), double(__uint_as_float(a & 0xffff0000u)),
-                              double(__uint_as_float(b << 16)), double(__uint_as_float(b & 0xffff0000u))};
+    for (int jj = pg; jj < n; jj += 4) {
+        float vf[4];
+        if (jj < nk) {
+            const uint2 ab = *reinterpret_cast<const uint2 *>(&sm.vb[jj][4 * c]);
+            vf[0] = __uint_as_float(ab.x << 16);
+            vf[1] = __uint_as_float(ab.x & 0xffff0000u);
+            vf[2] = __uint_as_float(ab.y << 16);
+            vf[3] = __uint_as_float(ab.y & 0xffff0000u);
+        } else {
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+                vf[x] = sm.vs[4 * c + x];
+        }
 #pragma unroll
         for (int g = 0; g < kMaxGroup; ++g) {
             if (g >= G)
                 break;
-            const double e = double(ew[g][jj]);
+            const double e = sm.ew[g][jj];
 #pragma unroll
             for (int x = 0; x < 4; ++x)
-                acc[g][x] = __fma_rn(e, vf[x], acc[g][x]);     // exact products (fp32 x bf16)
+                acc[g][x] = __fma_rn(e, double(vf[x]), acc[g][x]);
         }
     }
 #pragma unroll
@@ -307,53 +283,73 @@ __global__ void __launch_bounds__(kValueThreads) attn_values_kernel(const AttnPa
             break;
 #pragma unroll
         for (int x = 0; x < 4; ++x)
-            part[pg][g][4 * c + x] = acc[g][x];
+            sm.part[pg][g][4 * c + x] = acc[g][x];
     }
     __syncthreads();
-    for (int t = tid; t < G * kHeadDim; t += kValueThreads) {
+    for (int t = tid; t < G * kHeadDim; t += kAttnThreads) {
         const int g = t / kHeadDim, d = t % kHeadDim;
         double num = 0.0;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4)
-            num = __dadd_rn(num, part[q4][g][d]);
+            num = __dadd_rn(num, sm.part[q4][g][d]);
         p.bnum[(size_t(kv * G + g) * p.nblk + blk) * kHeadDim + d] = num;
     }
-    for (int g = tid >> 5; g < G; g += kValueThreads / 32) {
-        const int lane = tid & 31;
-        double S = __dadd_rn(double(ew[g][lane]), double(ew[g][lane + 32]));   // e_j = 0 beyond j1
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            S = __dadd_rn(S, __shfl_xor_sync(0xffffffffu, S, o));
-        if (lane == 0)
-            p.bsum[size_t(kv * G + g) * p.nblk + blk] = S;
-    }
-    // the last block of this kv head to finish combines the blocks
+    // ---- the last block of this kv head to finish combines the blocks
+    const int nact = pos / kPosBlock + 1;
     __threadfence();
     __syncthreads();
     if (tid == 0)
-        last = atomicAdd(&p.ticket[kv], 1u) == unsigned(nact - 1);
+        sm.last = atomicAdd(&p.ticket[kv], 1u) == unsigned(nact - 1);
     __syncthreads();
-    if (!last)
+    if (!sm.last)
         return;
     __threadfence();
-    for (int t = tid; t < G * kHeadDim; t += kValueThreads) {
+    // factors exp(m_b - m) per head and block (reusing ew), and the sums
+    double *fac = &sm.ew[0][0];               // [G][nact] when nact <= 64, else recomputed
+    const bool fit = nact <= kPosBlock;
+    __shared__ float gm[kMaxGroup];
+    __shared__ double gs[kMaxGroup];
+    for (int g = warp; g < G; g += kAttnThreads / 32) {
+        const size_t hb = size_t(kv * G + g) * p.nblk;
+        float m = -INFINITY;
+        for (int b = lane; b < nact; b += 32)
+            m = fmaxf(m, __ldcg(p.bmax + hb + b));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        double S = 0.0;
+        for (int b = lane; b < nact; b += 32) {
+            const double f = exp(double(__ldcg(p.bmax + hb + b)) - double(m));
+            if (fit)
+                fac[g * kPosBlock + b] = f;
+            S = __fma_rn(__ldcg(p.bsum + hb + b), f, S);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            S = __dadd_rn(S, __shfl_xor_sync(0xffffffffu, S, o));
+        if (lane == 0) {
+            gm[g] = m;
+            gs[g] = S;
+        }
+    }
+    __syncthreads();
+    for (int t = tid; t < G * kHeadDim; t += kAttnThreads) {
         const int g = t / kHeadDim, d = t % kHeadDim;
         const size_t hb = size_t(kv * G + g) * p.nblk;
-        double num = 0.0, S = 0.0;
+        double num = 0.0;
 #pragma unroll 8
         for (int b = 0; b < nact; ++b) {
-            num = __dadd_rn(num, __ldcg(p.bnum + (hb + b) * kHeadDim + d));
-            S = __dadd_rn(S, __ldcg(p.bsum + hb + b));
+            const double f = fit ? fac[g * kPosBlock + b] : exp(double(__ldcg(p.bmax + hb + b)) - double(gm[g]));
+            num = __fma_rn(__ldcg(p.bnum + (hb + b) * kHeadDim + d), f, num);
         }
-        const float o = __fdiv_rn(__double2float_rn(num), __double2float_rn(S));
-        p.out[(kv * G + g) * kHeadDim + d] = __float2bfloat16_rn(o);
+        p.out[(kv * G + g) * kHeadDim + d] = __float2bfloat16_rn(__double2float_rn(__ddiv_rn(num, gs[g])));
     }
     if (tid == 0)
         p.ticket[kv] = 0u;
 }
 
 // (cos, sin) of pos * base^(-2i / D) for every position and pair, fp64 then
-// fp32 (the same values the attention kernels compute without a table).
+// fp32 (the same values the attention kernel computes without a table).
 __global__ void rope_table_kernel(float2 *tab, int T_max, double base)
 {
     const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -371,7 +367,7 @@ __global__ void position_advance_kernel(int32_t *pos)
 
 // Workspace carve-up (16-byte aligned pieces).
 struct AttnWs {
-    size_t sc, bmax, bsum, bnum, ticket, total;
+    size_t bmax, bsum, bnum, ticket, total;
 };
 
 AttnWs ws_layout(int H, int Hkv, int T_max)
@@ -379,30 +375,12 @@ AttnWs ws_layout(int H, int Hkv, int T_max)
     const int nblk = (T_max + kPosBlock - 1) / kPosBlock;
     auto up = [](size_t v) { return (v + 15) / 16 * 16; };
     AttnWs w{};
-    w.sc = 0;
-    w.bmax = up(w.sc + size_t(H) * T_max * 4);
+    w.bmax = 0;
     w.bsum = up(w.bmax + size_t(H) * nblk * 4);
     w.bnum = up(w.bsum + size_t(H) * nblk * 8);
     w.ticket = up(w.bnum + size_t(H) * nblk * kHeadDim * 8);
     w.total = up(w.ticket + size_t(Hkv) * 4);
     return w;
-}
-
-template <class K>
-int launch_pdl(K kern, dim3 grid, int threads, cudaStream_t s, unsigned flags, const AttnParams &p)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(threads);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    if (flags & BL_FLAG_PDL) {
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
-    return cuda_status(cudaLaunchKernelEx(&cfg, kern, p));
 }
 
 }  // namespace
@@ -445,18 +423,31 @@ int launch_attention_decode(const void *q, const void *k, const void *v, void *c
     p.rope_base = rope_base;
     p.rope = reinterpret_cast<const float2 *>(rope);
     p.out = static_cast<__nv_bfloat16 *>(out);
-    p.sc = reinterpret_cast<float *>(base + w.sc);
     p.bmax = reinterpret_cast<float *>(base + w.bmax);
     p.bsum = reinterpret_cast<double *>(base + w.bsum);
     p.bnum = reinterpret_cast<double *>(base + w.bnum);
     p.ticket = reinterpret_cast<unsigned *>(base + w.ticket);
     p.status = di->status;
-    const dim3 grid(unsigned(Hkv), unsigned(p.nblk));
-    int st = launch_pdl(attn_scores_kernel, grid, kScoreThreads, s, flags, p);
+    const size_t smem = sizeof(AttnSmem);
+    int per_sm = 0;
+    int st = occupancy(reinterpret_cast<const void *>(attention_decode_kernel), kAttnThreads, smem, &per_sm);
     if (st)
         return st;
-    // the values launch always follows the scores launch programmatically
-    return launch_pdl(attn_values_kernel, grid, kValueThreads, s, BL_FLAG_PDL, p);
+    if (per_sm < 1)
+        return BL_ERR_SHAPE;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(Hkv), unsigned(p.nblk));
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    if (flags & BL_FLAG_PDL) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cuda_status(cudaLaunchKernelEx(&cfg, attention_decode_kernel, p));
 }
 
 int launch_position_advance(int32_t *pos, cudaStream_t s)

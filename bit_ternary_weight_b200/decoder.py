@@ -1,8 +1,7 @@
 """A synthetic BitNet b1.58 decoder-layer stack for decode, on the library's
-kernels: every layer is six launches (RMSNorm + q/k/v BitLinears; RoPE +
-KV-cache append + attention scores; softmax + values; o BitLinear +
-residual; RMSNorm + gate/up BitLinears; squared-ReLU gate + down BitLinear
-+ residual), chained with
+kernels: every layer is five launches (RMSNorm + q/k/v BitLinears; RoPE +
+KV-cache append + attention; o BitLinear + residual; RMSNorm + gate/up
+BitLinears; squared-ReLU gate + down BitLinear + residual), chained with
 programmatic dependent launch, one position advance per token, and the whole
 token capturable in a CUDA graph.
 
@@ -130,7 +129,7 @@ class Decoder:
         self.pos.fill_(int(pos))
 
     def layer_step(self, L: DecoderLayer, pdl: bool = True):
-        """One layer for the current token (six launches)."""
+        """One layer for the current token (five launches)."""
         c, s, h = self.cfg, self.scratch, self.h
         decode_linear([L.q, L.k, L.v], h, BL_ACT_RMSNORM, gain=L.g_attn, eps=c.eps,
                       outs=[s["q"], s["k"], s["v"]], pdl=pdl)
@@ -145,7 +144,7 @@ class Decoder:
 
     def step(self, pdl: bool = True):
         """One decode step: the token in self.h through every layer, then the
-        position advances.  6 * layers + 1 launches."""
+        position advances.  5 * layers + 1 launches."""
         for L in self.layers:
             self.layer_step(L, pdl)
         position_advance(self.pos)

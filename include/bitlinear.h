@@ -327,9 +327,9 @@ int bitlinear_decode_linear(int count, const uint8_t *const *packed,
  * pairs (2i, 2i + 1) turned by pos * rope_base^(-2i / D) (angle, cos, sin in
  * fp64, rounded to fp32; rotation in fp32; rotated q and k rounded to bf16);
  * s_j = (float)(q . K[j]) * (float)(1 / sqrt(D)) with the dot product in
- * fp64; softmax weights e_j = (float)exp(s_j - max s); out = bf16((float)(sum_j
- * e_j V[j]) / (float)(sum_j e_j)), sums in fp64.  Query head h reads kv head
- * h / (H / Hkv).
+ * fp64; softmax weights e_j = exp(s_j - max s), S = sum_j e_j and out =
+ * bf16((float)((sum_j e_j V[j]) / S)), all in fp64.  Query head h reads kv
+ * head h / (H / Hkv).
  *   q, k, v          device bf16 [H*D], [Hkv*D], [Hkv*D] (this token)
  *   cache_k, cache_v device bf16 [Hkv][T_max][D]; position *pos of every kv
  *                    head is written, positions 0 .. *pos read
@@ -342,17 +342,21 @@ int bitlinear_decode_linear(int count, const uint8_t *const *packed,
  *   out              device bf16 [H*D]
  *   ws, ws_bytes     device workspace of at least
  *                    bitlinear_attention_workspace_bytes(H, Hkv, T_max) bytes,
- *                    16-byte aligned: scores, per-block maxima and fp64
- *                    partial sums, and one arrival ticket per kv head.  It
+ *                    16-byte aligned: per-block maxima and fp64 partial
+ *                    sums, and one arrival ticket per kv head.  It
  *                    must be all zero before its first use; every call that
  *                    completes leaves the tickets zero.  Calls ordered on one
  *                    stream may share it; calls that can overlap may not.
  *   flags            0 or BL_FLAG_PDL (q, k, v may come from the kernel just
  *                    before; the cache and pos from earlier work)
- * Two launches on `stream` (scores, then values), over blocks of 64 cached
- * positions.  D must be 128; H a multiple of Hkv with H / Hkv <= 8; T_max
- * <= 32768.  A position outside [0, T_max) writes nothing and makes the next
- * bitlinear_last_device_status() return BL_ERR_SHAPE.
+ * One launch on `stream` over (kv head, block of 64 cached positions) CTAs;
+ * each block's softmax is taken against its own maximum and the blocks are
+ * combined with the factors exp(m_block - m), the whole softmax in fp64.
+ * D must be 128; H a multiple of Hkv with H / Hkv <= 8; T_max <= 32768.  A
+ * position outside [0, T_max) writes nothing and makes the next
+ * bitlinear_last_device_status() return BL_ERR_SHAPE; a block whose bulk
+ * copy does not land in 2 s makes it return BL_ERR_TIMEOUT, leaves `out`
+ * unwritten and the workspace's ticket non-zero (zero it again).
  */
 int bitlinear_attention_decode(const void *q, const void *k, const void *v,
                                void *cache_k, void *cache_v, const int32_t *pos,
