@@ -105,12 +105,12 @@ __device__ __forceinline__ float2 rope_angle(int pos, int i, double base)
     return make_float2(__double2float_rn(cos(ang)), __double2float_rn(sin(ang)));
 }
 
-// Rotate pair i of a head vector x (bf16) by (cos, sin) cs; the two rotated
-// values rounded to bf16 (as fp32).
-__device__ __forceinline__ void rope_pair(const __nv_bfloat16 *x, int i, float2 cs, float &o0, float &o1)
+// Rotate the pair (a, b) (one 32-bit word of two bf16 values, a in the low
+// half) by (cos, sin) cs; the two rotated values rounded to bf16 (as fp32).
+__device__ __forceinline__ void rope_pair(uint32_t ab, float2 cs, float &o0, float &o1)
 {
     const float c = cs.x, s = cs.y;
-    const float a = bf16_bits_f32(ld_dep_u16(x + 2 * i)), b = bf16_bits_f32(ld_dep_u16(x + 2 * i + 1));
+    const float a = __uint_as_float(ab << 16), b = __uint_as_float(ab & 0xffff0000u);
     const float r0 = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
     const float r1 = __fadd_rn(__fmul_rn(a, s), __fmul_rn(b, c));
     o0 = bf16_bits_f32(f32_bf16_bits(r0));
@@ -162,24 +162,45 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
             mbar_arrive(smem_u32(&sm.bar));
         }
     }
+    // this thread's query pairs (and the new key and value pair), loaded
+    // together before any is used (they come from the preceding launch: L2)
+    constexpr int kPairsPerThread = kMaxGroup * (kHeadDim / 2) / kAttnThreads;
+    uint32_t qw[kPairsPerThread];
+#pragma unroll
+    for (int u = 0; u < kPairsPerThread; ++u) {
+        const int t = tid + u * kAttnThreads;
+        qw[u] = t < G * (kHeadDim / 2)
+                    ? __ldcg(reinterpret_cast<const unsigned *>(p.q + (kv * G) * kHeadDim) + t)
+                    : 0u;
+    }
+    const bool has_new = nk < n;
+    uint32_t kw = 0, vw = 0;
+    if (has_new && tid < kHeadDim / 2) {
+        kw = __ldcg(reinterpret_cast<const unsigned *>(p.k + kv * kHeadDim) + tid);
+        vw = __ldcg(reinterpret_cast<const unsigned *>(p.v + kv * kHeadDim) + tid);
+    }
     if (tid < kHeadDim / 2)
         sm.cs[tid] = p.rope ? __ldg(p.rope + size_t(pos) * (kHeadDim / 2) + tid) : rope_angle(pos, tid, p.rope_base);
     __syncthreads();
-    for (int t = tid; t < G * (kHeadDim / 2); t += kAttnThreads) {
-        const int g = t / (kHeadDim / 2), i = t % (kHeadDim / 2);
-        float a, b;
-        rope_pair(p.q + (kv * G + g) * kHeadDim, i, sm.cs[i], a, b);
-        sm.qs[g][2 * i] = a;
-        sm.qs[g][2 * i + 1] = b;
+#pragma unroll
+    for (int u = 0; u < kPairsPerThread; ++u) {
+        const int t = tid + u * kAttnThreads;
+        if (t < G * (kHeadDim / 2)) {
+            const int g = t / (kHeadDim / 2), i = t % (kHeadDim / 2);
+            float a, b;
+            rope_pair(qw[u], sm.cs[i], a, b);
+            sm.qs[g][2 * i] = a;
+            sm.qs[g][2 * i + 1] = b;
+        }
     }
-    if (nk < n && tid < kHeadDim / 2) {
+    if (has_new && tid < kHeadDim / 2) {
         // the block holding pos: rotate the new key, append key and value
         float a, b;
-        rope_pair(p.k + kv * kHeadDim, tid, sm.cs[tid], a, b);
+        rope_pair(kw, sm.cs[tid], a, b);
         sm.ks[2 * tid] = a;
         sm.ks[2 * tid + 1] = b;
-        const float v0 = bf16_bits_f32(ld_dep_u16(p.v + kv * kHeadDim + 2 * tid));
-        const float v1 = bf16_bits_f32(ld_dep_u16(p.v + kv * kHeadDim + 2 * tid + 1));
+        const float v0 = __uint_as_float(vw << 16);
+        const float v1 = __uint_as_float(vw & 0xffff0000u);
         sm.vs[2 * tid] = v0;
         sm.vs[2 * tid + 1] = v1;
         p.cache_k[head_base + size_t(pos) * kHeadDim + 2 * tid] = __float2bfloat16_rn(a);
