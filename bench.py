@@ -797,8 +797,18 @@ def run_ours(args, world, rank, local):
         measure("rmsnorm_gemv", lambda: [rmsnorm_gemv_cost(bl, 2560, [6912, 6912], device=device),
                                          rmsnorm_gemv_cost(bl, 2560, [2560, 640, 640], device=device),
                                          rmsnorm_gemv_cost(bl, 8192, [28672], device=device)])
+        measure("mma_peak", lambda: bl.probe_mma_i8(device=device))
         measure("prefill", lambda: [prefill_gemm(bl, K, N, M, device=device)
                                     for (K, N) in si.PREFILL_SHAPES for M in si.PREFILL_TOKENS])
+        probe = extra.get("mma_peak", {}).get("tops")
+        for r in extra.get("prefill", []) if isinstance(extra.get("prefill"), list) else []:
+            r["roofline"] = {"bound": "tensor", "achieved": r["TOPS"], "unit": "TOPS",
+                             "peak_2x_bf16": 2 * bf16, "frac_2x_bf16": r["TOPS"] / (2 * bf16),
+                             "peak_probe": probe,
+                             "frac_probe": r["TOPS"] / probe if probe else None,
+                             "peak_kind": f"2 x {peak_kind} bf16 cuBLAS burst (nominal int8/bf16 "
+                                          "ratio); probe: back-to-back tcgen05.mma.kind::i8 of "
+                                          "the GEMM's form (bitlinear_probe_mma_i8)"}
 
     if rank != 0:
         return
@@ -861,6 +871,15 @@ def run_case(args):
         w = bl.binary_pack(W)
         fn = lambda: bl.binary_gemv(w, x[0])  # noqa: E731
         nbytes, ops = N * K // 8, 2 * N * K
+    elif args.case == "bitplane":
+        w = bl.bitplane_pack(bl.pack(W))
+        fn = lambda: bl.bitplane_gemv(w, x[0])  # noqa: E731
+        nbytes, ops = N * K // 4, 2 * N * K
+    elif args.case == "lut":
+        w = bl.pack(W)
+        q, d, _ = bl.quantize_act(x[:1])
+        fn = lambda: bl.lut_gemv(w, q, d)  # noqa: E731
+        nbytes, ops = bl.packed_bytes(N, K), 2 * N * K
     else:
         w = bl.pack(W)
         if args.case == "gemv":
@@ -886,9 +905,27 @@ def run_case(args):
                       "note": "same weights every launch (L2-warm unless profiled)"}), flush=True)
 
 
+def run_mma_peak(args):
+    """The int8 tensor-core rate of the prefill GEMM's MMA form, with the SM
+    clocks sampled while it runs; prints one JSON line."""
+    import bit_ternary_weight_b200 as bl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    bl.probe_mma_i8(reps=1000, device=dev)                 # warm-up
+    with ClockSampler(0) as clk:
+        runs = [bl.probe_mma_i8(reps=100000, device=dev) for _ in range(max(3, args.iters))]
+    best = max(runs, key=lambda r: r["tops"])
+    print(json.dumps({"case": "mma_peak", "mac_per_clk_per_sm": best["mac_per_clk_per_sm"],
+                      "tops": best["tops"], "ctas": best["ctas"], "runs": len(runs),
+                      "clocks": clk.summary(),
+                      "note": "back-to-back tcgen05.mma.kind::i8 128x128x32 (A in TMEM, B in "
+                              "swizzled smem), no operand traffic, one CTA per SM"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["stream", "gemv", "gemm", "binary"], default="stream",
+    ap.add_argument("--case", choices=["stream", "gemv", "gemm", "binary", "bitplane", "lut", "mma_peak"],
+                    default="stream",
                     help="stream: the benchmark; others: one kernel on one shape (profiling)")
     ap.add_argument("--K", type=int, default=8192)
     ap.add_argument("--N", type=int, default=28672)
@@ -913,6 +950,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.case == "mma_peak":
+        run_mma_peak(args)
+        return
     if args.case != "stream":
         run_case(args)
         return

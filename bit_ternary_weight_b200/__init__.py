@@ -125,6 +125,7 @@ _SIGNATURES.update({
     "bitlinear_rope_table": (_int, [_int, _int, ctypes.c_double, _vp, _vp]),
     "bitlinear_attention_workspace_bytes": (_sz, [_int, _int, _int]),
     "bitlinear_position_advance": (_int, [_vp, _vp]),
+    "bitlinear_probe_mma_i8": (_int, [_int, _vp, _int, _vp]),
     "bitlinear_chain_plan_bytes": (_sz, [_int]),
     "bitlinear_chain_plan": (_int, [_int, ctypes.POINTER(ChainStepC), _vp, _sz, _vp]),
     "bitlinear_chain_run": (_int, [_vp, _int, _vp]),
@@ -619,6 +620,28 @@ def bitplane_gemv(w: BitPlaneWeight, x: torch.Tensor, out_dtype=torch.bfloat16, 
                                             _ptr(acc_dbg), _stream(x.device)),
                "bitlinear_bitplane_gemv")
     return out
+
+
+def probe_mma_i8(reps: int = 4000, device="cuda") -> dict:
+    """Time back-to-back tcgen05 int8 MMAs of the prefill GEMM's form on every
+    SM (no operand traffic): MAC per clock per SM and TOPS over the grid."""
+    dev = torch.device(device)
+    grid = sm_count()
+    out = torch.zeros(2 * grid, dtype=torch.int64, device=dev)
+    with _on(dev):
+        _check(_lib.bitlinear_probe_mma_i8(reps, _ptr(out), grid, _stream(dev)),
+               "bitlinear_probe_mma_i8")
+        torch.cuda.synchronize(dev)
+    res = out.view(grid, 2).cpu()
+    if bool((res < 0).any()):
+        raise BitLinearError(BL_ERR_TIMEOUT, "bitlinear_probe_mma_i8")
+    macs = float(reps) * 8 * 128 * 128 * 32
+    cyc = res[:, 0].double()
+    ns = res[:, 1].double()
+    return {"reps": reps, "ctas": grid,
+            "mac_per_clk_per_sm": float((macs / cyc).median()),
+            "tops": float(2 * macs * grid / ns.max() / 1e3),
+            "ns_max": float(ns.max()), "cycles_median": float(cyc.median())}
 
 
 def last_device_status(stream=None) -> int:

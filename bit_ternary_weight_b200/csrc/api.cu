@@ -828,6 +828,25 @@ int bitlinear_bitplane_gemv(const uint64_t *planes, const float *w_scale, int64_
                                 static_cast<cudaStream_t>(stream));
 }
 
+int bitlinear_probe_mma_i8(int reps, long long *out, int grid, void *stream)
+{
+    if (!out)
+        return BL_ERR_NULL;
+    if (reps < 1 || reps > (1 << 17) || grid < 1)   // (1 << 17) stages: ~35 ms, far inside the 2 s wait
+        return BL_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(out) & 7u)
+        return BL_ERR_ALIGN;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    if (grid > di->sm_count)
+        return BL_ERR_SHAPE;
+    if ((st = check_dev_ptrs({out})))
+        return st;
+    return launch_mma_probe(reps, out, grid, static_cast<cudaStream_t>(stream));
+}
+
 int bitlinear_last_device_status(void *stream)
 {
     const DeviceInfo *di = device_info();

@@ -165,6 +165,9 @@ int launch_lut_gemv(const uint8_t *packed, const float *w_scale, int64_t N, int6
                     const int8_t *q, const float *d, void *y, int yt, int32_t *acc_dbg,
                     cudaStream_t s);
 
+// int8 tensor-core rate probe (mma_probe.cu): per CTA (clock cycles, ns).
+int launch_mma_probe(int reps, long long *out, int grid, cudaStream_t s);
+
 // Persistent decode chain (gemv_chain.cu).
 size_t chain_plan_bytes(int nsteps);
 bool chain_step_fits(int64_t K);

@@ -572,6 +572,19 @@ int bitlinear_bitplane_gemv(const uint64_t *planes, const float *w_scale,
                             void *y, int yt, int32_t *acc_dbg, void *stream);
 
 /*
+ * Measurement aid: the int8 tensor-core rate the prefill GEMM can draw on.
+ * `grid` CTAs (at most one per SM) each issue `reps` stages of eight
+ * back-to-back tcgen05.mma.kind::i8 of the GEMM's form (128 x 128 x 32: A =
+ * unsigned codes in tensor memory, B = signed activations in 128-byte-swizzled
+ * shared memory, int32 accumulators), with no operand traffic, and time them.
+ *   out   device int64 [2 * grid]: per CTA, clock cycles and nanoseconds
+ *         (-1 if the final wait ran out; BL_ERR_TIMEOUT in the status word)
+ * MACs per CTA = reps * 8 * 128 * 128 * 32; reps <= 131072.  Asynchronous on
+ * `stream`.
+ */
+int bitlinear_probe_mma_i8(int reps, long long *out, int grid, void *stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device: BL_OK, BL_ERR_TIMEOUT if a kernel's bounded wait ran out,
  * or BL_ERR_SHAPE if a kernel found a device-side argument out of range (a

@@ -577,3 +577,12 @@ def test_small_batch_pdl_chain_in_graph(bl):
         y_o, _ = _oracle_gemv(gam, codes, x)
         compare_outputs(xs[i + 1], y_o)
         x = torch.from_numpy(oracle.to_bf16_bits(y_o).view(np.int16)).view(torch.bfloat16).reshape(M, K)
+
+
+def test_mma_probe_rate_is_plausible(bl):
+    """The int8 tensor-core probe runs on every SM and reports a rate within
+    the physically possible range (1 to 20 thousand MAC per clock per SM)."""
+    r = bl.probe_mma_i8(reps=2000, device=dev())
+    assert r["ctas"] == bl.sm_count()
+    assert 1000 < r["mac_per_clk_per_sm"] < 20000
+    assert bl.last_device_status() == 0
