@@ -76,6 +76,7 @@ def _load():
             "oracle_relu2_gate": (None, [vp, vp, i64, vp]),
             "oracle_residual_add": (None, [vp, vp, i64, vp]),
             "oracle_num_threads": (ctypes.c_int, []),
+            "oracle_set_num_threads": (None, [ctypes.c_int]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -116,6 +117,11 @@ def ternary_codes(W: np.ndarray, gamma_eff) -> np.ndarray:
 def num_threads() -> int:
     """Threads the oracle's parallel loops use."""
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Thread count for the oracle's parallel loops (timing only; results do not depend on it)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def packed_bytes(N: int, K: int) -> int:

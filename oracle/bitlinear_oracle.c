@@ -482,3 +482,14 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Sets the thread count of those loops (no effect without OpenMP). */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
