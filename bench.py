@@ -325,32 +325,27 @@ def time_graph(graph, steps, world):
 
 
 def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda", pdl=False,
-                  force_fused=None):
+                  force_fused=None, small_batch="auto", ws=None):
     """Per-launch time of one shape, rotating distinct weight copies (>= 4x L2).
 
     pdl: consecutive launches (M = 1) overlap through programmatic dependent
     launch, as consecutive GEMVs of a decode step do; each still reads x only
-    after the previous launch has finished."""
+    after the previous launch has finished.  small_batch: for 2 .. 16 tokens,
+    "auto", "tensor" or "dp4a" (the kernel the fused call runs).  ws: the
+    rotated weight copies, built here when not given."""
     nbytes = bl.packed_bytes(N, K)
-    if copies is None:
-        copies = max(2, int((4 * 126e6) // nbytes) + 1)
-    copies = min(copies, 400)
-    gen = torch.Generator(device=device)
-    ws = []
-    for c in range(copies):
-        gen.manual_seed(7 + c)
-        W = torch.randn(N, K, generator=gen, device=device) * 0.02
-        ws.append(bl.pack(W))
-        del W
+    if ws is None:
+        if copies is None:
+            copies = max(2, int((4 * 126e6) // nbytes) + 1)
+        ws = _weight_copies(bl, K, N, nbytes, 7, device, limit=min(copies, 400))
+    copies = len(ws)
     x = si.activations(M, K, seed=5).to(device)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
-    # the path bl.linear takes: fused dp4a GEMV for few tokens, else quantise +
+    # the path bl.linear takes: a fused GEMV for few tokens, else quantise +
     # tensor-core GEMM (both launches timed)
-    fused = M <= bl.GEMV_FUSED_MAX_M if force_fused is None else force_fused
-    if fused and pdl:
-        call = lambda wt: bl.gemv_fused_multi([wt], x, outs=[y], pdl=True)  # noqa: E731
-    elif fused:
-        call = lambda wt: bl.gemv_fused(wt, x, out=y)  # noqa: E731
+    fused = bl.fused_gemv_preferred(M, N, K) if force_fused is None else force_fused
+    if fused:
+        call = lambda wt: bl.gemv_fused_multi([wt], x, outs=[y], pdl=pdl, small_batch=small_batch)  # noqa: E731
     else:
         q = torch.empty(M, K, dtype=torch.int8, device=device)
         d = torch.empty(M, dtype=torch.float32, device=device)
@@ -376,40 +371,44 @@ def isolated_gemv(bl, K, N, M=1, iters=200, copies=None, device="cuda", pdl=Fals
     e.record()
     torch.cuda.synchronize()
     t = s.elapsed_time(e) / 1000.0 / iters
-    del g, ws
+    del g
     return {"K": K, "N": N, "M": M, "us": t * 1e6, "GBps": nbytes / t / 1e9,
             "weight_copies": copies, "pdl": pdl,
-            "path": gemv_path(K, N, M, fused)}
+            "path": gemv_path(bl, K, N, M, fused, small_batch)}
 
 
-def gemv_path(K, N, M, fused):
-    """Which kernel the library runs for this shape (mirrors its dispatch)."""
+def gemv_path(bl, K, N, M, fused, small_batch="auto"):
+    """Which kernel the library runs for this shape (the library's own plan)."""
     if not fused:
-        return "quantise + tcgen05 GEMM (32-token tiles, split K)"
-    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    ng = (N + 7) // 8
-    if M == 1 and K % 256 == 0 and K <= 32768 and ng <= 64 * sms:
-        return "fused streaming GEMV (producer warp, bulk copies, mbarrier ring)"
-    if 2 <= M <= 16 and K % 256 == 0 and ng <= 32 * sms:
-        return "fused multi-token streaming GEMV (one weight pass for all tokens)"
-    return "fused dp4a GEMV (per-warp cp.async ring)"
+        return "quantise + tcgen05 GEMM"
+    kern, cluster = bl.gemv_plan([N], K, M, small_batch=small_batch)
+    return {"stream": "fused streaming GEMV (producer warp, bulk copies, mbarrier ring)",
+            "tensor": f"tensor-core small-batch GEMV (clusters of {cluster} CTAs per 128-row block)",
+            "stream_mt": "fused multi-token streaming GEMV (dp4a, one weight pass for all tokens)",
+            "dp4a": "fused dp4a GEMV (per-warp cp.async ring)"}[kern]
 
 
 def small_batch_sweep(bl, device="cuda"):
     """Config 3's timing: M in {1, 2, 4, 8, 16} on the four 2.4B shapes.
-    `us` / `GBps` are the path linear() takes (bl.fused_gemv_preferred); from
-    8 tokens both paths are timed (`fused_us`, `tensor_core_us`)."""
+    `us` / `GBps` / `path` are what linear() runs (the library's routing); from
+    2 tokens the two small-batch kernels are timed side by side (`tensor_us`,
+    `dp4a_us`) and from 8 tokens also quantise + GEMM (`gemm_us`)."""
     out = []
     for (K, N) in si.DECODE_SHAPES_2B:
+        nbytes = bl.packed_bytes(N, K)
+        ws = _weight_copies(bl, K, N, nbytes, 7, device)
         for m in si.SMALL_BATCH_M:
-            f = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=True)
-            r = dict(f)
+            r = dict(isolated_gemv(bl, K, N, M=m, iters=100, device=device, ws=ws))
+            if m >= 2:
+                r["tensor_us"] = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=True,
+                                               small_batch="tensor", ws=ws)["us"]
+                r["dp4a_us"] = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=True,
+                                             small_batch="dp4a", ws=ws)["us"]
             if m >= 8:
-                g = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=False)
-                r["fused_us"], r["tensor_core_us"] = f["us"], g["us"]
-                if not bl.fused_gemv_preferred(m, N, K):
-                    r.update(us=g["us"], GBps=g["GBps"], path=g["path"])
+                r["gemm_us"] = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=False,
+                                             ws=ws)["us"]
             out.append(r)
+        del ws
     return out
 
 

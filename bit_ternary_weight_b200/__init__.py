@@ -79,6 +79,7 @@ _SIGNATURES = {
                                     _i64, _vp, _vp]),
     "bitlinear_gemv_fused_multi": (_int, [_int, _vp, _vp, _vp, _i64, _vp, _int, _i64, _i64,
                                           _vp, _int, _vp, _vp, ctypes.c_uint, _vp]),
+    "bitlinear_gemv_plan": (_int, [_int, _vp, _i64, _i64, _int, _int, ctypes.c_uint, _vp, _vp]),
     "bitlinear_rmsnorm_quantize_act": (_int, [_vp, _int, _i64, _i64, _i64, _vp, _int,
                                               ctypes.c_float, _vp, _vp, _vp, _vp]),
     "bitlinear_rmsnorm_gemv_fused_multi": (_int, [_int, _vp, _vp, _vp, _i64, _vp, _int, _vp,
@@ -278,15 +279,23 @@ def gemv_fused(w: TernaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16, out=
 
 GEMV_MAX_PROBLEMS = 8
 BL_FLAG_PDL = 1
+BL_FLAG_SMALL_BATCH_DP4A = 2
+BL_FLAG_SMALL_BATCH_TENSOR = 4
+
+
+_SMALL_BATCH = {"auto": 0, "dp4a": BL_FLAG_SMALL_BATCH_DP4A, "tensor": BL_FLAG_SMALL_BATCH_TENSOR}
 
 
 def gemv_fused_multi(weights, x: torch.Tensor, out_dtype=torch.bfloat16, outs=None,
-                     acc_dbgs=None, pdl: bool = False):
+                     acc_dbgs=None, pdl: bool = False, small_batch: str = "auto"):
     """Several decode BitLinears sharing the activations x, in one launch.
 
     weights: list of TernaryWeight with the same K (q/k/v or gate/up of a layer).
     pdl: allow the launch to overlap the preceding kernel's tail (programmatic
     dependent launch); only when the weights were not written by that kernel.
+    small_batch: for 2 .. 16 tokens, "auto" (the measured crossover), "dp4a"
+    (the multi-token streaming kernel) or "tensor" (the tensor-core kernel),
+    each where it applies; the results are identical.
     """
     if x.dim() == 1:
         x = x.unsqueeze(0)
@@ -305,9 +314,27 @@ def gemv_fused_multi(weights, x: torch.Tensor, out_dtype=torch.bfloat16, outs=No
     with _on(x.device):
         _check(_lib.bitlinear_gemv_fused_multi(n, packed, scales, Ns, weights[0].K, _ptr(x),
                                                _dt(x.dtype), x.stride(0), M, ys, _dt(outs[0].dtype),
-                                               ldys, accs, BL_FLAG_PDL if pdl else 0,
+                                               ldys, accs,
+                                               (BL_FLAG_PDL if pdl else 0) | _SMALL_BATCH[small_batch],
                                                _stream(x.device)), "bitlinear_gemv_fused_multi")
     return outs
+
+
+GEMV_KERNELS = {1: "stream", 2: "tensor", 3: "stream_mt", 4: "dp4a"}
+
+
+def gemv_plan(Ns, K: int, M: int, xdtype=torch.bfloat16, fused: bool = True,
+              small_batch: str = "auto"):
+    """Which GEMV kernel gemv_fused_multi (fused) or gemv (pre-quantised) runs
+    for these shapes on the current device: ("stream" | "tensor" | "stream_mt"
+    | "dp4a", cluster size of the tensor-core kernel or 0)."""
+    n = len(Ns)
+    Narr = (ctypes.c_int64 * n)(*Ns)
+    kern, cl = ctypes.c_int(0), ctypes.c_int(0)
+    _check(_lib.bitlinear_gemv_plan(n, Narr, K, M, _dt(xdtype), 1 if fused else 0,
+                                    _SMALL_BATCH[small_batch],
+                                    ctypes.byref(kern), ctypes.byref(cl)), "bitlinear_gemv_plan")
+    return GEMV_KERNELS[kern.value], cl.value
 
 
 RMS_EPS = 1e-5  # default RMSNorm epsilon (the library's reading; the pages give none)
@@ -527,16 +554,19 @@ def gemm(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc
     return out
 
 
-GEMV_FUSED_MAX_M = 8          # up to here the fused streaming GEMV is the faster path
-GEMV_FUSED_SMALL_W_MAX_M = 16  # ... and up to here for weights of at most
-GEMV_SMALL_W = 4 * 1024 * 1024  # this many entries (measured on B200)
+GEMV_FUSED_MAX_M = 8          # up to here the fused GEMV kernels are always the faster path
 
 
 def fused_gemv_preferred(M: int, N: int, K: int) -> bool:
-    """Whether the fused dp4a GEMV beats quantise + tensor-core GEMM for M tokens."""
-    if M * K > 163840:
+    """Whether the fused GEMV beats quantise + tensor-core GEMM for M tokens:
+    up to 8 tokens always; 9 .. 16 tokens where the small-batch tensor-core
+    or multi-token streaming kernel takes the shape (measured on B200: both
+    under the GEMM's ~11-13 us there), not the per-warp dp4a kernel."""
+    if M * K > 163840 or M > 16:
         return False
-    return M <= GEMV_FUSED_MAX_M or (M <= GEMV_FUSED_SMALL_W_MAX_M and N * K <= GEMV_SMALL_W)
+    if M <= GEMV_FUSED_MAX_M:
+        return True
+    return gemv_plan([N], K, M)[0] in ("tensor", "stream_mt")
 
 
 def linear(w: TernaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16):

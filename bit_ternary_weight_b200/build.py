@@ -26,7 +26,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 SOURCES = ["api.cu", "quant.cu", "pack.cu", "gemv.cu", "gemv_stream.cu", "gemm.cu", "binary.cu",
            "popc_stream.cu", "lut_gemv.cu", "gemv_chain.cu", "attention.cu",
-           "gemv_stream_mt.cu", "mma_probe.cu"]
+           "gemv_stream_mt.cu", "mma_probe.cu", "gemv_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
                      "-Xcompiler", "-Wall", "--expt-relaxed-constexpr",

@@ -293,8 +293,7 @@ int check_gemv_common(const uint8_t *packed, const float *w_scale, int64_t N,
 }
 
 constexpr int64_t kGemvMaxM = 16;
-constexpr int64_t kGemvTensorM = 8;     // above this, bitlinear_gemv may take the tcgen05 path
-constexpr int64_t kGemvSmallW = int64_t(4) << 20;   // weights up to this stay on dp4a to 16 tokens
+constexpr int64_t kGemvTensorM = 8;     // above this, bitlinear_gemv may take the tcgen05 GEMM
 constexpr int64_t kGemvMaxMK = 163840;
 
 }  // namespace
@@ -319,11 +318,21 @@ int bitlinear_gemv(const uint8_t *packed, const float *w_scale, int64_t N, int64
     if ((st = check_dev_ptrs({packed, w_scale, q, d, rowsum, y, acc_dbg})))
         return st;
     GemvArgs a{packed, w_scale, N, K, M, q, d, rowsum, nullptr, BL_F32, 0, y, yt, ldy, acc_dbg};
-    // beyond kGemvTensorM tokens (on weights of more than kGemvSmallW entries)
-    // the dp4a work outgrows the weight stream while the tensor cores are idle:
-    // the product runs on the tcgen05 path (same results)
-    if (M > kGemvTensorM && N * K > kGemvSmallW)
-        return launch_gemm(a, nullptr, 0, static_cast<cudaStream_t>(stream));
+    // beyond kGemvTensorM tokens, where neither small-batch kernel takes the
+    // shape (tensor-core or multi-token streaming), the per-warp dp4a work
+    // outgrows the weight stream: the product runs on the tcgen05 GEMM
+    // (same results)
+    if (M > kGemvTensorM) {
+        GemvBatch b{};
+        b.count = 1;
+        b.prob[0].N = N;
+        b.K = K;
+        b.M = M;
+        b.xt = BL_F32;
+        int cluster = 0;
+        if (plan_gemv_batch(b, false, &cluster) == BL_GEMV_KERNEL_DP4A)
+            return launch_gemm(a, nullptr, 0, static_cast<cudaStream_t>(stream));
+    }
     return launch_gemv(a, false, static_cast<cudaStream_t>(stream));
 }
 
@@ -362,7 +371,8 @@ int bitlinear_gemv_fused_multi(int count, const uint8_t *const *packed,
         return BL_ERR_NULL;
     if (count < 1 || count > kGemvMaxProblems)
         return BL_ERR_SHAPE;
-    if (flags & ~BL_FLAG_PDL)
+    if ((flags & ~(BL_FLAG_PDL | BL_FLAG_SMALL_BATCH_DP4A | BL_FLAG_SMALL_BATCH_TENSOR)) ||
+        (flags & BL_FLAG_SMALL_BATCH_DP4A && flags & BL_FLAG_SMALL_BATCH_TENSOR))
         return BL_ERR_SHAPE;
     if (!valid_dtype(xt) || !valid_dtype(yt))
         return BL_ERR_DTYPE;
@@ -399,6 +409,39 @@ int bitlinear_gemv_fused_multi(int count, const uint8_t *const *packed,
     b.yt = yt;
     b.flags = flags;
     return launch_gemv_batch(b, true, static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_gemv_plan(int count, const int64_t *N, int64_t K, int64_t M, int xt,
+                        int fused, unsigned flags, int *kernel, int *cluster)
+{
+    if (!N || !kernel || !cluster)
+        return BL_ERR_NULL;
+    if (count < 1 || count > kGemvMaxProblems || K < 1 || M < 1 || M > kGemvMaxM ||
+        (flags & ~(BL_FLAG_PDL | BL_FLAG_SMALL_BATCH_DP4A | BL_FLAG_SMALL_BATCH_TENSOR)) ||
+        (flags & BL_FLAG_SMALL_BATCH_DP4A && flags & BL_FLAG_SMALL_BATCH_TENSOR))
+        return BL_ERR_SHAPE;
+    if (!valid_dtype(xt))
+        return BL_ERR_DTYPE;
+    GemvBatch b{};
+    b.count = count;
+    for (int i = 0; i < count; ++i) {
+        if (N[i] < 1)
+            return BL_ERR_SHAPE;
+        b.prob[i].N = N[i];
+    }
+    b.K = K;
+    b.M = M;
+    b.xt = xt;
+    b.flags = flags;
+    const DeviceInfo *di;
+    int st = need_device(&di);
+    if (st)
+        return st;
+    const int k = plan_gemv_batch(b, fused != 0, cluster);
+    if (k < 0)
+        return BL_ERR_CUDA;
+    *kernel = k;
+    return BL_OK;
 }
 
 int bitlinear_rmsnorm_gemv_fused_multi(int count, const uint8_t *const *packed,

@@ -115,6 +115,17 @@ struct GemvBatch {
 
 int launch_gemv_batch(const GemvBatch &b, bool fused, cudaStream_t s);
 
+// Which kernel launch_gemv_batch runs for the batch (BL_GEMV_KERNEL_*), and
+// for the tensor-core kernel its cluster size (else 0).
+int plan_gemv_batch(const GemvBatch &b, bool fused, int *cluster);
+
+// The tensor-core small-batch kernel (gemv_tc.cu): 2 .. 16 tokens, K a
+// multiple of 256, bf16 x when fused; whether it takes the batch (a cluster
+// split of the row blocks that is resident at once), and its launch.
+bool gemv_tc_applies(const GemvBatch &b, bool fused);
+int gemv_tc_cluster(const GemvBatch &b, bool fused);   // CTAs per cluster, 0: not taken
+int launch_gemv_tc(const GemvBatch &b, bool fused, cudaStream_t s);
+
 // The streaming one-token kernel (gemv_stream.cu): whether it takes the batch,
 // and its launch with the token normalised (RMSNorm with gain / eps) before
 // quantisation when `norm` is set.

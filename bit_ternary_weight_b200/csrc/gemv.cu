@@ -631,15 +631,59 @@ int dispatch_m(const Params &p, unsigned flags, cudaStream_t s)
 int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s);
 bool gemv_stream_applies(const GemvBatch &b, int sm_count);
 
+// 2 .. 16 tokens: the tensor-core kernel or the dp4a multi-token kernel.
+// The dp4a kernel's cost grows with the tokens x weights it multiplies and
+// with K (each warp quantises whole token rows); the tensor-core kernel's is
+// nearly flat in M but carries ~2 us more fixed latency (cluster exchange,
+// MMA commit, tensor memory).  Measured crossover on the 2.4B shapes: the
+// tensor cores from M N K >= 48 Mi, or for K above 4096.
+bool small_batch_prefers_tensor(const GemvBatch &b)
+{
+    int64_t nk = 0;
+    for (int i = 0; i < b.count; ++i)
+        nk += b.prob[i].N * b.K;
+    return b.M * nk >= (int64_t(48) << 20) || b.K > 4096;
+}
+
+bool small_batch_tensor(const GemvBatch &b, bool fused, int *cluster)
+{
+    *cluster = 0;
+    if (b.flags & BL_FLAG_SMALL_BATCH_DP4A)
+        return false;
+    if (!(b.flags & BL_FLAG_SMALL_BATCH_TENSOR) && !small_batch_prefers_tensor(b))
+        return false;
+    *cluster = gemv_tc_cluster(b, fused);
+    return *cluster > 0;
+}
+
+int plan_gemv_batch(const GemvBatch &b, bool fused, int *cluster)
+{
+    *cluster = 0;
+    const DeviceInfo *di = device_info();
+    if (!di)
+        return -1;
+    if (gemv_stream_applies(b, di->sm_count))
+        return BL_GEMV_KERNEL_STREAM;
+    if (small_batch_tensor(b, fused, cluster))
+        return BL_GEMV_KERNEL_TENSOR;
+    if (gemv_stream_mt_applies(b, fused, di->sm_count, di->max_smem_optin))
+        return BL_GEMV_KERNEL_STREAM_MT;
+    return BL_GEMV_KERNEL_DP4A;
+}
+
 int launch_gemv_batch(const GemvBatch &b, bool fused, cudaStream_t s)
 {
     const DeviceInfo *di = device_info();
     if (!di)
         return BL_ERR_CUDA;
     // one token on a large layer: the producer/consumer streaming kernel;
-    // 2 .. 16 tokens: its multi-token form (one weight pass for all tokens)
+    // 2 .. 16 tokens: the tensor-core kernel or the multi-token streaming
+    // kernel (one weight pass for all tokens), as small_batch_tensor picks
     if (gemv_stream_applies(b, di->sm_count))
         return launch_gemv_stream(b, fused, s);
+    int cluster = 0;
+    if (small_batch_tensor(b, fused, &cluster))
+        return launch_gemv_tc(b, fused, s);
     if (gemv_stream_mt_applies(b, fused, di->sm_count, di->max_smem_optin))
         return launch_gemv_stream_mt(b, fused, s);
     Params p{};

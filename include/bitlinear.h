@@ -164,11 +164,12 @@ int bitlinear_quantize_act(const void *x, int xt, int64_t M, int64_t K,
  *   q, d, rowsum      from bitlinear_quantize_act (device), q is [M][K]
  *   y                 device, [M][ldy] of dtype yt (BL_F32 or BL_BF16), ldy >= N
  *   acc_dbg           NULL, or device [M][N] int32 receiving acc (before rescale)
- * M * K must not exceed 163840 (the activations are staged on chip).  Above
- * 8 tokens on weights of more than 4M entries the product runs on the
- * tensor-core path of bitlinear_gemm (dp4a work grows with M); otherwise 2 ..
- * 16 tokens share one streaming pass over the weights.  Results are
- * identical either way.
+ * M * K must not exceed 163840 (the activations are staged on chip).  2 ..
+ * 16 tokens run the tensor-core small-batch kernel or the dp4a multi-token
+ * streaming kernel (the crossover of BL_FLAG_SMALL_BATCH_DP4A's note), both
+ * one pass over the weights for all tokens; above 8 tokens on a shape that
+ * neither takes, the product runs on the tcgen05 GEMM of bitlinear_gemm.
+ * Results are identical either way.
  */
 int bitlinear_gemv(const uint8_t *packed, const float *w_scale, int64_t N,
                    int64_t K, const int8_t *q, const float *d,
@@ -203,6 +204,15 @@ int bitlinear_gemv_fused(const uint8_t *packed, const float *w_scale,
  * kernel immediately before this call in the stream. */
 #define BL_FLAG_PDL 1u
 
+/* Launch flags for 2 .. 16 tokens, which run either the tensor-core
+ * small-batch kernel or the dp4a multi-token streaming kernel.  By default the
+ * tensor cores take a batch when M * sum(N) * K >= 48 * 2^20 or K > 4096 (the
+ * measured crossover; the dp4a kernel's cost grows with M * N * K, the tensor
+ * cores' is nearly flat in M).  These flags force one or the other (where it
+ * applies); both give identical results. */
+#define BL_FLAG_SMALL_BATCH_DP4A 2u
+#define BL_FLAG_SMALL_BATCH_TENSOR 4u
+
 /*
  * Decode BitLinear for `count` weights that share the same activations x
  * (for instance the q, k and v products, or the gate and up products, of one
@@ -217,7 +227,8 @@ int bitlinear_gemv_fused(const uint8_t *packed, const float *w_scale,
  *   y[i], ldy[i]     device outputs [M][ldy[i]] of dtype yt
  *   acc_dbg          NULL, or a host array of `count` device pointers (each
  *                    NULL or [M][N[i]] int32)
- *   flags            0 or BL_FLAG_PDL
+ *   flags            0, or BL_FLAG_PDL and / or one of BL_FLAG_SMALL_BATCH_DP4A,
+ *                    BL_FLAG_SMALL_BATCH_TENSOR
  * The pointer arrays are host memory, read during the call only.
  */
 int bitlinear_gemv_fused_multi(int count, const uint8_t *const *packed,
@@ -226,6 +237,30 @@ int bitlinear_gemv_fused_multi(int count, const uint8_t *const *packed,
                                int64_t M, void *const *y, int yt,
                                const int64_t *ldy, int32_t *const *acc_dbg,
                                unsigned flags, void *stream);
+
+/* Kernels of the decode / small-batch GEMV entry points (bitlinear_gemv_plan). */
+#define BL_GEMV_KERNEL_STREAM 1      /* one token: producer-warp streaming kernel */
+#define BL_GEMV_KERNEL_TENSOR 2      /* 2 .. 16 tokens: tensor-core small-batch kernel */
+#define BL_GEMV_KERNEL_STREAM_MT 3   /* 2 .. 16 tokens: dp4a multi-token streaming kernel */
+#define BL_GEMV_KERNEL_DP4A 4        /* any other shape: per-warp dp4a kernel */
+
+/*
+ * Which kernel bitlinear_gemv_fused_multi (fused = 1, activations of dtype
+ * xt) or bitlinear_gemv (fused = 0, pre-quantised) runs for these shapes and
+ * flags, without running it; for the tensor-core kernel also the number of
+ * CTAs of a thread-block cluster that share one 128-row block's k range.
+ * The choice depends on the device (its SM count and how many clusters of a
+ * size it holds at once), so this needs the current device.  Where it
+ * answers BL_GEMV_KERNEL_DP4A for more than 8 pre-quantised tokens,
+ * bitlinear_gemv runs the tcgen05 GEMM instead.
+ *   count, N, K, M   as for bitlinear_gemv_fused_multi (N: host array)
+ *   kernel, cluster  host outputs: BL_GEMV_KERNEL_*, and the cluster size (0
+ *                    unless the tensor-core kernel)
+ * Returns BL_OK, or BL_ERR_NULL / BL_ERR_SHAPE / BL_ERR_DTYPE /
+ * BL_ERR_NO_DEVICE / BL_ERR_UNSUPPORTED.
+ */
+int bitlinear_gemv_plan(int count, const int64_t *N, int64_t K, int64_t M, int xt,
+                        int fused, unsigned flags, int *kernel, int *cluster);
 
 /*
  * RMSNorm, then per-token absmax int8 quantisation of the normalised rows:

@@ -269,3 +269,21 @@ def test_rope_table_argument_errors(bl):
     assert L.bitlinear_rope_table(128, 0, 1e4, A, None) == bl.BL_ERR_SHAPE
     assert L.bitlinear_rope_table(128, 64, 0.5, A, None) == bl.BL_ERR_SHAPE
     assert L.bitlinear_rope_table(128, 64, 1e4, A + 4, None) == bl.BL_ERR_ALIGN
+
+
+def test_gemv_plan_argument_errors(bl):
+    """bitlinear_gemv_plan checks its arguments before it asks for a device."""
+    import torch
+    L = bl.lib
+    N = (ctypes.c_int64 * 2)(2560, 640)
+    k, c = ctypes.c_int(0), ctypes.c_int(0)
+    kp, cp = ctypes.byref(k), ctypes.byref(c)
+    assert L.bitlinear_gemv_plan(2, None, 2560, 4, 1, 1, 0, kp, cp) == bl.BL_ERR_NULL
+    assert L.bitlinear_gemv_plan(2, N, 2560, 4, 1, 1, 0, None, cp) == bl.BL_ERR_NULL
+    assert L.bitlinear_gemv_plan(0, N, 2560, 4, 1, 1, 0, kp, cp) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_gemv_plan(2, N, 2560, 17, 1, 1, 0, kp, cp) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_gemv_plan(2, N, 2560, 4, 1, 1, 8, kp, cp) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_gemv_plan(2, N, 2560, 4, 9, 1, 0, kp, cp) == bl.BL_ERR_DTYPE
+    if not torch.cuda.is_available():
+        st = L.bitlinear_gemv_plan(2, N, 2560, 4, 1, 1, 0, kp, cp)
+        assert st in (bl.BL_ERR_CUDA, bl.BL_ERR_UNSUPPORTED)
