@@ -953,12 +953,20 @@ def run_mma_peak(args):
     bl.probe_mma_i8(reps=1000, device=dev)                 # warm-up
     with ClockSampler(0) as clk:
         runs = [bl.probe_mma_i8(reps=100000, device=dev) for _ in range(max(3, args.iters))]
+        # narrow MMAs (the small-batch GEMV's 128 x 32 x 32) from 1, 2 and 4 issuing warps
+        issue = [min((bl.probe_mma_i8(reps=50000, device=dev, n=32, issuers=w) for _ in range(3)),
+                     key=lambda r: r["cycles_per_mma_per_sm"]) for w in (1, 2, 4)]
     best = max(runs, key=lambda r: r["tops"])
     print(json.dumps({"case": "mma_peak", "mac_per_clk_per_sm": best["mac_per_clk_per_sm"],
                       "tops": best["tops"], "ctas": best["ctas"], "runs": len(runs),
+                      "cycles_per_mma_per_sm": best["cycles_per_mma_per_sm"],
+                      "narrow_mma_issue": [{"n": r["n"], "issuers": r["issuers"],
+                                            "cycles_per_mma_per_sm": r["cycles_per_mma_per_sm"],
+                                            "mac_per_clk_per_sm": r["mac_per_clk_per_sm"]} for r in issue],
                       "clocks": clk.summary(),
                       "note": "back-to-back tcgen05.mma.kind::i8 128x128x32 (A in TMEM, B in "
-                              "swizzled smem), no operand traffic, one CTA per SM"}), flush=True)
+                              "swizzled smem), no operand traffic, one CTA per SM; narrow_mma_issue: "
+                              "128x32x32 from 1, 2, 4 warps at once, each its own accumulator"}), flush=True)
 
 
 def main():

@@ -127,6 +127,7 @@ _SIGNATURES.update({
     "bitlinear_attention_workspace_bytes": (_sz, [_int, _int, _int]),
     "bitlinear_position_advance": (_int, [_vp, _vp]),
     "bitlinear_probe_mma_i8": (_int, [_int, _vp, _int, _vp]),
+    "bitlinear_probe_mma_i8_issue": (_int, [_int, _int, _int, _vp, _int, _vp]),
     "bitlinear_chain_plan_bytes": (_sz, [_int]),
     "bitlinear_chain_plan": (_int, [_int, ctypes.POINTER(ChainStepC), _vp, _sz, _vp]),
     "bitlinear_chain_run": (_int, [_vp, _int, _vp]),
@@ -652,25 +653,31 @@ def bitplane_gemv(w: BitPlaneWeight, x: torch.Tensor, out_dtype=torch.bfloat16, 
     return out
 
 
-def probe_mma_i8(reps: int = 4000, device="cuda") -> dict:
-    """Time back-to-back tcgen05 int8 MMAs of the prefill GEMM's form on every
-    SM (no operand traffic): MAC per clock per SM and TOPS over the grid."""
+def probe_mma_i8(reps: int = 4000, device="cuda", n: int = 128, issuers: int = 1) -> dict:
+    """Time back-to-back tcgen05 int8 MMAs (128 x n x 32, A in tensor memory,
+    B in shared memory, no operand traffic) on every SM from `issuers` warps
+    at once: MAC per clock per SM and TOPS over the grid.  n = 128 with one
+    issuer is the prefill GEMM's form."""
     dev = torch.device(device)
     grid = sm_count()
-    out = torch.zeros(2 * grid, dtype=torch.int64, device=dev)
+    out = torch.zeros(2 * issuers * grid, dtype=torch.int64, device=dev)
     with _on(dev):
-        _check(_lib.bitlinear_probe_mma_i8(reps, _ptr(out), grid, _stream(dev)),
-               "bitlinear_probe_mma_i8")
+        if n == 128 and issuers == 1:
+            _check(_lib.bitlinear_probe_mma_i8(reps, _ptr(out), grid, _stream(dev)), "bitlinear_probe_mma_i8")
+        else:
+            _check(_lib.bitlinear_probe_mma_i8_issue(n, issuers, reps, _ptr(out), grid, _stream(dev)),
+                   "bitlinear_probe_mma_i8_issue")
         torch.cuda.synchronize(dev)
-    res = out.view(grid, 2).cpu()
+    res = out.view(grid, issuers, 2).cpu()
     if bool((res < 0).any()):
         raise BitLinearError(BL_ERR_TIMEOUT, "bitlinear_probe_mma_i8")
-    macs = float(reps) * 8 * 128 * 128 * 32
-    cyc = res[:, 0].double()
-    ns = res[:, 1].double()
-    return {"reps": reps, "ctas": grid,
-            "mac_per_clk_per_sm": float((macs / cyc).median()),
-            "tops": float(2 * macs * grid / ns.max() / 1e3),
+    macs = float(reps) * 8 * 128 * n * 32            # per issuer
+    cyc = res[:, :, 0].double().max(dim=1).values      # per CTA: its slowest issuer
+    ns = res[:, :, 1].double()
+    return {"reps": reps, "ctas": grid, "n": n, "issuers": issuers,
+            "mac_per_clk_per_sm": float((issuers * macs / cyc).median()),
+            "cycles_per_mma_per_sm": float((cyc / (reps * 8 * issuers)).median()),
+            "tops": float(2 * issuers * macs * grid / ns.max() / 1e3),
             "ns_max": float(ns.max()), "cycles_median": float(cyc.median())}
 
 

@@ -871,11 +871,13 @@ int bitlinear_bitplane_gemv(const uint64_t *planes, const float *w_scale, int64_
                                 static_cast<cudaStream_t>(stream));
 }
 
-int bitlinear_probe_mma_i8(int reps, long long *out, int grid, void *stream)
+static int probe_mma(int n, int issuers, int reps, long long *out, int grid, void *stream)
 {
     if (!out)
         return BL_ERR_NULL;
     if (reps < 1 || reps > (1 << 17) || grid < 1)   // (1 << 17) stages: ~35 ms, far inside the 2 s wait
+        return BL_ERR_SHAPE;
+    if (!((n == 128 && (issuers == 1 || issuers == 2)) || (n == 32 && (issuers == 1 || issuers == 2 || issuers == 4))))
         return BL_ERR_SHAPE;
     if (reinterpret_cast<uintptr_t>(out) & 7u)
         return BL_ERR_ALIGN;
@@ -887,7 +889,17 @@ int bitlinear_probe_mma_i8(int reps, long long *out, int grid, void *stream)
         return BL_ERR_SHAPE;
     if ((st = check_dev_ptrs({out})))
         return st;
-    return launch_mma_probe(reps, out, grid, static_cast<cudaStream_t>(stream));
+    return launch_mma_probe(n, issuers, reps, out, grid, static_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_probe_mma_i8(int reps, long long *out, int grid, void *stream)
+{
+    return probe_mma(128, 1, reps, out, grid, stream);
+}
+
+int bitlinear_probe_mma_i8_issue(int n, int issuers, int reps, long long *out, int grid, void *stream)
+{
+    return probe_mma(n, issuers, reps, out, grid, stream);
 }
 
 int bitlinear_last_device_status(void *stream)

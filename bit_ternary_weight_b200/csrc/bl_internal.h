@@ -177,7 +177,7 @@ int launch_lut_gemv(const uint8_t *packed, const float *w_scale, int64_t N, int6
                     cudaStream_t s);
 
 // int8 tensor-core rate probe (mma_probe.cu): per CTA (clock cycles, ns).
-int launch_mma_probe(int reps, long long *out, int grid, cudaStream_t s);
+int launch_mma_probe(int n, int issuers, int reps, long long *out, int grid, cudaStream_t s);
 
 // Persistent decode chain (gemv_chain.cu).
 size_t chain_plan_bytes(int nsteps);

@@ -620,6 +620,18 @@ int bitlinear_bitplane_gemv(const uint64_t *planes, const float *w_scale,
 int bitlinear_probe_mma_i8(int reps, long long *out, int grid, void *stream);
 
 /*
+ * Measurement aid: how the issue rate of narrow MMAs depends on the number of
+ * issuing threads.  As bitlinear_probe_mma_i8, with MMAs of 128 x n x 32 (n =
+ * 32 or 128) issued by `issuers` warps of each CTA at once (1, 2 or 4 for n =
+ * 32; 1 or 2 for n = 128), each into its own accumulator columns.
+ *   out   device int64 [2 * issuers * grid]: per CTA and issuer, clock cycles
+ *         and nanoseconds (-1 if its final wait ran out)
+ * MACs per issuer = reps * 8 * 128 * n * 32; reps <= 131072.
+ */
+int bitlinear_probe_mma_i8_issue(int n, int issuers, int reps, long long *out, int grid,
+                                 void *stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device: BL_OK, BL_ERR_TIMEOUT if a kernel's bounded wait ran out,
  * or BL_ERR_SHAPE if a kernel found a device-side argument out of range (a

@@ -287,3 +287,15 @@ def test_gemv_plan_argument_errors(bl):
     if not torch.cuda.is_available():
         st = L.bitlinear_gemv_plan(2, N, 2560, 4, 1, 1, 0, kp, cp)
         assert st in (bl.BL_ERR_CUDA, bl.BL_ERR_UNSUPPORTED)
+
+
+def test_probe_argument_errors(bl):
+    """The tensor-core probes check their shapes before any CUDA call."""
+    A = 0x7f0000000000
+    L = bl.lib
+    assert L.bitlinear_probe_mma_i8(100, None, 1, None) == bl.BL_ERR_NULL
+    assert L.bitlinear_probe_mma_i8(0, A, 1, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_probe_mma_i8_issue(64, 1, 100, A, 1, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_probe_mma_i8_issue(32, 3, 100, A, 1, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_probe_mma_i8_issue(128, 4, 100, A, 1, None) == bl.BL_ERR_SHAPE
+    assert L.bitlinear_probe_mma_i8_issue(32, 4, 100, A + 4, 1, None) == bl.BL_ERR_ALIGN

@@ -586,3 +586,12 @@ def test_mma_probe_rate_is_plausible(bl):
     assert r["ctas"] == bl.sm_count()
     assert 1000 < r["mac_per_clk_per_sm"] < 20000
     assert bl.last_device_status() == 0
+
+
+def test_narrow_mma_issue_probe(bl):
+    """The 128 x 32 x 32 probe runs from 1, 2 and 4 warps; more issuers never
+    lower the per-SM rate, and every rate is physically possible."""
+    rates = [bl.probe_mma_i8(reps=2000, device=dev(), n=32, issuers=w)["mac_per_clk_per_sm"] for w in (1, 2, 4)]
+    assert all(500 < r < 20000 for r in rates)
+    assert rates[2] >= 0.9 * rates[0]
+    assert bl.last_device_status() == 0
