@@ -9,7 +9,8 @@
 //
 // Design (B200, persistent CTAs):
 //   * A CTA is KC consumer warps plus one producer warp: KC = 8 up to
-//     K = 8192, else KC = 16.  Large launches (at least 16 row groups per
+//     K = 8192 (10 for a launch of at most one CTA per SM whose k range has
+//     more than eight pieces of 256 k), else KC = 16.  Large launches (at least 16 row groups per
 //     SM) run two 8-warp CTAs per SM, so that a CTA of the next launch
 //     (programmatic dependent launch) can take the place of one that has
 //     finished, or one 16-warp CTA per SM, which halves the per-SM cost of
@@ -331,6 +332,21 @@ int launch_kc(const StreamParams &p, bool fused, int xt, cudaStream_t s, unsigne
     return launch_mode<KC, SMODE_X_BF16, 0>(p, s, flags);
 }
 
+// Ten consumer warps instead of eight for a launch of at most one CTA per SM
+// (fewer than kLargeGroupsPerSm row groups per SM) whose k range has more
+// than eight pieces: at K = 2560 (ten pieces) every warp takes one piece of a
+// group instead of two warps taking two, and at K = 6912 (27 pieces) a group
+// takes three stage rounds instead of four.  The stage work is bound by the
+// latency of each warp's dp4a chains, so the busiest warp sets its length.
+// Two such CTAs (352 threads) still fit on an SM beside each other, so the
+// next launch's CTA keeps fetching its weights early.
+bool ten_warps(const StreamParams &p)
+{
+    const DeviceInfo *di = device_info();
+    const int64_t ng_total = p.gstart[p.count];
+    return di && p.K / 256 > 8 && ng_total < kLargeGroupsPerSm * int64_t(di->sm_count);
+}
+
 }  // namespace
 
 // One token, K a multiple of 256 (at most 32768), at most kMaxGroupsPerCta
@@ -367,7 +383,8 @@ int launch_gemv_stream(const GemvBatch &b, bool fused, cudaStream_t s, const voi
     p.eps = eps;
     p.yt = b.yt;
     if (b.K <= kSmallK)
-        return launch_kc<8>(p, fused, b.xt, s, b.flags, norm);
+        return ten_warps(p) ? launch_kc<10>(p, fused, b.xt, s, b.flags, norm)
+                            : launch_kc<8>(p, fused, b.xt, s, b.flags, norm);
     return launch_kc<16>(p, fused, b.xt, s, b.flags, norm);
 }
 
@@ -392,7 +409,8 @@ int launch_gemv_stream_relu2(const GemvBatch &b, const void *x2, cudaStream_t s)
     p.x2 = x2;
     p.yt = b.yt;
     if (b.K <= kSmallK)
-        return launch_mode<8, SMODE_RELU2, 0>(p, s, b.flags);
+        return ten_warps(p) ? launch_mode<10, SMODE_RELU2, 0>(p, s, b.flags)
+                            : launch_mode<8, SMODE_RELU2, 0>(p, s, b.flags);
     return launch_mode<16, SMODE_RELU2, 0>(p, s, b.flags);
 }
 

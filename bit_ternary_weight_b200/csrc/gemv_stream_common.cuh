@@ -24,7 +24,8 @@ template <int KC>
 struct Geo {
     static constexpr int kConsumerThreads = 32 * KC;
     static constexpr int kThreads = kConsumerThreads + 32;   // + the producer warp
-    static constexpr int kCtasPerSm = KC == 8 ? 2 : 1;
+    // two CTAs of up to ten consumer warps fit on an SM (at <= 93 registers)
+    static constexpr int kCtasPerSm = KC <= 10 ? 2 : 1;
 };
 
 // Activations: pre-quantised q; raw bf16 / fp32 x quantised in the prologue;
@@ -159,10 +160,13 @@ __device__ __forceinline__ float stream_scale(Smem &sm, float amax)
     consumers_sync<KC>();
     float a = 0.0f;
 #pragma unroll
-    for (int w = 0; w < KC; w += 4) {
+    for (int w = 0; w + 4 <= KC; w += 4) {
         const float4 b4 = *reinterpret_cast<const float4 *>(&sm.bmax[w]);
         a = fmaxf(fmaxf(a, b4.x), fmaxf(b4.y, fmaxf(b4.z, b4.w)));
     }
+#pragma unroll
+    for (int w = KC & ~3; w < KC; ++w)
+        a = fmaxf(a, sm.bmax[w]);
     const float a_eff = fmaxf(a, kEps);
     if (tid == 0)
         sm.d = __fdiv_rn(a_eff, kQb);
