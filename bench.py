@@ -77,21 +77,32 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+def kernel_source_sha(csrc, names):
+    """sha256 of the kernel's source files, concatenated in the given order."""
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def profiled_traffic(chain: bool = True):
     """DRAM bytes per launch of the timed kernel from the committed ncu
     summary, or None when the kernel source has changed since those counters
     were taken."""
     import hashlib
     import re
+    csrc = os.path.join(ROOT, "bit_ternary_weight_b200", "csrc")
     if chain:
         prof = os.path.join(ROOT, "profiles", "decode_chain_2b_launches.md")
-        src = os.path.join(ROOT, "bit_ternary_weight_b200", "csrc", "gemv_chain.cu")
+        srcs = ["gemv_chain.cu", "gemv_stream_common.cuh"]
     else:
         prof = os.path.join(ROOT, "profiles", "decode_stream_2b_gemv_launches.md")
-        src = os.path.join(ROOT, "bit_ternary_weight_b200", "csrc", "gemv_stream.cu")
+        srcs = ["gemv_stream.cu", "gemv_stream_common.cuh"]
     try:
         text = open(prof).read()
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        sha = kernel_source_sha(csrc, srcs)
         m = re.search(r"sha256 prefix `([0-9a-f]+)`", text)
         t = re.search(r"traffic_per_launch_bytes: (\d+)", text)
         if m and t and sha.startswith(m.group(1)):
@@ -877,7 +888,7 @@ def run_ours(args, world, rank, local):
                      "peak_kind": f"{peak_kind} HBM copy bandwidth",
                      "kernel": ("gemv_chain_kernel (one persistent launch per token)"
                                 if kernel_launches_per_step == 1 else
-                                "gemv_stream_kernel<KC=8, bf16 fused> (4 launches per layer)"),
+                                "gemv_stream_kernel<KC=10, bf16 fused> (4 launches per layer)"),
                      "note": "algorithmic bytes = packed weight bytes per launch; duration = "
                              "step time / launches per step (CUDA events over the timed "
                              "region, on the launching stream)"},
