@@ -30,6 +30,8 @@
 // the absmax quantiser above.  The fp64 sum's order differs from the
 // oracle's, which can change ms only when S / K lies within about 1e-15
 // (relative) of an fp32 rounding boundary.
+#include <algorithm>
+
 #include "bl_common.cuh"
 
 namespace bl {
@@ -421,6 +423,85 @@ int launch_row_quant(const void *x, int xt, int64_t M, int64_t K, int64_t ldx, c
     return launch_row_quant_x<BL_F32>(p, norm, gt, s);
 }
 
+// Many short rows (bf16, K <= 3072): one warp per token over a grid of a
+// few CTAs per SM, each warp walking tokens gw, gw + warps, ...  The whole
+// row sits in the lanes' registers (CH 16-byte vectors per lane), both
+// reductions are warp shuffles, and there is no block barrier: a CTA per
+// token (above) is bound by how fast the GPU starts CTAs when a row is only
+// a few KB.  Same arithmetic as quantize_act_kernel.
+constexpr int kRowsThreads = 256;
+
+template <int CH>
+__global__ void __launch_bounds__(kRowsThreads, 2)
+quantize_rows_bf16_kernel(const __nv_bfloat16 *__restrict__ x, int64_t M, int64_t K, int64_t ldx,
+                          int8_t *__restrict__ q, float *__restrict__ d, int32_t *__restrict__ rowsum)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = int64_t(gridDim.x) * (kRowsThreads / 32);
+    const int chunks = int(K / 8);
+    for (int64_t m = (int64_t(blockIdx.x) * kRowsThreads + threadIdx.x) >> 5; m < M; m += nwarps) {
+        const __nv_bfloat16 *xr = x + m * ldx;
+        uint4 raw[CH];
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int c = lane + 32 * i;
+            raw[i] = c < chunks ? ld_ro_v4(xr + int64_t(c) * 8) : make_uint4(0, 0, 0, 0);
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            float f[8];
+            bf16x8_to_f32(raw[i], f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                amax = fmaxf(amax, fabsf(f[j]));
+        }
+        // per-lane maxima are finite and >= 0: their bit patterns order like the values
+        amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+        const float a_eff = fmaxf(amax, kEps);
+        const float s = __fdiv_rn(kQb, a_eff);
+        int sum = 0;
+        int8_t *qrow = q + m * K;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int c = lane + 32 * i;
+            if (c < chunks) {
+                float f[8];
+                bf16x8_to_f32(raw[i], f);
+                uint32_t lo = 0, hi = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int t0 = quant1(f[j], s), t1 = quant1(f[j + 4], s);
+                    sum += t0 + t1;
+                    lo |= (uint32_t(t0) & 0xffu) << (8 * j);
+                    hi |= (uint32_t(t1) & 0xffu) << (8 * j);
+                }
+                *reinterpret_cast<uint2 *>(qrow + int64_t(c) * 8) = make_uint2(lo, hi);
+            }
+        }
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0) {
+            rowsum[m] = sum;
+            d[m] = __fdiv_rn(a_eff, kQb);
+        }
+    }
+}
+
+template <int CH>
+int launch_rows(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q, float *d, int32_t *rowsum,
+                cudaStream_t s)
+{
+    const DeviceInfo *di = device_info();
+    if (!di)
+        return BL_ERR_CUDA;
+    const int64_t warps_needed = M;
+    const int64_t cap = int64_t(di->sm_count) * 2;   // two CTAs of eight warps per SM
+    const int64_t grid = std::min<int64_t>(cap, (warps_needed + 7) / 8);
+    quantize_rows_bf16_kernel<CH><<<unsigned(grid), kRowsThreads, 0, s>>>(
+        static_cast<const __nv_bfloat16 *>(x), M, K, ldx, q, d, rowsum);
+    return launch_status();
+}
+
 }  // namespace
 
 // Plain quantisation runs the CTA-per-token kernel: measured against the
@@ -429,6 +510,11 @@ int launch_row_quant(const void *x, int xt, int64_t M, int64_t K, int64_t ldx, c
 int launch_quantize_act(const void *x, int xt, int64_t M, int64_t K, int64_t ldx,
                         int8_t *q, float *d, int32_t *rowsum, cudaStream_t s)
 {
+    // many tokens of short bf16 rows: a warp per token
+    if (xt == BL_BF16 && M >= 1024 && K <= 2048)
+        return launch_rows<8>(x, M, K, ldx, q, d, rowsum, s);
+    if (xt == BL_BF16 && M >= 1024 && K <= 3072)
+        return launch_rows<12>(x, M, K, ldx, q, d, rowsum, s);
     dim3 grid(static_cast<unsigned>(M));
     if (xt == BL_BF16)
         quantize_act_kernel<BL_BF16><<<grid, kQuantThreads, 0, s>>>(x, K, ldx, q, d, rowsum);

@@ -66,7 +66,8 @@ def test_pack_zero_weight(bl):
 # ------------------------------------------------------------------ activation quant
 
 @pytest.mark.parametrize("M,K", [(1, 256), (3, 2560), (16, 6912), (128, 256), (512, 2560),
-                                 (2, 28672), (8192, 6912)])
+                                 (2, 28672), (8192, 6912), (8192, 2560), (1024, 2048), (1031, 3072),
+                                 (2048, 320)])
 @pytest.mark.parametrize("xdtype", [torch.bfloat16, torch.float32])
 def test_quantize_parity(bl, M, K, xdtype):
     x = si.activations(M, K, seed=M + K, dtype=xdtype)
@@ -95,6 +96,27 @@ def test_quantize_edge_tokens(bl):
         np.testing.assert_array_equal(q.cpu().numpy(), q_o)
         np.testing.assert_array_equal(f32_bits(d.cpu().numpy()), f32_bits(d_o))
         np.testing.assert_array_equal(r.cpu().numpy(), r_o)
+
+
+def test_quantize_many_short_rows_edge_tokens(bl):
+    """The warp-per-token kernel (bf16, many rows, K <= 3072) on the edge
+    tokens of test_quantize_edge_tokens, spread over 1500 rows of a strided
+    view, with a ragged K (a last lane chunk only partly used)."""
+    M, K, ld = 1500, 2368, 2560
+    base = si.activations(M, ld, seed=11, dtype=torch.bfloat16)
+    x = base[:, :K].clone()
+    x[0] = 0.0
+    x[77, 17] = 1e4
+    x[500] = 3.0
+    x[500, ::2] = -3.0
+    x[1001] = 1e-30
+    x[1499, 5] = -x[1499].abs().max() * 2
+    base[:, :K] = x
+    q_o, d_o, r_o = oracle.quantize_act(x.float().numpy())
+    q, d, r = bl.quantize_act(base.to(dev())[:, :K])
+    np.testing.assert_array_equal(q.cpu().numpy(), q_o)
+    np.testing.assert_array_equal(f32_bits(d.cpu().numpy()), f32_bits(d_o))
+    np.testing.assert_array_equal(r.cpu().numpy(), r_o)
 
 
 def test_quantize_strided_rows(bl):
