@@ -955,6 +955,30 @@ def run_case(args):
                       "note": "same weights every launch (L2-warm unless profiled)"}), flush=True)
 
 
+def run_decoder_case(args):
+    """The synthetic decoder stack, eager (no graph), `--iters` tokens from
+    `--ctx` cached positions with `--layers` layers: for launch lists and
+    per-launch profiles of one token's kernels; prints one JSON line."""
+    import bit_ternary_weight_b200 as bl  # noqa: F401  (loads the library)
+    from bit_ternary_weight_b200.decoder import Decoder, DecoderConfig
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = DecoderConfig(layers=args.layers, max_seq=args.ctx + args.iters + 8)
+    dec = Decoder.random(cfg, seed=1, device=dev)
+    dec.h.copy_(si.activations(1, cfg.hidden, seed=5)[0])
+    dec.set_position(args.ctx)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.iters):
+        dec.step()
+    e.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"case": "decoder", "layers": args.layers, "context": args.ctx, "tokens": args.iters,
+                      "us_per_token_eager": s.elapsed_time(e) * 1000.0 / args.iters,
+                      "launches_per_token": 5 * args.layers + 1}), flush=True)
+
+
 def run_mma_peak(args):
     """The int8 tensor-core rate of the prefill GEMM's MMA form, with the SM
     clocks sampled while it runs; prints one JSON line."""
@@ -982,7 +1006,8 @@ def run_mma_peak(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["stream", "gemv", "gemm", "binary", "bitplane", "lut", "mma_peak"],
+    ap.add_argument("--case", choices=["stream", "gemv", "gemm", "binary", "bitplane", "lut", "mma_peak",
+                                       "decoder"],
                     default="stream",
                     help="stream: the benchmark; others: one kernel on one shape (profiling)")
     ap.add_argument("--K", type=int, default=8192)
@@ -994,6 +1019,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=si.LAYERS_2B)
+    ap.add_argument("--ctx", type=int, default=512, help="--case decoder: cached positions")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=2.0)
     ap.add_argument("--no-extra", action="store_true")
@@ -1010,6 +1036,9 @@ def main():
         args.warmup = 3
     if args.case == "mma_peak":
         run_mma_peak(args)
+        return
+    if args.case == "decoder":
+        run_decoder_case(args)
         return
     if args.case != "stream":
         run_case(args)

@@ -36,13 +36,17 @@
 //   * meanwhile rotates the queries of the kv head's query heads and, in the
 //     block holding pos, the new key, which it appends with the new value;
 //   * scores its positions (eight lanes per position, sixteen dimensions each,
-//     fp64 partial dot products for every query head), takes the block
-//     maximum, the fp64 weights, their sum and the fp64 weighted values
-//     (lanes over dimensions, four position groups), and writes them to the
-//     workspace;
+//     fp64 partial dot products for every query head, in four independent
+//     partial sums), takes the block maximum, the fp64 weights, their sum and
+//     the fp64 weighted values (lanes over dimensions, eight position groups),
+//     and writes them to the workspace;
 //   * arrives on the kv head's ticket (fence, atomic add); the last CTA to
-//     arrive combines the blocks in block order, divides, rounds and stores,
-//     and resets the ticket.
+//     arrive combines the blocks in block order (sixteen blocks' partial
+//     values of two outputs loaded together before they are added), divides,
+//     rounds and stores, and resets the ticket.
+// 256 threads: the fp64 phases are bound by latency (fp64 runs at half the
+// fp32 rate here), so each SM sub-partition needs two warps; the queries are
+// kept as fp64 in shared memory (one conversion each, not one per position).
 // A position outside the cache records BL_ERR_SHAPE in the device status word
 // and writes nothing; a bulk copy that does not land in 2 s records
 // BL_ERR_TIMEOUT and that CTA leaves without output (the workspace's ticket
@@ -54,7 +58,8 @@ namespace {
 
 constexpr int kHeadDim = 128;
 constexpr int kPosBlock = 64;             // cached positions per CTA
-constexpr int kAttnThreads = 128;
+constexpr int kAttnThreads = 256;
+constexpr int kAttnWarps = kAttnThreads / 32;
 constexpr int kMaxGroup = 8;              // query heads per kv head
 constexpr uint32_t kRowBytes = kHeadDim * 2;
 
@@ -79,13 +84,16 @@ struct AttnSmem {
     int abort_flag;
     int last;
     float2 cs[kHeadDim / 2];               // (cos, sin) of the token's angles
-    float qs[kMaxGroup][kHeadDim];         // rotated queries of the group
+    // rotated queries of the group (bf16 values, as fp64): dimension 16 c + e
+    // at [17 c + e], so the eight lanes of a position (one chunk c each) read
+    // different banks
+    double qs[kMaxGroup][kHeadDim / 16 * 17];
     float ks[kHeadDim];                    // rotated new key (block holding pos)
     float vs[kHeadDim];                    // new value
     float sc[kMaxGroup][kPosBlock];        // scores
     float mb[kMaxGroup];                   // block maxima
     double ew[kMaxGroup][kPosBlock];       // weights exp(s - m_b)
-    double part[4][kMaxGroup][kHeadDim];   // per position group weighted values
+    double part[kAttnWarps][kMaxGroup][kHeadDim];   // per position group weighted values
     alignas(128) __nv_bfloat16 kb[kPosBlock][kHeadDim];   // the block's cached keys
     alignas(128) __nv_bfloat16 vb[kPosBlock][kHeadDim];   // ... and values
 };
@@ -189,8 +197,8 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
             const int g = t / (kHeadDim / 2), i = t % (kHeadDim / 2);
             float a, b;
             rope_pair(qw[u], sm.cs[i], a, b);
-            sm.qs[g][2 * i] = a;
-            sm.qs[g][2 * i + 1] = b;
+            sm.qs[g][(2 * i) / 16 * 17 + (2 * i) % 16] = double(a);
+            sm.qs[g][(2 * i) / 16 * 17 + (2 * i) % 16 + 1] = double(b);
         }
     }
     if (has_new && tid < kHeadDim / 2) {
@@ -215,7 +223,7 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
     // ---- scores: eight lanes per position, sixteen dims each
     const float scale = __double2float_rn(1.0 / sqrt(double(kHeadDim)));
     const int sub = lane & 7, r = lane >> 3;
-    for (int jb = warp * 4; jb < n; jb += 4 * (kAttnThreads / 32)) {
+    for (int jb = warp * 4; jb < n; jb += 4 * kAttnWarps) {
         const int jj = jb + r;
         float kf[16];
         if (jj < nk) {
@@ -227,14 +235,21 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
             for (int e = 0; e < 16; ++e)
                 kf[e] = jj < n ? sm.ks[sub * 16 + e] : 0.0f;
         }
+        double kd[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            kd[e] = double(kf[e]);
 #pragma unroll
         for (int g = 0; g < kMaxGroup; ++g) {
             if (g >= G)
                 break;
-            double dot = 0.0;
+            // four independent partial sums (every product exact; the order
+            // of the fp64 sums is free, see above)
+            double d4[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-                dot = __fma_rn(double(sm.qs[g][sub * 16 + e]), double(kf[e]), dot);   // exact products
+                d4[e & 3] = __fma_rn(sm.qs[g][sub * 17 + e], kd[e], d4[e & 3]);
+            double dot = __dadd_rn(__dadd_rn(d4[0], d4[1]), __dadd_rn(d4[2], d4[3]));
             dot = __dadd_rn(dot, __shfl_xor_sync(0xffffffffu, dot, 1));
             dot = __dadd_rn(dot, __shfl_xor_sync(0xffffffffu, dot, 2));
             dot = __dadd_rn(dot, __shfl_xor_sync(0xffffffffu, dot, 4));
@@ -244,7 +259,7 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
     }
     __syncthreads();
     // ---- block maxima, fp64 weights and their sums (warp g per head)
-    for (int g = warp; g < G; g += kAttnThreads / 32) {
+    for (int g = warp; g < G; g += kAttnWarps) {
         float m = -INFINITY;
         for (int jj = lane; jj < n; jj += 32)
             m = fmaxf(m, sm.sc[g][jj]);
@@ -267,7 +282,7 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
         }
     }
     __syncthreads();
-    // ---- weighted values: thread (pg, c) dims 4c .. 4c+3, positions pg, pg + 4, ...
+    // ---- weighted values: thread (pg, c) dims 4c .. 4c+3, positions pg, pg + kAttnWarps, ...
     const int pg = tid >> 5, c = tid & 31;
     double acc[kMaxGroup][4];
 #pragma unroll
@@ -275,7 +290,7 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
 #pragma unroll
         for (int x = 0; x < 4; ++x)
             acc[g][x] = 0.0;
-    for (int jj = pg; jj < n; jj += 4) {
+    for (int jj = pg; jj < n; jj += kAttnWarps) {
         float vf[4];
         if (jj < nk) {
             const uint2 ab = *reinterpret_cast<const uint2 *>(&sm.vb[jj][4 * c]);
@@ -311,7 +326,7 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
         const int g = t / kHeadDim, d = t % kHeadDim;
         double num = 0.0;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
+        for (int q4 = 0; q4 < kAttnWarps; ++q4)
             num = __dadd_rn(num, sm.part[q4][g][d]);
         p.bnum[(size_t(kv * G + g) * p.nblk + blk) * kHeadDim + d] = num;
     }
@@ -330,7 +345,7 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
     const bool fit = nact <= kPosBlock;
     __shared__ float gm[kMaxGroup];
     __shared__ double gs[kMaxGroup];
-    for (int g = warp; g < G; g += kAttnThreads / 32) {
+    for (int g = warp; g < G; g += kAttnWarps) {
         const size_t hb = size_t(kv * G + g) * p.nblk;
         float m = -INFINITY;
         for (int b = lane; b < nact; b += 32)
@@ -354,16 +369,49 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
         }
     }
     __syncthreads();
-    for (int t = tid; t < G * kHeadDim; t += kAttnThreads) {
-        const int g = t / kHeadDim, d = t % kHeadDim;
-        const size_t hb = size_t(kv * G + g) * p.nblk;
-        double num = 0.0;
-#pragma unroll 8
-        for (int b = 0; b < nact; ++b) {
-            const double f = fit ? fac[g * kPosBlock + b] : exp(double(__ldcg(p.bmax + hb + b)) - double(gm[g]));
-            num = __fma_rn(__ldcg(p.bnum + (hb + b) * kHeadDim + d), f, num);
+    if (fit) {
+        // each thread's outputs (g, d) for t = tid, tid + kAttnThreads, ...;
+        // sixteen blocks' partial values of both of a thread's first two
+        // outputs loaded together, then added
+        for (int t0 = tid; t0 < G * kHeadDim; t0 += 2 * kAttnThreads) {
+            const int t1 = t0 + kAttnThreads;
+            const bool two = t1 < G * kHeadDim;
+            const int g0 = t0 / kHeadDim, d0 = t0 % kHeadDim;
+            const int g1 = two ? t1 / kHeadDim : g0, d1 = two ? t1 % kHeadDim : d0;
+            const size_t hb0 = size_t(kv * G + g0) * p.nblk, hb1 = size_t(kv * G + g1) * p.nblk;
+            double num0 = 0.0, num1 = 0.0;
+            for (int b0 = 0; b0 < nact; b0 += 16) {
+                double v0[16], v1[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const bool in = b0 + u < nact;
+                    v0[u] = in ? __ldcg(p.bnum + (hb0 + b0 + u) * kHeadDim + d0) : 0.0;
+                    v1[u] = in && two ? __ldcg(p.bnum + (hb1 + b0 + u) * kHeadDim + d1) : 0.0;
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    if (b0 + u < nact) {
+                        num0 = __fma_rn(v0[u], fac[g0 * kPosBlock + b0 + u], num0);
+                        num1 = __fma_rn(v1[u], fac[g1 * kPosBlock + b0 + u], num1);
+                    }
+                }
+            }
+            p.out[(kv * G + g0) * kHeadDim + d0] = __float2bfloat16_rn(__double2float_rn(__ddiv_rn(num0, gs[g0])));
+            if (two)
+                p.out[(kv * G + g1) * kHeadDim + d1] =
+                    __float2bfloat16_rn(__double2float_rn(__ddiv_rn(num1, gs[g1])));
         }
-        p.out[(kv * G + g) * kHeadDim + d] = __float2bfloat16_rn(__double2float_rn(__ddiv_rn(num, gs[g])));
+    } else {
+        for (int t = tid; t < G * kHeadDim; t += kAttnThreads) {
+            const int g = t / kHeadDim, d = t % kHeadDim;
+            const size_t hb = size_t(kv * G + g) * p.nblk;
+            double num = 0.0;
+            for (int b = 0; b < nact; ++b) {
+                const double f = exp(double(__ldcg(p.bmax + hb + b)) - double(gm[g]));
+                num = __fma_rn(__ldcg(p.bnum + (hb + b) * kHeadDim + d), f, num);
+            }
+            p.out[(kv * G + g) * kHeadDim + d] = __float2bfloat16_rn(__double2float_rn(__ddiv_rn(num, gs[g])));
+        }
     }
     if (tid == 0)
         p.ticket[kv] = 0u;
