@@ -343,6 +343,21 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
     // factors exp(m_b - m) per head and block (reusing ew), and the sums
     double *fac = &sm.ew[0][0];               // [G][nact] when nact <= 64, else recomputed
     const bool fit = nact <= kPosBlock;
+    // up to 16 blocks and two outputs per thread: the blocks' partial values
+    // are loaded first, so that their round trip overlaps the factors'
+    const bool pre = fit && nact <= 16 && G * kHeadDim <= 2 * kAttnThreads;
+    const int pt1 = tid + kAttnThreads;
+    const bool has0 = tid < G * kHeadDim, has1 = pt1 < G * kHeadDim;
+    const int pg0 = tid / kHeadDim, pd0 = tid % kHeadDim, pg1 = pt1 / kHeadDim, pd1 = pt1 % kHeadDim;
+    double pv0[16], pv1[16];
+    if (pre) {
+        const size_t hb0 = size_t(kv * G + pg0) * p.nblk, hb1 = size_t(kv * G + pg1) * p.nblk;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            pv0[u] = has0 && u < nact ? __ldcg(p.bnum + (hb0 + u) * kHeadDim + pd0) : 0.0;
+            pv1[u] = has1 && u < nact ? __ldcg(p.bnum + (hb1 + u) * kHeadDim + pd1) : 0.0;
+        }
+    }
     __shared__ float gm[kMaxGroup];
     __shared__ double gs[kMaxGroup];
     for (int g = warp; g < G; g += kAttnWarps) {
@@ -369,7 +384,20 @@ __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const At
         }
     }
     __syncthreads();
-    if (fit) {
+    if (pre) {
+        double num0 = 0.0, num1 = 0.0;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            if (u < nact) {
+                num0 = __fma_rn(pv0[u], fac[(has0 ? pg0 : 0) * kPosBlock + u], num0);
+                num1 = __fma_rn(pv1[u], fac[(has1 ? pg1 : 0) * kPosBlock + u], num1);
+            }
+        }
+        if (has0)
+            p.out[(kv * G + pg0) * kHeadDim + pd0] = __float2bfloat16_rn(__double2float_rn(__ddiv_rn(num0, gs[pg0])));
+        if (has1)
+            p.out[(kv * G + pg1) * kHeadDim + pd1] = __float2bfloat16_rn(__double2float_rn(__ddiv_rn(num1, gs[pg1])));
+    } else if (fit) {
         // each thread's outputs (g, d) for t = tid, tid + kAttnThreads, ...;
         // sixteen blocks' partial values of both of a thread's first two
         // outputs loaded together, then added
