@@ -41,9 +41,9 @@
 //     the fp64 weighted values (lanes over dimensions, eight position groups),
 //     and writes them to the workspace;
 //   * arrives on the kv head's ticket (fence, atomic add); the last CTA to
-//     arrive combines the blocks in block order (sixteen blocks' partial
-//     values of two outputs loaded together before they are added), divides,
-//     rounds and stores, and resets the ticket.
+//     arrive combines the blocks in block order (the blocks' partial values
+//     of its outputs loaded first, overlapping the round trip for the block
+//     maxima and sums), divides, rounds and stores, and resets the ticket.
 // 256 threads: the fp64 phases are bound by latency (fp64 runs at half the
 // fp32 rate here), so each SM sub-partition needs two warps; the queries are
 // kept as fp64 in shared memory (one conversion each, not one per position).
