@@ -135,13 +135,16 @@ __device__ __forceinline__ void bf16x8(const uint4 v, float *f)
     }
 }
 
+// GT: the query heads per kv head when known at compile time (1, 2, 4, 8),
+// so that the per-head loops unroll without a runtime bound; 0: any.
+template <int GT>
 __global__ void __launch_bounds__(kAttnThreads) attention_decode_kernel(const AttnParams p)
 {
     extern __shared__ __align__(128) unsigned char attn_raw[];
     AttnSmem &sm = *reinterpret_cast<AttnSmem *>(attn_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kv = blockIdx.x, blk = blockIdx.y;
-    const int G = p.H / p.Hkv;
+    const int G = GT > 0 ? GT : p.H / p.Hkv;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int pos = int(ld_dep_u32(p.pos));
@@ -495,6 +498,35 @@ int launch_rope_table(float *tab, int D, int T_max, double base, cudaStream_t s)
     return launch_status();
 }
 
+namespace {
+
+template <int GT>
+int launch_attn_t(const AttnParams &p, unsigned flags, cudaStream_t s)
+{
+    const size_t smem = sizeof(AttnSmem);
+    int per_sm = 0;
+    int st = occupancy(reinterpret_cast<const void *>(attention_decode_kernel<GT>), kAttnThreads, smem, &per_sm);
+    if (st)
+        return st;
+    if (per_sm < 1)
+        return BL_ERR_SHAPE;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(p.Hkv), unsigned(p.nblk));
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    if (flags & BL_FLAG_PDL) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cuda_status(cudaLaunchKernelEx(&cfg, attention_decode_kernel<GT>, p));
+}
+
+}  // namespace
+
 int launch_attention_decode(const void *q, const void *k, const void *v, void *cache_k, void *cache_v,
                             const int32_t *pos, int H, int Hkv, int D, int T_max, double rope_base,
                             const float *rope, void *out, void *ws, unsigned flags, cudaStream_t s)
@@ -525,26 +557,14 @@ int launch_attention_decode(const void *q, const void *k, const void *v, void *c
     p.bnum = reinterpret_cast<double *>(base + w.bnum);
     p.ticket = reinterpret_cast<unsigned *>(base + w.ticket);
     p.status = di->status;
-    const size_t smem = sizeof(AttnSmem);
-    int per_sm = 0;
-    int st = occupancy(reinterpret_cast<const void *>(attention_decode_kernel), kAttnThreads, smem, &per_sm);
-    if (st)
-        return st;
-    if (per_sm < 1)
-        return BL_ERR_SHAPE;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(Hkv), unsigned(p.nblk));
-    cfg.blockDim = dim3(kAttnThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    if (flags & BL_FLAG_PDL) {
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+    const int g = H / Hkv;
+    switch (g) {
+    case 1: return launch_attn_t<1>(p, flags, s);
+    case 2: return launch_attn_t<2>(p, flags, s);
+    case 4: return launch_attn_t<4>(p, flags, s);
+    case 8: return launch_attn_t<8>(p, flags, s);
+    default: return launch_attn_t<0>(p, flags, s);
     }
-    return cuda_status(cudaLaunchKernelEx(&cfg, attention_decode_kernel, p));
 }
 
 int launch_position_advance(int32_t *pos, cudaStream_t s)
