@@ -66,8 +66,8 @@ namespace bl {
 namespace {
 
 constexpr int kBM = 128;     // weight rows per tile (MMA M)
-constexpr int kBK = 256;     // k per pipeline stage: eight MMAs between barrier waits
-constexpr int kBoxK = 128;   // k per TMA box (one 128-byte swizzle span of activations)
+constexpr int kBK = kTcStageK;   // k per pipeline stage: eight MMAs between barrier waits
+constexpr int kBoxK = kTcBoxK;  // k per TMA box (one 128-byte swizzle span of activations)
 constexpr int kBoxes = kBK / kBoxK;
 constexpr int kQStages = 5;  // operand ring (shared memory): activations and packed weights
 constexpr int kAStages = 4;  // expanded weight ring (tensor memory)
@@ -76,7 +76,6 @@ constexpr int kProducerWarps = 2;
 constexpr int kMmaWarp = kProducerWarps;
 constexpr int kExpWarp0 = kMmaWarp + 1;
 constexpr int kEpiWarp0 = kExpWarp0 + 4 * kExpGroups;
-constexpr int kMmaK = 32;    // k per tcgen05.mma.kind::i8
 constexpr uint32_t kTmemCols = 512;  // D: 2 x BN columns in [0, 256); A: kAStages x 64 columns in [256, 512)
 constexpr uint32_t kDCols = 256;
 constexpr uint32_t kPBox = kBM * kBoxK / 4;    // 4 KB of packed weights per box

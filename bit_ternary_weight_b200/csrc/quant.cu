@@ -65,7 +65,7 @@ quantize_act_kernel(const void *__restrict__ x, int64_t K, int64_t ldx,
     const bool in_regs = chunks <= int64_t(kQuantThreads) * kQuantRegChunks;
     // register copy of the row: raw bf16 vectors, or eight floats per chunk
     constexpr int kRegF = XT == BL_BF16 ? 1 : 8;
-    uint4 raw[XT == BL_BF16 ? kQuantRegChunks : 1];
+    uint4 raw[XT == BL_BF16 ? kQuantRegChunks : 1] = {};
     float v[XT == BL_BF16 ? 1 : kQuantRegChunks][kRegF];
     auto chunk_f32 = [&](int i, float f[8]) {
         if constexpr (XT == BL_BF16) {
