@@ -299,3 +299,18 @@ def test_probe_argument_errors(bl):
     assert L.bitlinear_probe_mma_i8_issue(32, 3, 100, A, 1, None) == bl.BL_ERR_SHAPE
     assert L.bitlinear_probe_mma_i8_issue(128, 4, 100, A, 1, None) == bl.BL_ERR_SHAPE
     assert L.bitlinear_probe_mma_i8_issue(32, 4, 100, A + 4, 1, None) == bl.BL_ERR_ALIGN
+
+
+def test_binding_constants_match_the_header(bl):
+    """The binding's launch flags and kernel ids are the header's."""
+    text = open(os.path.join(ROOT, "include", "bitlinear.h")).read()
+    defs = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define\s+(BL_\w+)\s+(\d+)u?\b", text)}
+    for name in ("BL_FLAG_PDL", "BL_FLAG_SMALL_BATCH_DP4A", "BL_FLAG_SMALL_BATCH_TENSOR"):
+        assert getattr(bl, name) == defs[name], name
+    kernels = {v: k for k, v in bl.GEMV_KERNELS.items()}
+    assert kernels["stream"] == defs["BL_GEMV_KERNEL_STREAM"]
+    assert kernels["tensor"] == defs["BL_GEMV_KERNEL_TENSOR"]
+    assert kernels["stream_mt"] == defs["BL_GEMV_KERNEL_STREAM_MT"]
+    assert kernels["dp4a"] == defs["BL_GEMV_KERNEL_DP4A"]
+    assert bl.BL_ACT_PLAIN == defs["BL_ACT_PLAIN"] and bl.BL_ACT_RMSNORM == defs["BL_ACT_RMSNORM"]
+    assert bl.BL_ACT_RELU2_GATE == defs["BL_ACT_RELU2_GATE"]
