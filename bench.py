@@ -933,7 +933,8 @@ def run_case(args):
     else:
         w = bl.pack(W)
         if args.case == "gemv":
-            fn = lambda: bl.gemv_fused(w, x)  # noqa: E731
+            y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            fn = lambda: bl.gemv_fused_multi([w], x, outs=[y], small_batch=args.small_batch)  # noqa: E731
         else:
             q, d, r = bl.quantize_act(x)
             ws = torch.zeros(max(bl.gemm_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=dev)
@@ -950,9 +951,12 @@ def run_case(args):
     e.record()
     torch.cuda.synchronize()
     t = s.elapsed_time(e) / 1000.0 / args.iters
-    print(json.dumps({"case": args.case, "K": K, "N": N, "M": M, "iters": args.iters,
-                      "us": t * 1e6, "weight_GBps": nbytes / t / 1e9, "TOPS": ops / t / 1e12,
-                      "note": "same weights every launch (L2-warm unless profiled)"}), flush=True)
+    line = {"case": args.case, "K": K, "N": N, "M": M, "iters": args.iters,
+            "us": t * 1e6, "weight_GBps": nbytes / t / 1e9, "TOPS": ops / t / 1e12,
+            "note": "same weights every launch (L2-warm unless profiled)"}
+    if args.case == "gemv":
+        line["kernel"] = list(bl.gemv_plan([N], K, M, small_batch=args.small_batch))
+    print(json.dumps(line), flush=True)
 
 
 def run_decoder_case(args):
@@ -1020,6 +1024,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=si.LAYERS_2B)
     ap.add_argument("--ctx", type=int, default=512, help="--case decoder: cached positions")
+    ap.add_argument("--small-batch", choices=["auto", "tensor", "dp4a"], default="auto",
+                    help="--case gemv with 2..16 tokens: the small-batch kernel to run")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=2.0)
     ap.add_argument("--no-extra", action="store_true")
