@@ -74,3 +74,27 @@ def test_clock_summary_without_samples_says_so():
     cs = bench.ClockSampler(0)
     s = cs.summary()
     assert s["sm_mhz"] is None and s["reasons"] == ["unavailable"]
+
+
+def test_cpu_baseline_reports_all_cores_one_core_and_prefill():
+    """The CPU baseline of the GPU arm: the best of three all-core samples,
+    one single-core sample and a prefill timing, each with its own cores."""
+    bench = _bench()
+    import oracle
+    cores = oracle.num_threads()
+    cb = bench.cpu_baseline(0.0)
+    assert cb["kind"] == "oracle" and cb["unit"] == "GB/s"
+    assert len(cb["runs_GBps"]) == 3 and cb["value"] == max(cb["runs_GBps"])
+    assert int(cb["cores"]) == cores
+    assert cb["one_core"]["cores"] == 1 and cb["one_core"]["value"] > 0
+    assert cb["prefill"]["TOPS"] > 0 and cb["prefill"]["M"] == 64
+    assert oracle.num_threads() == cores          # the thread count is restored
+
+
+def test_gemv_path_names_every_kernel():
+    """bench.py's path names cover every kernel the library's plan can report."""
+    bench = _bench()
+    import bit_ternary_weight_b200 as bl
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    for kern in bl.GEMV_KERNELS.values():
+        assert f'"{kern}":' in src, kern
