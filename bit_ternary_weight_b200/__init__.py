@@ -50,11 +50,13 @@ GEMV_MAX_M = 16
 
 
 class BitLinearError(RuntimeError):
-    def __init__(self, status: int, where: str):
+    def __init__(self, status: int, where: str, detail: str | None = None):
         self.status = status
         msg = _lib.bitlinear_status_string(status).decode()
         if status == BL_ERR_CUDA:
             msg += " (" + _lib.bitlinear_last_cuda_error().decode() + ")"
+        if detail:
+            msg += f" ({detail})"
         super().__init__(f"{where}: {msg}")
 
 
@@ -173,6 +175,113 @@ def _on(device: torch.device):
     return contextlib.nullcontext()
 
 
+_FLOATS = (torch.float32, torch.bfloat16)
+_I8 = (torch.int8,)
+_I32 = (torch.int32,)
+_U8 = (torch.uint8,)
+_F32 = (torch.float32,)
+_BF16 = (torch.bfloat16,)
+
+
+def _fits(t, where: str, name: str, dtypes, rows: int, cols: int, ld: int | None = None):
+    """Refuse, before the call, a caller buffer of another element type than
+    the kernel reads or writes there, or one that does not hold the `rows` x
+    `cols` elements the kernel addresses (row r at element r * ld, ld = cols
+    unless given): the library sees only a pointer, so a short or mistyped
+    buffer would be read or written out of its bounds."""
+    if t is None:
+        return
+    if t.dtype not in dtypes:
+        want = " or ".join(str(d).replace("torch.", "") for d in dtypes)
+        raise BitLinearError(BL_ERR_DTYPE, where,
+                             f"{name} is {str(t.dtype).replace('torch.', '')}, needs {want}")
+    if rows < 1 or cols < 1:
+        return                      # the library rejects the shape itself
+    ld = cols if ld is None else ld
+    if rows == 1:
+        ok = t.numel() >= cols and (t.is_contiguous() or
+                                    (t.size(-1) >= cols and t.stride(-1) == 1))
+    elif t.dim() == 2:
+        ok = (t.size(0) >= rows and t.size(1) >= cols and t.stride(0) == ld and
+              (t.size(1) == 1 or t.stride(1) == 1))
+    else:
+        ok = t.dim() == 1 and t.is_contiguous() and ld == cols and t.numel() >= rows * cols
+    esz = t.element_size()
+    if ok:
+        avail = t.untyped_storage().nbytes() - t.storage_offset() * esz
+        ok = ((rows - 1) * ld + cols) * esz <= avail
+    if not ok:
+        pitch = f" with row pitch {ld}" if rows > 1 and ld != cols else ""
+        raise BitLinearError(BL_ERR_SHAPE, where, f"{name} of shape {tuple(t.shape)} and strides "
+                             f"{tuple(t.stride())} does not hold [{rows}][{cols}]{pitch}")
+
+
+def _same_k(weights, where: str) -> int:
+    """The shared K of products that read one activation row."""
+    if not weights:
+        raise BitLinearError(BL_ERR_SHAPE, where, "no weights")
+    K = weights[0].K
+    if any(w.K != K for w in weights):
+        raise BitLinearError(BL_ERR_SHAPE, where,
+                             f"weights of different K {sorted({w.K for w in weights})} share x")
+    return K
+
+
+def _per_product(lst, n: int, where: str, name: str):
+    if lst is not None and len(lst) != n:
+        raise BitLinearError(BL_ERR_SHAPE, where, f"{len(lst)} {name} for {n} weights")
+
+
+def _same_dtype(outs, where: str):
+    if any(o.dtype != outs[0].dtype for o in outs):
+        raise BitLinearError(BL_ERR_DTYPE, where, "outputs of mixed element types")
+
+
+def _weight(w, where: str):
+    """The buffers of a packed ternary weight hold its N x K codes and gamma."""
+    _fits(w.packed, where, "packed", _U8, 1, packed_bytes(w.N, w.K))
+    _fits(w.w_scale, where, "w_scale", _F32, 1, 1)
+
+
+def _act(x, where: str, K: int, name: str = "x"):
+    """The activations of a product have the weight's K features."""
+    if x.dim() == 0 or x.shape[-1] != K:
+        raise BitLinearError(BL_ERR_SHAPE, where,
+                             f"{name} of shape {tuple(x.shape)} for a weight of K={K}")
+
+
+def _outputs(where: str, weights, outs, acc_dbgs, M: int, lds=None):
+    """Products sharing one launch: an output (one element type for all) and
+    an optional int32 accumulator per weight, each [M][N]."""
+    n = len(weights)
+    _per_product(outs, n, where, "outputs")
+    _per_product(acc_dbgs, n, where, "accumulators")
+    _same_dtype(outs, where)
+    for i, w in enumerate(weights):
+        _weight(w, where)
+        _fits(outs[i], where, f"outs[{i}]", _FLOATS, M, w.N, None if lds is None else lds[i])
+        _fits(None if acc_dbgs is None else acc_dbgs[i], where, f"acc_dbgs[{i}]", _I32, M, w.N)
+
+
+def _one_token(where: str, w, x, xtypes, out, acc_dbg, name: str = "x"):
+    """One token x [K] in, y [N] (and the int32 accumulators) out."""
+    _act(x, where, w.K, name)
+    _fits(x, where, name, xtypes, 1, w.K)
+    _fits(out, where, "out", _FLOATS, 1, w.N)
+    _fits(acc_dbg, where, "acc_dbg", _I32, 1, w.N)
+
+
+def _pre_quantised(where: str, w, q, d, rowsum, M: int, out, acc_dbg):
+    """The operands of a product on pre-quantised activations."""
+    _weight(w, where)
+    _act(q, where, w.K, "q")
+    _fits(q, where, "q", _I8, M, w.K)
+    _fits(d, where, "d", _F32, 1, M)
+    _fits(rowsum, where, "rowsum", _I32, 1, M)
+    _fits(out, where, "out", _FLOATS, M, w.N, out.stride(0))
+    _fits(acc_dbg, where, "acc_dbg", _I32, M, w.N)
+
+
 @dataclass
 class TernaryWeight:
     """A packed ternary weight: TL bytes, the fp32 gamma_eff and the shape."""
@@ -220,6 +329,10 @@ def pack_noalloc(W: torch.Tensor, packed: torch.Tensor, w_scale: torch.Tensor) -
     not exceed PACK_NOALLOC_MAX_ROWS).  For callers that cannot allocate
     device memory when they pack; this function allocates nothing either."""
     N, K = W.shape
+    where = "bitlinear_pack_noalloc"
+    _fits(W, where, "W", _FLOATS, N, K)
+    _fits(packed, where, "packed", _U8, 1, packed_bytes(N, K))
+    _fits(w_scale, where, "w_scale", _F32, 1, 1)
     with _on(W.device):
         _check(_lib.bitlinear_pack_noalloc(_ptr(W), _dt(W.dtype), N, K, _ptr(packed),
                                            _ptr(w_scale), _stream(W.device)),
@@ -239,6 +352,11 @@ def quantize_act(x: torch.Tensor, out=None):
         r = torch.empty(M, dtype=torch.int32, device=x.device)
     else:
         q, d, r = out
+    where = "bitlinear_quantize_act"
+    _fits(x, where, "x", _FLOATS, M, K, x.stride(0))
+    _fits(q, where, "q", _I8, M, K)
+    _fits(d, where, "d", _F32, 1, M)
+    _fits(r, where, "rowsum", _I32, 1, M)
     with _on(x.device):
         _check(_lib.bitlinear_quantize_act(_ptr(x), _dt(x.dtype), M, K, x.stride(0), _ptr(q),
                                            _ptr(d), _ptr(r), _stream(x.device)),
@@ -256,6 +374,7 @@ def gemv(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc
     """Decode GEMV (1 <= M <= 16) on pre-quantised activations."""
     M = q.shape[0]
     out = _out(M, w.N, out_dtype, q.device, out)
+    _pre_quantised("bitlinear_gemv", w, q, d, rowsum, M, out, acc_dbg)
     with _on(q.device):
         _check(_lib.bitlinear_gemv(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q), _ptr(d),
                                    _ptr(rowsum), M, _ptr(out), _dt(out.dtype), out.stride(0),
@@ -270,6 +389,12 @@ def gemv_fused(w: TernaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16, out=
         x = x.unsqueeze(0)
     M = x.shape[0]
     out = _out(M, w.N, out_dtype, x.device, out)
+    where = "bitlinear_gemv_fused"
+    _weight(w, where)
+    _act(x, where, w.K)
+    _fits(x, where, "x", _FLOATS, M, w.K, x.stride(0))
+    _fits(out, where, "out", _FLOATS, M, w.N, out.stride(0))
+    _fits(acc_dbg, where, "acc_dbg", _I32, M, w.N)
     with _on(x.device):
         _check(_lib.bitlinear_gemv_fused(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(x),
                                          _dt(x.dtype), x.stride(0), M, _ptr(out), _dt(out.dtype),
@@ -302,8 +427,13 @@ def gemv_fused_multi(weights, x: torch.Tensor, out_dtype=torch.bfloat16, outs=No
         x = x.unsqueeze(0)
     n = len(weights)
     M = x.shape[0]
+    where = "bitlinear_gemv_fused_multi"
+    K = _same_k(weights, where)
     if outs is None:
         outs = [torch.empty(M, w.N, dtype=out_dtype, device=x.device) for w in weights]
+    _act(x, where, K)
+    _fits(x, where, "x", _FLOATS, M, K, x.stride(0))
+    _outputs(where, weights, outs, acc_dbgs, M, [o.stride(0) for o in outs])
     P = ctypes.c_void_p * n
     I64 = ctypes.c_int64 * n
     packed = P(*[w.packed.data_ptr() for w in weights])
@@ -354,6 +484,12 @@ def rmsnorm_quantize_act(x: torch.Tensor, gain=None, eps: float = RMS_EPS, out=N
     else:
         q, d, r = out
     gt = BL_F32 if gain is None else _dt(gain.dtype)
+    where = "bitlinear_rmsnorm_quantize_act"
+    _fits(x, where, "x", _FLOATS, M, K, x.stride(0))
+    _fits(gain, where, "gain", _FLOATS, 1, K)
+    _fits(q, where, "q", _I8, M, K)
+    _fits(d, where, "d", _F32, 1, M)
+    _fits(r, where, "rowsum", _I32, 1, M)
     with _on(x.device):
         _check(_lib.bitlinear_rmsnorm_quantize_act(_ptr(x), _dt(x.dtype), M, K, x.stride(0),
                                                    _ptr(gain), gt, float(eps), _ptr(q), _ptr(d),
@@ -369,8 +505,14 @@ def rmsnorm_gemv_fused_multi(weights, x: torch.Tensor, gain=None, eps: float = R
     sharing it (gate/up, q/k/v), in one launch.  x: [K] or [1, K]."""
     x = x.reshape(-1)
     n = len(weights)
+    where = "bitlinear_rmsnorm_gemv_fused_multi"
+    K = _same_k(weights, where)
     if outs is None:
         outs = [torch.empty(1, w.N, dtype=out_dtype, device=x.device) for w in weights]
+    _act(x, where, K)
+    _fits(x, where, "x", _FLOATS, 1, K)
+    _fits(gain, where, "gain", _FLOATS, 1, K)
+    _outputs(where, weights, outs, acc_dbgs, 1)
     P = ctypes.c_void_p * n
     I64 = ctypes.c_int64 * n
     packed = P(*[w.packed.data_ptr() for w in weights])
@@ -402,8 +544,20 @@ def decode_linear(weights, x: torch.Tensor, act: int = BL_ACT_PLAIN, x2=None, ga
     (resid[i]: bf16 [N] added before the rounding; may be outs[i] itself)."""
     x = x.reshape(-1)
     n = len(weights)
+    where = "bitlinear_decode_linear"
+    K = _same_k(weights, where)
     if outs is None:
         outs = [torch.empty(w.N, dtype=out_dtype, device=x.device) for w in weights]
+    _act(x, where, K)
+    _fits(x, where, "x", _FLOATS, 1, K)
+    if x2 is not None:
+        _act(x2.reshape(-1), where, K, "x2")
+        _fits(x2, where, "x2", _FLOATS, 1, K)
+    _fits(gain, where, "gain", _FLOATS, 1, K)
+    _outputs(where, weights, outs, acc_dbgs, 1)
+    _per_product(resid, n, where, "residuals")
+    for i, w in enumerate(weights):
+        _fits(None if resid is None else resid[i], where, f"resid[{i}]", _BF16, 1, w.N)
     P = ctypes.c_void_p * n
     I64 = ctypes.c_int64 * n
     packed = P(*[w.packed.data_ptr() for w in weights])
@@ -449,18 +603,30 @@ def attention_decode(q, k, v, cache_k, cache_v, pos, H: int, Hkv: int, out=None,
         out = torch.empty(H * D, dtype=torch.bfloat16, device=q.device)
     if workspace is None:
         workspace = attention_workspace(H, Hkv, T_max, q.device)
+    where = "bitlinear_attention_decode"
+    _fits(q, where, "q", _BF16, 1, H * D)
+    _fits(k, where, "k", _BF16, 1, Hkv * D)
+    _fits(v, where, "v", _BF16, 1, Hkv * D)
+    _fits(cache_k, where, "cache_k", _BF16, 1, Hkv * T_max * D)
+    _fits(cache_v, where, "cache_v", _BF16, 1, Hkv * T_max * D)
+    _fits(pos, where, "pos", _I32, 1, 1)
+    _fits(out, where, "out", _BF16, 1, H * D)
+    _fits(table, where, "table", _F32, 1, T_max * D)
+    _fits(workspace, where, "workspace", (workspace.dtype,), 1, workspace.numel())
+    ws_bytes = workspace.numel() * workspace.element_size()
     with _on(q.device):
         _check(_lib.bitlinear_attention_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(cache_k),
                                                _ptr(cache_v), _ptr(pos), H, Hkv, D, T_max,
                                                float(rope_base), _ptr(table), _ptr(out),
-                                               _ptr(workspace),
-                                               workspace.numel(), BL_FLAG_PDL if pdl else 0,
+                                               _ptr(workspace), ws_bytes,
+                                               BL_FLAG_PDL if pdl else 0,
                                                _stream(q.device)),
                "bitlinear_attention_decode")
     return out
 
 
 def position_advance(pos: torch.Tensor):
+    _fits(pos, "bitlinear_position_advance", "pos", _I32, 1, 1)
     with _on(pos.device):
         _check(_lib.bitlinear_position_advance(_ptr(pos), _stream(pos.device)),
                "bitlinear_position_advance")
@@ -491,6 +657,12 @@ class DecodeChain:
         device = device or steps[0].x.device
         arr = (ChainStepC * n)()
         for i, st in enumerate(steps):
+            where = f"bitlinear_chain_plan (step {i})"
+            K = _same_k(st.weights, where)
+            _act(st.x, where, K)
+            _fits(st.x, where, "x", _FLOATS, 1, K)
+            _fits(st.gain, where, "gain", _FLOATS, 1, K)
+            _outputs(where, st.weights, st.outs, st.acc_dbgs, 1)
             c = arr[i]
             c.count = len(st.weights)
             for j, (w, o) in enumerate(zip(st.weights, st.outs)):
@@ -547,6 +719,10 @@ def gemm(w: TernaryWeight, q, d, rowsum, out_dtype=torch.bfloat16, out=None, acc
         # zero before its first use; every call leaves it zero again
         workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    where = "bitlinear_gemm"
+    _pre_quantised(where, w, q, d, rowsum, M, out, acc_dbg)
+    if workspace is not None:
+        _fits(workspace, where, "workspace", (workspace.dtype,), 1, workspace.numel())
     with _on(q.device):
         _check(_lib.bitlinear_gemm(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q), _ptr(d),
                                    _ptr(rowsum), M, _ptr(out), _dt(out.dtype), out.stride(0),
@@ -601,6 +777,10 @@ def binary_gemv(w: BinaryWeight, x: torch.Tensor, out_dtype=torch.bfloat16, out=
     x = x.reshape(-1)
     if out is None:
         out = torch.empty(w.N, dtype=out_dtype, device=x.device)
+    where = "bitlinear_binary_gemv"
+    _fits(w.bits, where, "bits", (torch.int64,), 1, w.N * (w.K // 64))
+    _fits(w.s_w, where, "s_w", _F32, 1, 1)
+    _one_token(where, w, x, _FLOATS, out, acc_dbg)
     with _on(x.device):
         _check(_lib.bitlinear_binary_gemv(_ptr(w.bits), _ptr(w.s_w), w.N, w.K, _ptr(x),
                                           _dt(x.dtype), _ptr(out), _dt(out.dtype), _ptr(acc_dbg),
@@ -614,6 +794,10 @@ def lut_gemv(w: TernaryWeight, q, d, out_dtype=torch.bfloat16, out=None, acc_dbg
     q = q.reshape(-1)
     if out is None:
         out = torch.empty(1, w.N, dtype=out_dtype, device=q.device)
+    where = "bitlinear_lut_gemv"
+    _weight(w, where)
+    _one_token(where, w, q, _I8, out, acc_dbg, "q")
+    _fits(d, where, "d", _F32, 1, 1)
     with _on(q.device):
         _check(_lib.bitlinear_lut_gemv(_ptr(w.packed), _ptr(w.w_scale), w.N, w.K, _ptr(q),
                                        _ptr(d), _ptr(out), _dt(out.dtype), _ptr(acc_dbg),
@@ -632,6 +816,7 @@ class BitPlaneWeight:
 
 def bitplane_pack(w: TernaryWeight) -> BitPlaneWeight:
     """Bit-planes of a packed ternary weight (same codes, same gamma)."""
+    _weight(w, "bitlinear_bitplane_pack")
     planes = torch.empty(w.N, w.K // 64, 2, dtype=torch.int64, device=w.packed.device)
     with _on(w.packed.device):
         _check(_lib.bitlinear_bitplane_pack(_ptr(w.packed), w.N, w.K, _ptr(planes),
@@ -645,6 +830,10 @@ def bitplane_gemv(w: BitPlaneWeight, x: torch.Tensor, out_dtype=torch.bfloat16, 
     x = x.reshape(-1)
     if out is None:
         out = torch.empty(w.N, dtype=out_dtype, device=x.device)
+    where = "bitlinear_bitplane_gemv"
+    _fits(w.planes, where, "planes", (torch.int64,), 1, w.N * (w.K // 64) * 2)
+    _fits(w.w_scale, where, "w_scale", _F32, 1, 1)
+    _one_token(where, w, x, _FLOATS, out, acc_dbg)
     with _on(x.device):
         _check(_lib.bitlinear_bitplane_gemv(_ptr(w.planes), _ptr(w.w_scale), w.N, w.K, _ptr(x),
                                             _dt(x.dtype), _ptr(out), _dt(out.dtype),
