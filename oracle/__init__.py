@@ -28,6 +28,10 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "bitlinear_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
+# The test of the pins themselves (tests/test_oracle_mutations.py) builds
+# copies of the C source with one planted mistake each and points the oracle
+# at such a copy through this variable; nothing else sets it.
+_LIB_OVERRIDE = os.environ.get("BITLINEAR_ORACLE_LIB")
 _lock = threading.Lock()
 _lib = None
 
@@ -36,7 +40,10 @@ _CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle C source into ``liboracle.so`` next to it."""
+    """Compile the oracle C source into ``liboracle.so`` next to it (or, under
+    BITLINEAR_ORACLE_LIB, return that prebuilt library untouched)."""
+    if _LIB_OVERRIDE:
+        return _LIB_OVERRIDE
     stale = (not os.path.exists(_LIB_PATH)
              or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
     if force or stale:

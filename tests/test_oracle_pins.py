@@ -311,6 +311,24 @@ def test_rmsnorm_constant_row_gives_the_gain(c):
     np.testing.assert_array_equal(h[0], np.sign(c) * gain)
 
 
+def test_rmsnorm_then_quantise_gives_the_gain_on_a_constant_token():
+    """RMSNorm of a constant token is the gain times one common factor, and the
+    absmax quantiser removes that factor: with integer gains 1 .. 127 the codes
+    are the gains themselves (every x*s lies within a few ulp of an integer,
+    far from a rounding tie), d = max h / 127, and the row sum is the sum of
+    the gains.  Quantising the raw token instead would give 127 everywhere."""
+    K = 254
+    gain = (np.arange(K) % 127 + 1).astype(np.float32)
+    for c in (1.0, -3.5, 0.01):
+        x = np.full((1, K), c, np.float32)
+        q, d, r = oracle.rmsnorm_quantize_act(x, gain)
+        want = np.sign(c) * gain
+        np.testing.assert_array_equal(q[0], want.astype(np.int8))
+        assert r[0] == int(want.sum())
+        h = oracle.rmsnorm(x, gain)
+        assert d[0] == np.float32(np.abs(h).max() / np.float32(127.0))
+
+
 def test_rmsnorm_power_of_two_scale_invariance():
     x = si.activations(3, 512, seed=4, dtype=torch.float32).numpy()
     gain = 1.0 + 0.1 * si.activations(1, 512, seed=5, outliers=False, dtype=torch.float32).numpy()
@@ -494,3 +512,100 @@ def test_decoder_layer_closed_forms():
     out = oracle.decoder_layer(h, layer, ck, cv, 3, cfg)
     np.testing.assert_array_equal(out, h)
     assert (ck[:, [0, 1, 2, 4, 5, 6, 7]] == 7.0).all() and not (ck[:, 3] == 7.0).all()
+
+
+def _run_layer(layer, cfg, h, pos, T=8):
+    ck = np.zeros((cfg["kv_heads"], T, cfg["head_dim"]), np.float32)
+    cv = np.zeros_like(ck)
+    return oracle.decoder_layer(h, layer, ck, cv, pos, cfg), ck, cv
+
+
+def _h(seed, positive=False):
+    a = si.activations(1, 256, seed=seed, dtype=torch.float32).numpy()[0]
+    return oracle.bf16_round(np.abs(a) + 0.25 if positive else a)
+
+
+def test_decoder_layer_first_position_attends_to_itself():
+    """At position 0 the softmax runs over the token's own key: the layer's
+    output is finite and differs from its input, and cache row 0 holds the
+    token's key and value."""
+    layer, cfg = _layer(3)
+    h = _h(5)
+    out, ck, cv = _run_layer(layer, cfg, h, 0)
+    assert np.isfinite(out).all()
+    assert (out != h).any()
+    assert ck[:, 0].any() and cv[:, 0].any() and not ck[:, 1:].any() and not cv[:, 1:].any()
+
+
+def test_decoder_layer_each_gain_belongs_to_its_sublayer():
+    """A zero RMSNorm gain zeroes every BitLinear input behind it.  Zero
+    attention gain and zero FFN weights: the token's q, k, v are 0 (cache row
+    0), attention over zero caches gives 0, and the stream is unchanged.  Zero
+    FFN gain and zero attention weights: gate = up = 0, unchanged again.  In
+    each case the other gain is 1 and the other sublayer's weights are not
+    zero, so a gain applied in front of the wrong sublayer shows."""
+    layer, cfg = _layer(4, zero=("gate", "up", "down"))
+    layer["g_attn"] = np.zeros(256, np.float32)
+    h = _h(6)
+    out, ck, cv = _run_layer(layer, cfg, h, 2)
+    np.testing.assert_array_equal(out, h)
+    assert not ck.any() and not cv.any()
+    layer, cfg = _layer(5, zero=("q", "k", "v", "o"))
+    layer["g_ffn"] = np.zeros(256, np.float32)
+    out, _, _ = _run_layer(layer, cfg, h, 2)
+    np.testing.assert_array_equal(out, h)
+
+
+def test_decoder_layer_ffn_adds_to_the_attention_output():
+    """Zero FFN weights: the output is the stream after the attention
+    residual, which moved (the o projection is not zero)."""
+    layer, cfg = _layer(6, zero=("gate", "up", "down"))
+    h = _h(7)
+    out, _, _ = _run_layer(layer, cfg, h, 1)
+    assert (out != h).any()
+    # and the FFN with zero weights adds exactly nothing to it: one more
+    # layer whose attention is silenced (zero gain) leaves it unchanged
+    layer["g_attn"] = np.zeros(256, np.float32)
+    out2, _, _ = _run_layer(layer, cfg, out, 1)
+    np.testing.assert_array_equal(out2, out)
+
+
+def test_decoder_layer_gate_is_the_relu_squared_factor():
+    """A positive token (after RMSNorm with a positive gain it quantises to
+    q >= 0) against gate weights <= 0 gives gate <= 0, so relu(gate)^2 = 0
+    closes the FFN whatever up is: with the o projection zero the stream is
+    unchanged.  With gate and up exchanged the FFN would not be closed."""
+    layer, cfg = _layer(8, zero=("o",))
+    Wg = -np.abs(si.weight(384, 256, seed=81).numpy())
+    g = oracle.weight_scale(Wg)
+    layer["gate"] = (g, oracle.ternary_codes(Wg, g))
+    assert (layer["gate"][1] <= 0).all() and (layer["gate"][1] < 0).any()
+    h = _h(9, positive=True)
+    out, _, _ = _run_layer(layer, cfg, h, 3)
+    np.testing.assert_array_equal(out, h)
+    # the same layer with gate weights >= 0 does move the stream
+    layer["gate"] = (g, -layer["gate"][1])
+    out, _, _ = _run_layer(layer, cfg, h, 3)
+    assert (out != h).any()
+
+
+def test_decoder_layer_caches_rotated_keys_and_plain_values():
+    """The cached key at position p is the position-0 key (RoPE at 0 is the
+    identity) rotated by p; the cached value does not depend on p; a zero
+    value projection caches zero values but non-zero keys, and the reverse."""
+    layer, cfg = _layer(10)
+    h = _h(11)
+    _, ck0, cv0 = _run_layer(layer, cfg, h, 0)
+    for p in (1, 5):
+        _, ckp, cvp = _run_layer(layer, cfg, h, p)
+        rot = oracle.bf16_round(oracle.rope(ck0[:, 0].reshape(-1), cfg["kv_heads"],
+                                            cfg["head_dim"], p))
+        np.testing.assert_array_equal(ckp[:, p].reshape(-1), rot)
+        np.testing.assert_array_equal(cvp[:, p], cv0[:, 0])
+        assert (ckp[:, p] != ck0[:, 0]).any()
+    layer, cfg = _layer(12, zero=("v",))
+    _, ck, cv = _run_layer(layer, cfg, h, 2)
+    assert ck[:, 2].any() and not cv.any()
+    layer, cfg = _layer(13, zero=("k",))
+    _, ck, cv = _run_layer(layer, cfg, h, 2)
+    assert not ck.any() and cv[:, 2].any()
