@@ -30,6 +30,10 @@
  *   acc[m][n] = sum_k code[n][k] * q[m][k] (exact int32, |acc| <= 128 K).
  *   y[m][n]   = ((float)acc * d[m]) * gamma_eff, two fp32 round-to-nearest
  *               products in that order; bf16 output rounds y to nearest even.
+ *   Inputs must be finite (the pages define no other case): a NaN or +-Inf
+ *   in token m of x leaves q[m], d[m], rowsum[m] and row m of y unspecified,
+ *   and one in W leaves gamma and every output unspecified.  Such input
+ *   causes no fault and no error status, and other tokens are unaffected.
  *
  * Packed ternary layout "TL" (the pages fix none; this library's choice):
  *   stored value s = code + 1 in {0, 1, 2} (3 never appears), rows padded to
