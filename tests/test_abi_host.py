@@ -314,3 +314,53 @@ def test_binding_constants_match_the_header(bl):
     assert kernels["dp4a"] == defs["BL_GEMV_KERNEL_DP4A"]
     assert bl.BL_ACT_PLAIN == defs["BL_ACT_PLAIN"] and bl.BL_ACT_RMSNORM == defs["BL_ACT_RMSNORM"]
     assert bl.BL_ACT_RELU2_GATE == defs["BL_ACT_RELU2_GATE"]
+
+
+_C_HOST = r"""
+#include <stdio.h>
+#include <stdint.h>
+#include "bitlinear.h"
+
+int main(void)
+{
+    /* sizes and strings need no device */
+    printf("%zu %zu %s\n", bitlinear_packed_bytes(13, 256), bitlinear_packed_bytes(8, 100),
+           bitlinear_status_string(BL_ERR_SHAPE));
+    /* argument errors come back before any CUDA call */
+    uintptr_t a = (uintptr_t)0x7f0000000000ull;
+    const uint8_t *packed = (const uint8_t *)a;
+    const float *scale = (const float *)a;
+    const int8_t *q = (const int8_t *)a;
+    const float *d = (const float *)a;
+    const int32_t *r = (const int32_t *)a;
+    void *y = (void *)a;
+    int s1 = bitlinear_gemv(packed, scale, 256, 256, NULL, d, r, 1, y, BL_BF16, 256, NULL, NULL);
+    int s2 = bitlinear_gemv(packed, scale, 256, 100, q, d, r, 1, y, BL_BF16, 256, NULL, NULL);
+    int s3 = bitlinear_gemv(packed, scale, 256, 256, q, d, r, 1, y, 7, 256, NULL, NULL);
+    printf("%d %d %d\n", s1, s2, s3);
+    return 0;
+}
+"""
+
+
+@pytest.mark.parametrize("compiler,std", [("gcc", "-std=c11"), ("g++", "-std=c++17")])
+def test_plain_c_host_links_and_calls_the_library(bl, tmp_path, compiler, std):
+    """A C (and a C++) program with no Python or torch includes the header
+    under strict warnings, links libbitlinear.so and gets the documented
+    sizes, strings and argument errors."""
+    import shutil
+    import subprocess
+    if not shutil.which(compiler):
+        pytest.skip("no compiler")
+    src = tmp_path / ("host.c" if compiler == "gcc" else "host.cpp")
+    src.write_text(_C_HOST)
+    exe = tmp_path / "host"
+    libdir = os.path.dirname(bl.LIB_PATH)
+    subprocess.run([compiler, std, "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-lbitlinear", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    first = out[0].split(" ", 2)
+    assert int(first[0]) == oracle.packed_bytes(13, 256) and int(first[1]) == 0
+    assert first[2].startswith("BL_ERR_SHAPE")
+    assert [int(v) for v in out[1].split()] == [bl.BL_ERR_NULL, bl.BL_ERR_SHAPE, bl.BL_ERR_DTYPE]
