@@ -157,6 +157,7 @@ def job_throughput(bytes_per_step_per_rank: float, steps: int, world: int, t_max
 class ClockSampler:
     """nvidia-smi samples of this GPU's clocks during the timed region."""
 
+    PERIOD_MS = 100
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -170,14 +171,14 @@ class ClockSampler:
         except Exception:
             sel = []
         self.cmd = ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}",
-                    "--format=csv,noheader,nounits", "-lms", "200"]
+                    "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)]
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(self.cmd, stdout=self.out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
-        time.sleep(0.3)
+        time.sleep(0.15)            # nvidia-smi's start-up
         return self
 
     def __exit__(self, *exc):
@@ -319,6 +320,14 @@ def build_split_stream(bl, layers: int, seed: int, device):
 def run_split_step(chain, pdl=True):
     for cpd, x in chain:
         cpd(x, pdl=pdl)
+
+
+def load_replays(graph, n: int):
+    """n untimed replays of the step's graph, then a synchronize: the same load
+    as the timed steps, for the clock samples around them."""
+    for _ in range(n):
+        graph.replay()
+    torch.cuda.synchronize()
 
 
 def time_graph(graph, steps, world):
@@ -762,9 +771,21 @@ def run_ours(args, world, rank, local):
         graph.replay()
     torch.cuda.synchronize()
 
+    # the timed steps last milliseconds, far less than nvidia-smi's sampling
+    # period, so the same replays run for ~0.5 s on either side of them (each
+    # side ended by a synchronize; the timed steps keep their own barrier and
+    # synchronize on both sides) and the samples see the clocks under this
+    # load.  The replay count is agreed over the ranks: a split step's graph
+    # holds collectives, so every rank must replay it equally often.
+    t_est = max_over_ranks(time_graph(graph, args.warmup, world) / args.warmup, world)
+    n_load = max(1, min(100000, int(0.5 / max(t_est, 1e-6))))
     with ClockSampler(local) as clk:
+        load_replays(graph, n_load)
         t = time_graph(graph, args.steps, world)
+        load_replays(graph, n_load)
     clocks = clk.summary()
+    clocks["how"] = (f"nvidia-smi every {ClockSampler.PERIOD_MS} ms while the step's graph "
+                     f"replays {n_load} times (~0.5 s) on each side of the timed steps")
     t = max_over_ranks(t, world)
     # replicas: every rank streams a whole model per step (weak scaling);
     # split: the ranks stream one model between them (strong scaling)
