@@ -412,7 +412,9 @@ def small_batch_sweep(bl, device="cuda"):
     """Config 3's timing: M in {1, 2, 4, 8, 16} on the four 2.4B shapes.
     `us` / `GBps` / `path` are what linear() runs (the library's routing); from
     2 tokens the two small-batch kernels are timed side by side (`tensor_us`,
-    `dp4a_us`) and from 8 tokens also quantise + GEMM (`gemm_us`)."""
+    `dp4a_us`) and from 8 tokens also quantise + GEMM (`gemm_us`); `pdl_us` is
+    what linear() runs with consecutive launches overlapping through
+    programmatic dependent launch, as consecutive layers of a decode step do."""
     out = []
     for (K, N) in si.DECODE_SHAPES_2B:
         nbytes = bl.packed_bytes(N, K)
@@ -424,6 +426,8 @@ def small_batch_sweep(bl, device="cuda"):
                                                small_batch="tensor", ws=ws)["us"]
                 r["dp4a_us"] = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=True,
                                              small_batch="dp4a", ws=ws)["us"]
+                r["pdl_us"] = isolated_gemv(bl, K, N, M=m, iters=100, device=device, pdl=True,
+                                            ws=ws)["us"]
             if m >= 8:
                 r["gemm_us"] = isolated_gemv(bl, K, N, M=m, iters=100, device=device, force_fused=False,
                                              ws=ws)["us"]

@@ -467,8 +467,8 @@ def test_pdl_dependent_chain(bl, K, M):
     """A chain where each launch reads the previous launch's output, all with
     BL_FLAG_PDL, inside a CUDA graph (so that consecutive launches really
     overlap): the result must equal the oracle chain.  One token at K = 2560
-    runs small streaming launches, three tokens the per-warp-ring kernel, one
-    token at K = 8192 large streaming launches (two CTAs per SM)."""
+    runs small streaming launches, three tokens the multi-token streaming
+    kernel, one token at K = 8192 large streaming launches (two CTAs per SM)."""
     Ws = [si.weight(K, K, seed=70 + i) for i in range(6)]
     oracles = [oracle_weight(W) for W in Ws]
     ws = [_pack_gpu(bl, W) for W in Ws]
@@ -573,8 +573,9 @@ def test_small_batch_streaming_kernel(bl, M, K, Ns):
 
 
 def test_small_batch_pdl_chain_in_graph(bl):
-    """Eight tokens through a six-deep dependent chain of streaming launches
-    with programmatic dependent launch inside a CUDA graph."""
+    """Eight tokens through a six-deep dependent chain of launches (the
+    tensor-core small-batch GEMV at this size) with programmatic dependent
+    launch inside a CUDA graph."""
     K, M = 2560, 8
     Ws = [si.weight(K, K, seed=170 + i) for i in range(6)]
     oracles = [oracle_weight(W) for W in Ws]
