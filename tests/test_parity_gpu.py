@@ -11,8 +11,8 @@ import torch
 
 import oracle
 import synth_inputs as si
-from parity_helpers import (Guarded, assert_rel, bf16_bits_of, compare_outputs, dev,
-                            f32_bits, oracle_weight, seeded_problem)
+from parity_helpers import (Guarded, compare_outputs, dev, f32_bits, oracle_weight,
+                            seeded_problem)
 
 pytestmark = pytest.mark.gpu
 
